@@ -1,0 +1,268 @@
+/*
+ * sfx.h -- C ABI of the B200 (sm_100a) activation-sparse GEMV / FFN library.
+ *
+ * The library computes input-activation-sparse products for decoding at batch
+ * 1..16: input activations are masked by magnitude (|x| > t) or by top-k of a
+ * per-neuron score, the active neurons are compacted, and only the weight rows
+ * of active neurons are read from HBM.
+ *
+ * Sources (by page title and section):
+ *  [TEAL]  "TEAL: Training-Free Activation Sparsity in Large Language Models"
+ *          (reading-group slides), slide 8 (threshold t_p from calibration
+ *          data for a target sparsity), slide 11 ("Hardware-Aware
+ *          Acceleration": mask generation fused into the sparse GEMV so only
+ *          the needed weights are read).
+ *  [ATTR]  "Attribution-based Sparse Activation in Large Language Models",
+ *          sections "proposed method" (GxO score) and "implementation" (top
+ *          fraction per layer).
+ *  [GLASS] "GLASS: Global-Local Aggregation for inference-time
+ *          Sparsification", section 2.2 (rank aggregation, top-k selection).
+ *  [GLOSS] "Activation sparsity (LLM)" glossary, "why sparsity reduces
+ *          computation" (a zero intermediate skips one row of W2).
+ *  [MOE]   "Uncovering Intra-expert Activation Sparsity for Efficient
+ *          Mixture-of-Expert Model Execution", section "method".
+ *
+ * Conventions for every entry point
+ *  - Pointers marked (dev) are CUDA device pointers, (host) are host pointers.
+ *    The caller allocates and owns every buffer, including the workspace;
+ *    the library never allocates or frees memory.
+ *  - Weights are stored row-per-input-neuron: W is [K x N] row-major, so
+ *    y = x W and dropping input neuron i skips the contiguous row i ([GLOSS]).
+ *    Activations are [B x K] row-major, outputs [B x N] row-major.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = legacy default stream) unless stated otherwise.
+ *  - Return value: SFX_OK (0) or a negative sfx_status. Arguments are checked
+ *    on the host before any launch; a rejected call launches nothing.
+ *  - Device-side checks (an index outside [0, K) in a caller-provided list)
+ *    never trap: the offending row is skipped and a bit is OR-ed into the
+ *    status word at the start of the workspace. sfx_check_device_status()
+ *    reads (and clears) it.
+ *  - Alignment: weight matrices must be 16-byte aligned and their row length
+ *    a multiple of 8 elements, because weight rows are moved with 16-byte
+ *    bulk copies and read with 128-bit loads; otherwise SFX_ERR_ALIGN.
+ *  - Workspace: size it with sfx_workspace_bytes() and zero it once with
+ *    sfx_workspace_init() before first use; the library leaves it in a
+ *    reusable state after every successful call. Calls that share a workspace
+ *    must not run concurrently.
+ */
+#ifndef SFX_H_
+#define SFX_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { SFX_F16 = 0, SFX_BF16 = 1, SFX_F32 = 2 } sfx_dtype;
+
+typedef enum {
+  SFX_SEL_THRESHOLD = 0,   /* m_i = 1[|x_i| > t]                         [TEAL] */
+  SFX_SEL_TOPK_GXO = 1,    /* top-k of s_i = |fl32(x_i * g_i)|            [ATTR] */
+  SFX_SEL_TOPK_GLASS = 2   /* top-k of (1-l) R^l_i + l R^g_i             [GLASS] */
+} sfx_select;
+
+typedef enum {
+  SFX_OK = 0,
+  SFX_ERR_ARG = -1,          /* null pointer, bad size, k > n, ...          */
+  SFX_ERR_DTYPE = -2,        /* dtype not supported by this entry point     */
+  SFX_ERR_ALIGN = -3,        /* pointer or row stride not 16-byte aligned   */
+  SFX_ERR_WORKSPACE = -4,    /* workspace missing or smaller than required  */
+  SFX_ERR_CUDA = -5,         /* a CUDA runtime call or launch failed        */
+  SFX_ERR_DEVICE = -6,       /* device status word has a bit set            */
+  SFX_ERR_UNSUPPORTED = -7   /* shape outside the implemented range         */
+} sfx_status;
+
+/* Device status bits (OR-ed into the first word of the workspace). */
+#define SFX_DEV_BAD_INDEX   0x1u   /* caller index list held an index >= K   */
+#define SFX_DEV_TIMEOUT     0x2u   /* a bounded wait gave up                 */
+
+/* Flags for sfx_sparse_gemv / sfx_sparse_ffn_swiglu / sfx_moe_expert_sparse. */
+#define SFX_FLAG_GELU        0x1   /* epilogue y = GeLU(acc), erf form        */
+#define SFX_FLAG_GELU_TANH   0x2   /* epilogue y = GeLU(acc), tanh form       */
+#define SFX_FLAG_UNION_MASK  0x4   /* B>1: every token uses the batch union   */
+#define SFX_FLAG_NO_RENORM   0x8   /* MoE: keep raw top-k softmax weights     */
+#define SFX_FLAG_CUDA_CORES  0x10  /* B>1: force the CUDA-core kernel         */
+#define SFX_FLAG_SWIGLU      0x20  /* gemv: W columns interleave gate|up;
+                                      y = SiLU(g) * u as fp32 [B x N/2]       */
+
+/* Operation ids for sfx_workspace_bytes(). */
+typedef enum {
+  SFX_OP_CALIBRATE = 0,
+  SFX_OP_MASK_COMPACT = 1,
+  SFX_OP_SPARSE_GEMV = 2,
+  SFX_OP_FFN_SWIGLU = 3,
+  SFX_OP_MOE = 4
+} sfx_op;
+
+/* Bytes of workspace an operation needs (>= 256: the status header).
+ *  CALIBRATE:     a = S (draws), b = K, c = P (number of sparsities), d = dtype
+ *  MASK_COMPACT:  a = B, b = K (n), c = sfx_select,   d = unused
+ *  SPARSE_GEMV:   a = B, b = K,     c = N,            d = dtype of x
+ *  FFN_SWIGLU:    a = B, b = d,     c = ffn,          d = unused
+ *  MOE:           a = B, b = d,     c = E,            d = ffn (expert), e = top_k,
+ *                 f = ffn_shared
+ * Returns 0 for an unknown op or invalid sizes. */
+size_t sfx_workspace_bytes(int op, long long a, long long b, long long c, long long d,
+                           long long e, long long f);
+
+/* Zero `ws_bytes` bytes of a workspace (cudaMemsetAsync on `stream`). */
+int sfx_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Human-readable name of a status code (static string). */
+const char* sfx_status_string(int status);
+
+/* Synchronise `stream`, read and clear the device status word of `ws`.
+ * Returns SFX_OK if it was 0, SFX_ERR_DEVICE otherwise (*bits_out, if not
+ * NULL, receives the bits). */
+int sfx_check_device_status(void* ws, unsigned int* bits_out, void* stream);
+
+/* Number of SMs of the current device and the library's build target. */
+int sfx_device_sm_count(void);
+const char* sfx_build_info(void);
+
+/* ------------------------------------------------------------------------
+ * a1. Threshold calibration                                 [TEAL] slide 8
+ *
+ * For each target sparsity p_j, t_j is the lower empirical p_j-quantile of the
+ * pooled magnitudes |calib| (S draws x K activations): with the sorted
+ * magnitudes a_(1) <= ... <= a_(S K), t_j = a_(r) where r = ceil(p_j S K)
+ * (a product within 1e-9 S K of an integer counts as that integer); p_j <= 0
+ * gives t_j = -INFINITY (keep all). t_j is therefore a value of the input
+ * dtype and the strict mask |x| > t_j zeroes at least p_j of the calibration
+ * activations. Selection is exact (radix histogram of the magnitude bits).
+ *
+ *  calib          (dev)  [S x K] values of dtype dt (f16, bf16 or f32)
+ *  sparsities     (host) [P] in [0, 1], double
+ *  thresholds_out (host) [P] float
+ *  ws             (dev)  sfx_workspace_bytes(SFX_OP_CALIBRATE, S, K, P, dt)
+ * Synchronises `stream` (the thresholds are returned on the host).
+ * ---------------------------------------------------------------------- */
+int sfx_calibrate_thresholds(const void* calib, int dt, long long S, long long K,
+                             const double* sparsities, int P, float* thresholds_out,
+                             void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * a2-a4. Mask and compaction         [TEAL] slide 11, [ATTR], [GLASS] 2.2
+ *
+ * Per token b (row of x), builds the mask m_b over n = K neurons and its
+ * ascending index list:
+ *  THRESHOLD:   m_bi = 1[|x_bi| > t]                         (uses x, t)
+ *  TOPK_GXO:    keep the k largest s_bi = |fl32(x_bi * g_bi)|, x of dtype dt,
+ *               g = score_l (f32 [B x K]); equal scores go to the lower index
+ *  TOPK_GLASS:  R^l, R^g = ranks of score_l / score_g (f32 [B x K]) with the
+ *               most important neuron ranked n (score descending, then index
+ *               ascending); F = (1-lambda) R^l + lambda R^g in double; keep
+ *               the k largest F, ties to the lower index. x is unused.
+ *
+ *  x          (dev)  [B x K] of dtype dt (f16, bf16, f32); may be NULL for GLASS
+ *  bitmap     (dev)  [B x ceil(K/32)] uint32, bit (i % 32) of word i/32 = m_bi;
+ *                    may be NULL
+ *  idx        (dev)  [B x K] int32: row b holds cnt[b] ascending indices,
+ *                    the rest is left untouched; may be NULL
+ *  cnt        (dev)  [B] int32 active counts (required)
+ *  union_idx  (dev)  [K] int32 ascending indices of OR_b m_b; may be NULL
+ *  union_cnt  (dev)  [1] int32; required when union_idx is given
+ * Limits: 1 <= B <= 64; K <= 32768 for the top-k modes; 0 <= k <= K.
+ * ---------------------------------------------------------------------- */
+int sfx_mask_compact(const void* x, int dt, int B, int K, int sel, float t, int k,
+                     const float* score_l, const float* score_g, double lambda,
+                     uint32_t* bitmap, int32_t* idx, int32_t* cnt,
+                     int32_t* union_idx, int32_t* union_cnt,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * a5/a7. Input-sparse GEMV / skinny GEMM       [TEAL] slide 11, [GLOSS]
+ *
+ * y[b, n] = sum_{i active for b} x[b, i] * W[i, n], accumulated in fp32,
+ * reading only rows of W that some token of the batch needs.
+ *  - idx == NULL: the mask is built inside the kernel (fused, never stored):
+ *    token b keeps row i iff |x[b, i]| > t (t = -INFINITY: dense). Rows are
+ *    fetched once for the batch (the union) and each token applies its own
+ *    mask, unless SFX_FLAG_UNION_MASK makes every token use the union.
+ *  - idx != NULL (B must be 1): the active rows are idx[0 .. *cnt-1]
+ *    (device count), e.g. from sfx_mask_compact's top-k modes.
+ * Epilogue: SFX_FLAG_GELU / SFX_FLAG_GELU_TANH apply GeLU to y;
+ * SFX_FLAG_SWIGLU treats columns (2j, 2j+1) as (gate_j, up_j) and writes
+ * h_j = SiLU(gate_j) * up_j to y as fp32 [B x N/2] (ydt must be SFX_F32) --
+ * the first stage of sfx_sparse_ffn_swiglu on its own.
+ *
+ *  x        (dev)  [B x K] of dtype xdt (f16, bf16, f32); xdt == wdt or f32
+ *  W        (dev)  [K x N] of dtype wdt (f16, bf16), row-major, 16-byte aligned
+ *  y        (dev)  [B x N] of dtype ydt (f16, bf16, f32)
+ *  bitmap_out (dev, optional) [B x ceil(K/32)] receives the fused mask
+ *  ws       (dev)  sfx_workspace_bytes(SFX_OP_SPARSE_GEMV, B, K, N, xdt)
+ * Limits: 1 <= B <= 16, K >= 1, N >= 8 and N % 8 == 0.
+ * ---------------------------------------------------------------------- */
+int sfx_sparse_gemv(const void* x, int xdt, int B, int K, const void* W, int wdt, int N,
+                    float t, const int32_t* idx, const int32_t* cnt,
+                    void* y, int ydt, int flags, uint32_t* bitmap_out,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * a6. Activation-sparse SwiGLU FFN            [TEAL] slides 6 and 8
+ *
+ * m_x = |x| > t_in; [g | u] = (x m_x) [W_g | W_u]; h = SiLU(g) * u (fp32,
+ * never rounded to the weight dtype); m_h = |h| > t_h; y = (h m_h) W_d.
+ * Both products read only the rows of active neurons.
+ *
+ *  x      (dev) [B x d] of dtype dt (f16 or bf16)
+ *  W_gu   (dev) [d x 2 ffn] of dtype dt: row i interleaves gate and up,
+ *               W_gu[i, 2j] = W_g[i, j], W_gu[i, 2j+1] = W_u[i, j]
+ *               (build it once with sfx_pack_gate_up)
+ *  W_d    (dev) [ffn x d] of dtype dt
+ *  y      (dev) [B x d] of dtype ydt
+ *  h_out  (dev, optional) [B x ffn] fp32 receives h (before the m_h mask)
+ *  bitmap_x_out (dev, optional) [B x ceil(d/32)], bitmap_h_out (dev,
+ *               optional) [B x ceil(ffn/32)] receive the two fused masks
+ *  ws     (dev) sfx_workspace_bytes(SFX_OP_FFN_SWIGLU, B, d, ffn, dt)
+ * Limits: 1 <= B <= 16; d % 8 == 0; ffn % 4 == 0.
+ * ---------------------------------------------------------------------- */
+int sfx_sparse_ffn_swiglu(const void* x, int dt, int B, int d, int ffn,
+                          const void* W_gu, const void* W_d, float t_in, float t_h,
+                          void* y, int ydt, float* h_out, uint32_t* bitmap_x_out,
+                          uint32_t* bitmap_h_out, int flags,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Interleave W_g [d x ffn] and W_u [d x ffn] (dtype dt) into W_gu [d x 2 ffn]
+ * (layout preparation, done once per weight set). */
+int sfx_pack_gate_up(const void* W_g, const void* W_u, int dt, int d, int ffn,
+                     void* W_gu, void* stream);
+
+/* ------------------------------------------------------------------------
+ * a8. MoE layer with intra-expert activation sparsity             [MOE]
+ *
+ * Per token t: p = softmax(logits[t]) over E experts; the top_k experts by p
+ * (ties to the lower index) with weights w = p / sum(p_selected)
+ * (SFX_FLAG_NO_RENORM: raw p). For each selected expert e:
+ *   a = SiLU(x_t W_g[e])            (dense gate projection)
+ *   m_j = |a_j| > t_e[e]            (one threshold pass)
+ *   y_t += w_e * sum_{j: m_j} a_j (W_upT[e][j, :] . x_t) W_d[e][j, :]
+ * reading only rows j of W_upT[e] and W_d[e] with m_j = 1. If Ws_gu is not
+ * NULL, a dense shared SwiGLU expert (always on) is added:
+ * y_t += SwiGLU(x_t; Ws_gu [d x 2 ffn_shared] interleaved, Ws_d [ffn_shared x d]).
+ *
+ *  x       (dev) [B x d] dtype dt (bf16 or f16)
+ *  logits  (dev) [B x E] f32
+ *  W_g     (dev) [E x d x ffn]   W_upT (dev) [E x ffn x d]   W_d (dev) [E x ffn x d]
+ *  t_e     (dev) [E] f32 per-expert thresholds (-INFINITY: dense expert)
+ *  y       (dev) [B x d] dtype ydt
+ *  a_out   (dev, optional) [B x top_k x ffn] f32 gate activations a, in each
+ *          token's selection order; sel_out (dev, optional) [B x top_k] int32
+ *          selected experts
+ *  ws      (dev) sfx_workspace_bytes(SFX_OP_MOE, B, d, E, ffn, top_k, ffn_shared)
+ * Limits: 1 <= B <= 64, 1 <= top_k <= E <= 1024, d % 8 == 0, ffn % 8 == 0.
+ * ---------------------------------------------------------------------- */
+int sfx_moe_expert_sparse(const void* x, int dt, const float* logits, int B, int d, int E,
+                          int ffn, int top_k, const void* W_g, const void* W_upT,
+                          const void* W_d, const float* t_e, const void* Ws_gu,
+                          const void* Ws_d, int ffn_shared, void* y, int ydt,
+                          float* a_out, int32_t* sel_out, int flags,
+                          void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SFX_H_ */

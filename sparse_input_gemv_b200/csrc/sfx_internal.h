@@ -1,0 +1,87 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "sfx.h"
+
+namespace sfx {
+
+// Every workspace starts with a header: the device status word (bytes 0..3),
+// then, at byte 256, the split-K arrival counters. The counters are used by
+// the GEMV kernels only and are always left at zero, so no other operation may
+// use the header as scratch; operation-specific scratch starts after it.
+constexpr size_t kWsStatusBytes = 256;
+constexpr int kCounterSlots = 4096;  // max column tiles of one GEMV launch
+constexpr size_t kWsHeader = kWsStatusBytes + kCounterSlots * 4;
+
+enum Epi { EPI_NONE = 0, EPI_GELU = 1, EPI_GELU_TANH = 2, EPI_SWIGLU = 3 };
+
+// Arguments of one input-sparse GEMV launch (device pointers).
+struct GemvArgs {
+  const void* x;          // [B x K] activations, dtype xdt
+  const void* W;          // [K x N] weights, dtype wdt
+  void* y;                // [B x N] (or [B x N/2] fp32 h for EPI_SWIGLU)
+  const int32_t* idx;     // optional active list (B == 1)
+  const int32_t* cnt;     // device count of idx
+  uint32_t* bitmap_out;   // optional fused-mask output [B x ceil(K/32)]
+  float* partials;        // [S x B x N] split-K partial sums (workspace)
+  int32_t* counters;      // [col_tiles] arrival counters (workspace, zero between calls)
+  unsigned* status;       // device status word (workspace)
+  long long K, N;
+  int B;
+  int S;                  // number of K splits
+  int slice;              // rows of K per split (threshold mode), multiple of 32
+  int list_cap;           // capacity of the per-CTA active list
+  int nstage;             // bulk-copy ring depth (16 KB per stage)
+  int ydt;                // output dtype (ignored for EPI_SWIGLU: fp32)
+  int epi;                // Epi
+  int union_mask;         // every token uses the batch-union mask
+  float t;                // magnitude threshold (threshold mode)
+};
+
+struct GemvPlan {
+  int NT = 0;        // columns per CTA tile
+  int BMAX = 1;      // batch slots compiled into the kernel
+  int S = 1;         // K splits
+  int slice = 0;     // rows per split
+  int list_cap = 0;
+  int nstage = 0;
+  int col_tiles = 0;
+  size_t smem = 0;
+};
+
+int sm_count();
+GemvPlan plan_gemv(long long K, long long N, int B, bool idx_mode);
+size_t gemv_workspace_bytes(long long K, long long N, int B);  // excludes the header
+int launch_sparse_gemv(int wdt, int xdt, const GemvPlan& plan, GemvArgs a, cudaStream_t stream,
+                       bool pdl);
+
+// mask / selection kernels (sfx_mask.cu)
+size_t mask_workspace_bytes(int B, int K, int sel);
+int launch_mask_compact(const void* x, int dt, int B, int K, int sel, float t, int k,
+                        const float* score_l, const float* score_g, double lambda,
+                        uint32_t* bitmap, int32_t* idx, int32_t* cnt, int32_t* union_idx,
+                        int32_t* union_cnt, unsigned char* ws_body, unsigned* status,
+                        cudaStream_t stream);
+
+// calibration (sfx_calib.cu)
+size_t calib_workspace_bytes(long long S, long long K, int P, int dt);
+int run_calibrate(const void* calib, int dt, long long n, const long long* ranks, int P,
+                  float* thresholds_out_host, unsigned char* ws_body, cudaStream_t stream);
+
+// MoE (sfx_moe.cu)
+size_t moe_workspace_bytes(int B, int d, int E, int ffn, int top_k, int ffn_shared);
+int run_moe(const void* x, int dt, const float* logits, int B, int d, int E, int ffn, int top_k,
+            const void* W_g, const void* W_upT, const void* W_d, const float* t_e,
+            const void* Ws_gu, const void* Ws_d, int ffn_shared, void* y, int ydt,
+            float* a_out, int32_t* sel_out, int flags, unsigned char* ws_body, size_t body_bytes,
+            unsigned* status, cudaStream_t stream);
+
+// gate/up interleave (sfx_api.cu)
+int launch_pack_gate_up(const void* W_g, const void* W_u, int dt, int d, int ffn, void* W_gu,
+                        cudaStream_t stream);
+
+}  // namespace sfx

@@ -1,0 +1,319 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 CPU oracle.
+
+Masks, index lists, counts and calibrated thresholds are compared bit for bit;
+floating-point outputs within rel-L2 <= 1e-3 and max-abs <= 1e-2 max|y| of the
+oracle rounded to the output dtype. Inputs come from the seeded generators in
+sparse_input_gemv_b200.synth (Laplace activations, N(0, 0.02^2) weights).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from helpers import assert_close, pack_bitmap, to64
+from sparse_input_gemv_b200 import binding as sb
+from sparse_input_gemv_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+DT = {"f16": torch.float16, "bf16": torch.bfloat16, "f32": torch.float32}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    sb.load()
+    yield
+    ws = sb.default_workspace()
+    if ws.buf is not None:
+        assert ws.status() == 0, "device status word raised"
+
+
+def dev(t):
+    return t.to("cuda").contiguous()
+
+
+def weights(K, N, seed_name, dtype, device="cpu"):
+    return synth.normal((K, N), synth.seed_of(seed_name, "W"), 0.02, dtype, device=device)
+
+
+# ---------------------------------------------------------------- calibration
+
+@pytest.mark.parametrize("dtype,S,K,ps", [
+    ("f16", 64, 256, [0.5]),                                  # single input-sparse GEMV workload
+    ("bf16", 64, 4096, [0.25, 0.40, 0.50, 0.65]),             # Llama-3-8B block inputs
+    ("bf16", 16, 1000, [0.0, 0.1, 0.7, 0.9, 1.0]),            # ragged K, p = 0 and p = 1
+    ("f32", 64, 768, [0.5, 0.8, 0.9]),                        # fp32 activations (3 radix passes)
+])
+def test_calibration_bit_exact(dtype, S, K, ps):
+    calib = synth.calib_draws("calib-test", f"{dtype}-{K}", S, K, dtype)
+    t_gpu = sb.sfx_calibrate_thresholds(dev(calib), ps)
+    a = to64(calib)
+    for p, tg in zip(ps, t_gpu):
+        assert tg == O.calibrate_threshold(a, p), (p, tg)
+        if p > 0:
+            frac = np.mean(~O.magnitude_mask(a, tg))
+            assert frac >= p - 1e-12
+
+
+def test_calibration_heavy_ties_f32():
+    # values on a coarse grid: the order statistic sits inside long runs of ties
+    x = torch.from_numpy(np.round(np.random.default_rng(0).laplace(size=(32, 500)) * 4) / 4)
+    x = x.to(torch.float32)
+    ps = [0.3, 0.55, 0.95]
+    t = sb.sfx_calibrate_thresholds(dev(x), ps)
+    for p, tg in zip(ps, t):
+        assert tg == O.calibrate_threshold(to64(x), p)
+
+
+# ---------------------------------------------------------------- mask / compaction
+
+def test_teal_worked_example_on_gpu(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "teal_worked_example.json")))
+    for dtype in ("f32", "f16"):
+        x = torch.tensor([g["x"]], dtype=DT[dtype])
+        out = sb.sfx_mask_compact(dev(x), sb.SFX_SEL_THRESHOLD, t=g["threshold"])
+        c = int(out["cnt"][0])
+        assert c == 2 and out["idx"][0, :c].tolist() == g["active_idx"]
+        assert out["bitmap"][0, 0].item() == 0b01010
+    # and through the fused GEMV: y = sparse_x W on the stored (fp16) values
+    W = weights(5, 8, "worked", "f16")
+    x = torch.tensor(g["x"], dtype=torch.float16)
+    y, bm = sb.sfx_sparse_gemv(dev(x), dev(W), t=g["threshold"], out_dtype=torch.float32,
+                               want_bitmap=True)
+    assert bm[0, 0].item() == 0b01010
+    sparse_x = to64(x) * np.array(g["mask"])
+    assert_close(to64(y), O.round_to(sparse_x @ to64(W), "f32"), "worked")
+
+
+@pytest.mark.parametrize("dtype,B,K,t", [("bf16", 1, 4096, 0.69), ("f16", 4, 1000, 1.0),
+                                         ("f32", 16, 14336, 0.3), ("bf16", 3, 33, 0.5)])
+def test_threshold_mask_compact_bit_exact(dtype, B, K, t):
+    x = synth.eval_draw("mask-test", f"{dtype}{K}", B, K, dtype)
+    out = sb.sfx_mask_compact(dev(x), sb.SFX_SEL_THRESHOLD, t=t, want_union=True)
+    m = O.magnitude_mask(to64(x), t)
+    assert np.array_equal(out["bitmap"].cpu().numpy(), pack_bitmap(m))
+    for b in range(B):
+        idx, c = O.compact(m[b])
+        assert int(out["cnt"][b]) == c
+        assert np.array_equal(out["idx"][b, :c].cpu().numpy(), idx)
+    uidx, uc = O.compact(O.union_mask(m))
+    assert int(out["union_cnt"][0]) == uc
+    assert np.array_equal(out["union_idx"][:uc].cpu().numpy(), uidx)
+
+
+@pytest.mark.parametrize("K,keep", [(10240, 0.3), (10240, 0.5), (10240, 0.7), (1000, 0.5), (37, 1.0)])
+def test_topk_gxo_bit_exact(K, keep):
+    h = synth.normal((1, K), synth.seed_of("gxo", K, "h"), 1.0, "f32")
+    g = synth.normal((1, K), synth.seed_of("gxo", K, "g"), 1.0, "f32")
+    k = O.keep_count(keep, K)
+    out = sb.sfx_mask_compact(dev(h), sb.SFX_SEL_TOPK_GXO, k=k, score_l=dev(g))
+    m = O.topk_mask(O.gxo_score(h.numpy()[0], g.numpy()[0]), k)
+    assert int(out["cnt"][0]) == k
+    assert np.array_equal(out["idx"][0, :k].cpu().numpy(), O.compact(m)[0])
+    assert np.array_equal(out["bitmap"].cpu().numpy(), pack_bitmap(m[None]))
+
+
+def test_topk_gxo_ties_go_to_lower_index():
+    K = 3000
+    rng = np.random.default_rng(5)
+    h = torch.from_numpy(rng.integers(0, 5, size=(2, K)).astype(np.float32))  # heavy ties
+    g = torch.ones((2, K), dtype=torch.float32)
+    for k in (0, 1, 17, 1500, 2999, 3000):
+        out = sb.sfx_mask_compact(dev(h), sb.SFX_SEL_TOPK_GXO, k=k, score_l=dev(g))
+        for b in range(2):
+            m = O.topk_mask(O.gxo_score(g.numpy()[b], h.numpy()[b]), k)
+            assert int(out["cnt"][b]) == k
+            assert np.array_equal(out["idx"][b, :k].cpu().numpy(), O.compact(m)[0]), (k, b)
+
+
+@pytest.mark.parametrize("lam,K,keep", [(0.5, 10240, 0.5), (0.0, 2000, 0.3), (1.0, 2000, 0.7),
+                                        (0.3, 999, 0.5)])
+def test_glass_bit_exact(lam, K, keep):
+    sl = synth.abs_normal((1, K), synth.seed_of("glass", K, "local"))
+    sg = synth.abs_normal((1, K), synth.seed_of("glass", K, "global"))
+    k = O.keep_count(keep, K)
+    out = sb.sfx_mask_compact(None, sb.SFX_SEL_TOPK_GLASS, k=k, score_l=dev(sl), score_g=dev(sg),
+                              lam=lam)
+    m = O.glass_mask(sl.numpy()[0], sg.numpy()[0], lam, k)
+    assert int(out["cnt"][0]) == k
+    assert np.array_equal(out["idx"][0, :k].cpu().numpy(), O.compact(m)[0])
+
+
+# ---------------------------------------------------------------- sparse GEMV
+
+def gemv_case(B, K, N, p, wdt="bf16", xdt=None, seed="gemv", flags=0, out="bf16"):
+    xdt = xdt or wdt
+    calib = synth.calib_draws(seed, f"in{K}", 64, K, xdt)
+    t = O.calibrate_threshold(to64(calib), p) if p > 0 else -math.inf
+    x = synth.eval_draw(seed, f"in{K}", B, K, xdt)
+    W = weights(K, N, f"{seed}{K}x{N}", wdt)
+    y, bm = sb.sfx_sparse_gemv(dev(x), dev(W), t=t, out_dtype=DT[out], flags=flags,
+                               want_bitmap=True)
+    m = O.magnitude_mask(to64(x), t)
+    assert np.array_equal(bm.cpu().numpy(), pack_bitmap(m)), "fused mask differs"
+    want = O.masked_gemv(to64(x), m, to64(W))
+    if flags & sb.SFX_FLAG_GELU:
+        want = O.gelu_erf(want)
+    assert_close(to64(y), O.round_to(want, out), f"B={B} K={K} N={N} p={p}")
+    return y
+
+
+def test_single_input_sparse_gemv_workload():
+    # x fp16 [1 x 256] ~ Laplace, W fp16 [256 x 512] ~ N(0, 0.02^2), t_p for 50%
+    gemv_case(1, 256, 512, 0.5, "f16", out="f16")
+    gemv_case(1, 256, 512, 0.5, "f16", out="f32")
+
+
+@pytest.mark.parametrize("K,N,p", [(4096, 6144, 0.5), (4096, 4096, 0.25), (14336, 4096, 0.65),
+                                   (4096, 28672, 0.4), (1000, 264, 0.5), (33, 8, 0.5),
+                                   (1, 64, 0.0), (5000, 2056, 0.9)])
+def test_gemv_b1_shapes(K, N, p):
+    gemv_case(1, K, N, p)
+
+
+def test_gemv_dense_and_empty_limits():
+    # p = 0: every row (dense GEMV); p = 1: no row, y = 0
+    gemv_case(1, 2048, 1024, 0.0)
+    x = synth.eval_draw("lim", "x", 1, 2048, "bf16")
+    W = weights(2048, 1024, "lim", "bf16")
+    t = float(x.abs().max())
+    y = sb.sfx_sparse_gemv(dev(x), dev(W), t=t)
+    assert torch.count_nonzero(y).item() == 0
+
+
+@pytest.mark.parametrize("B,p", [(2, 0.5), (4, 0.5), (8, 0.7), (16, 0.9), (16, 0.3)])
+def test_gemv_batch_union(B, p):
+    y = gemv_case(B, 4096, 2048, p, seed="union")
+    # each token's row equals its batch-1 result
+    x = synth.eval_draw("union", "in4096", B, 4096, "bf16")
+    calib = synth.calib_draws("union", "in4096", 64, 4096, "bf16")
+    t = O.calibrate_threshold(to64(calib), p)
+    W = dev(weights(4096, 2048, "union4096x2048", "bf16"))
+    for b in (0, B - 1):
+        y1 = sb.sfx_sparse_gemv(dev(x[b]), W, t=t)
+        assert_close(to64(y[b]), to64(y1), "batch vs single")
+
+
+def test_gemv_union_mask_flag():
+    B, K, N = 4, 1024, 512
+    x = synth.eval_draw("umask", "x", B, K, "bf16")
+    W = weights(K, N, "umask", "bf16")
+    t = 1.2
+    y = sb.sfx_sparse_gemv(dev(x), dev(W), t=t, flags=sb.SFX_FLAG_UNION_MASK,
+                           out_dtype=torch.float32)
+    u = O.union_mask(O.magnitude_mask(to64(x), t))
+    want = O.masked_gemv(to64(x), np.broadcast_to(u, (B, K)), to64(W))
+    assert_close(to64(y), O.round_to(want, "f32"), "union-mask reading")
+
+
+def test_gemv_fp16_and_fp32_inputs_and_gelu():
+    gemv_case(1, 2560, 10240, 0.0, "f16", out="f32", flags=sb.SFX_FLAG_GELU)
+    gemv_case(1, 3000, 1000, 0.5, "bf16", xdt="f32", out="f32")
+    gemv_case(2, 3000, 1000, 0.5, "f16", xdt="f32", out="f16")
+
+
+def test_gemv_index_list_mode():
+    K, N = 10240, 2560
+    h = synth.normal((K,), synth.seed_of("idx", "h"), 1.0, "f32")
+    g = synth.normal((K,), synth.seed_of("idx", "g"), 1.0, "f32")
+    W2 = weights(K, N, "idxW2", "f16")
+    k = O.keep_count(0.3, K)
+    sel = sb.sfx_mask_compact(dev(h), sb.SFX_SEL_TOPK_GXO, k=k, score_l=dev(g))
+    y = sb.sfx_sparse_gemv(dev(h), dev(W2), idx=sel["idx"][0], cnt=sel["cnt"],
+                           out_dtype=torch.float16)
+    want, m = O.ffn_gelu_topk_down(h.numpy(), g.numpy(), to64(W2), k)
+    assert_close(to64(y), O.round_to(want, "f16"), "top-k rows")
+
+
+def test_gemv_bad_index_is_skipped_and_flagged():
+    K, N = 512, 256
+    x = synth.eval_draw("bad", "x", 1, K, "bf16")[0]
+    W = weights(K, N, "bad", "bf16")
+    idx = torch.tensor([3, 7, K + 5, 100], dtype=torch.int32)
+    cnt = torch.tensor([4], dtype=torch.int32)
+    ws = sb.Workspace()
+    y = sb.sfx_sparse_gemv(dev(x), dev(W), idx=dev(idx), cnt=dev(cnt), out_dtype=torch.float32,
+                           ws=ws)
+    assert ws.status() == sb.SFX_DEV_BAD_INDEX
+    assert ws.status() == 0  # read-and-clear
+    m = np.zeros(K, bool)
+    m[[3, 7, 100]] = True
+    assert_close(to64(y), O.round_to(O.masked_gemv(to64(x), m, to64(W))[0], "f32"), "bad idx")
+
+
+# ---------------------------------------------------------------- SwiGLU FFN
+
+def ffn_case(B, d, ffn, p, dtype="bf16", seed="ffn"):
+    calib_x = synth.calib_draws(seed, f"x{d}", 64, d, dtype)
+    t_in = O.calibrate_threshold(to64(calib_x), p) if p > 0 else -math.inf
+    Wg = weights(d, ffn, f"{seed}-g", dtype, "cuda")
+    Wu = weights(d, ffn, f"{seed}-u", dtype, "cuda")
+    Wd = weights(ffn, d, f"{seed}-d", dtype, "cuda")
+    Wgu = sb.sfx_pack_gate_up(Wg, Wu)
+    Wg64, Wu64, Wd64 = to64(Wg), to64(Wu), to64(Wd)
+    # down-site threshold: the oracle's dense FFN h on 16 calibration draws
+    if p > 0:
+        _, hc, _, _ = O.ffn_swiglu(to64(calib_x[:16]), -math.inf, Wg64, Wu64, Wd64, -math.inf)
+        t_h = float(np.float32(O.calibrate_threshold(hc, p)))
+    else:
+        t_h = -math.inf
+    x = synth.eval_draw(seed, f"x{d}", B, d, dtype)
+    out = sb.sfx_sparse_ffn_swiglu(dev(x), Wgu, Wd, t_in, t_h, want_h=True, want_bitmaps=True)
+    y, h, m_x, m_h = O.ffn_swiglu(to64(x), t_in, Wg64, Wu64, Wd64, t_h)
+    # stage 1: exact input mask, h (fp32, unrounded) within tolerance
+    assert np.array_equal(out["bitmap_x"].cpu().numpy(), pack_bitmap(m_x))
+    assert_close(to64(out["h"]), O.round_to(h, "f32"), "h")
+    # stage 2: the fused |h| > t_h mask may differ from the fp64 one only where
+    # the fp32 and fp64 h straddle t_h, i.e. within rounding distance of t_h
+    got_mh = out["bitmap_h"].cpu().numpy()
+    want_mh = pack_bitmap(m_h)
+    flips = np.flatnonzero(np.unpackbits((got_mh ^ want_mh).view(np.uint8), bitorder="little"))
+    flips = flips[flips % (((ffn + 31) // 32) * 32) < ffn]
+    hb = np.abs(h).ravel()
+    for f in flips:
+        b, j = divmod(int(f), ((ffn + 31) // 32) * 32)
+        assert abs(abs(h[b, j]) - t_h) <= 1e-4 * hb.max(), (b, j, h[b, j], t_h)
+    assert flips.size <= max(2, ffn * B // 1000)
+    assert_close(to64(out["y"]), O.round_to(y, dtype), "y (end to end)")
+    return int(flips.size)
+
+
+def test_ffn_swiglu_small_ragged():
+    ffn_case(1, 512, 1796, 0.5)
+    ffn_case(3, 264, 1000, 0.4, "f16")
+
+
+@pytest.mark.parametrize("p", [0.25, 0.40, 0.50, 0.65])
+def test_ffn_swiglu_llama3_8b(p):
+    flips = ffn_case(1, 4096, 14336, p, seed="llama3-8b-ffn")
+    assert flips <= 2
+
+
+def test_ffn_swiglu_dense_equals_p0():
+    ffn_case(2, 1024, 2048, 0.0)
+
+
+def test_workspace_shared_across_operations():
+    # One workspace for every call: scratch written by calibration, GLASS and
+    # the FFN must never disturb the GEMV's split-K counters in the header.
+    ws = sb.Workspace()
+    K, N = 2048, 28672   # many column tiles
+    for rep in range(2):
+        sl = synth.abs_normal((1, 4096), synth.seed_of("ws", "l"))
+        sg = synth.abs_normal((1, 4096), synth.seed_of("ws", "g"))
+        sb.sfx_mask_compact(None, sb.SFX_SEL_TOPK_GLASS, k=1000, score_l=dev(sl),
+                            score_g=dev(sg), ws=ws)
+        calib = synth.calib_draws("ws", "c", 64, 768, "f32")
+        sb.sfx_calibrate_thresholds(dev(calib), [0.5], ws=ws)
+        x = synth.eval_draw("ws", "x", 1, K, "bf16")
+        W = weights(K, N, "ws", "bf16")
+        y = sb.sfx_sparse_gemv(dev(x), dev(W), t=0.7, out_dtype=torch.float32, ws=ws)
+        want = O.masked_gemv(to64(x), O.magnitude_mask(to64(x), 0.7), to64(W))
+        assert_close(to64(y), O.round_to(want, "f32"), f"gemv after other ops ({rep})")
+    assert ws.status() == 0
