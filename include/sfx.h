@@ -201,6 +201,36 @@ int sfx_sparse_gemv(const void* x, int xdt, int B, int K, const void* W, int wdt
                     void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * sfx_sparse_gemv without a workspace. The source pages have no counterpart:
+ * this entry point exists for callers, not for the method.
+ *
+ * Same computation, arguments and limits as sfx_sparse_gemv, minus the fused
+ * mask output and the workspace. It is for callers that cannot allocate
+ * device memory: a plugin behind a fixed C interface that is handed only its
+ * inputs and outputs, or code inside a framework that owns all device memory
+ * through its own pool and forbids side allocations (cudaMalloc would also
+ * synchronise the device in the middle of a latency-critical decode loop).
+ * The call's scratch (status word, split-K arrival counters, partial sums)
+ * lives in a 4 MiB file-scope device array inside the library instead; every
+ * GPU that loads the library holds that array until the process exits. The
+ * call allocates and frees nothing.
+ *  - Shapes whose partial sums do not fit in the array are rejected with
+ *    SFX_ERR_UNSUPPORTED before any launch.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current: make that first call
+ *    before any stream capture.
+ *  - Each call clears the status word and the arrival counters it uses on
+ *    `stream`, then launches. All calls share the one array and it keeps the
+ *    last call's contents, so calls that overlap on the GPU (other streams,
+ *    other host threads) race with each other; issue them one after another.
+ *  - Out-of-range list indices are skipped as in sfx_sparse_gemv, but their
+ *    status bit is not reported.
+ * ---------------------------------------------------------------------- */
+int sfx_sparse_gemv_noalloc(const void* x, int xdt, int B, int K, const void* W, int wdt, int N,
+                            float t, const int32_t* idx, const int32_t* cnt,
+                            void* y, int ydt, int flags, void* stream);
+
+/* ------------------------------------------------------------------------
  * a6. Activation-sparse SwiGLU FFN            [TEAL] slides 6 and 8
  *
  * m_x = |x| > t_in; [g | u] = (x m_x) [W_g | W_u]; h = SiLU(g) * u (fp32,

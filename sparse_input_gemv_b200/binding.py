@@ -43,6 +43,8 @@ _SIGS = {
                               _VP, _SZ, _VP]),
     "sfx_sparse_gemv": (_I, [_VP, _I, _I, _I, _VP, _I, _I, _F, _VP, _VP, _VP, _I, _I, _VP, _VP,
                              _SZ, _VP]),
+    "sfx_sparse_gemv_noalloc": (_I, [_VP, _I, _I, _I, _VP, _I, _I, _F, _VP, _VP, _VP, _I, _I,
+                                     _VP]),
     "sfx_sparse_ffn_swiglu": (_I, [_VP, _I, _I, _I, _I, _VP, _VP, _F, _F, _VP, _I, _VP, _VP, _VP,
                                    _I, _VP, _SZ, _VP]),
     "sfx_pack_gate_up": (_I, [_VP, _VP, _I, _I, _I, _VP, _VP]),
@@ -217,6 +219,30 @@ def sfx_sparse_gemv(x, W, t=-math.inf, idx=None, cnt=None, out_dtype=None, flags
         _ptr(y), _DT[y.dtype], int(flags), _ptr(bitmap), _ptr(buf), buf.numel(), _stream(stream)))
     y_out = y[0] if squeeze else y
     return (y_out, bitmap) if want_bitmap else y_out
+
+
+def sfx_sparse_gemv_noalloc(x, W, t=-math.inf, idx=None, cnt=None, out_dtype=None, flags=0,
+                            y=None, stream=None):
+    """sfx_sparse_gemv for callers that cannot allocate device memory.
+
+    The library keeps this call's scratch in a fixed 4 MiB device array of its
+    own, so only inputs and outputs are passed (``y`` may be preallocated by
+    the caller; if it is None this wrapper allocates it with torch, which the
+    C entry point itself never does). Calls must not overlap on the GPU.
+    """
+    squeeze = x.dim() == 1
+    x2 = x[None] if squeeze else x
+    _need_cuda(x2, W, idx, cnt)
+    B, K = x2.shape
+    N = W.shape[1]
+    out_dtype = torch.float32 if flags & SFX_FLAG_SWIGLU else (out_dtype or W.dtype)
+    if y is None:
+        y = torch.empty((B, N // 2 if flags & SFX_FLAG_SWIGLU else N), dtype=out_dtype,
+                        device=W.device)
+    _check("sfx_sparse_gemv_noalloc", load().sfx_sparse_gemv_noalloc(
+        _ptr(x2), _DT[x2.dtype], B, K, _ptr(W), _DT[W.dtype], N, float(t), _ptr(idx), _ptr(cnt),
+        _ptr(y), _DT[y.dtype], int(flags), _stream(stream)))
+    return y[0] if squeeze else y
 
 
 def sfx_pack_gate_up(W_g, W_u, stream=None):
