@@ -36,29 +36,40 @@ static int env_int(const char* name, int dflt) {
   return (s && *s) ? std::atoi(s) : dflt;
 }
 
-static constexpr size_t kSmemBudget = 200 * 1024;
 static constexpr size_t kListBudget = 48 * 1024;
 
 GemvPlan plan_gemv(long long K, long long N, int B, bool idx_mode) {
   GemvPlan p;
   p.BMAX = bmax_for(B);
-  const int sms = sm_count();
-  // Column tile: the widest tile that still leaves at least 4 K-splits'
-  // worth of CTAs to fill the SMs (wider segments = longer contiguous reads).
+  // resident CTAs: two per SM at batch 1 (64 registers per thread), one above
+  const int slots = sm_count() * (p.BMAX == 1 ? 2 : 1);
+  // Column tile: the first of 256, 512, 1024, 2048 columns whose tiles times
+  // K splits fill at least 90% of the resident slots in one wave; otherwise
+  // the best filling one. (Measured on B200 for the Llama-3-8B shapes:
+  // 256-column tiles win for N = 4096 / 6144, 512 for N = 28672.)
   int nt = 256;
-  for (int cand : {2048, 1024, 512, 256}) {
+  double best = -1.0;
+  for (int cand : {256, 512, 1024, 2048}) {
     const long long ct = (N + cand - 1) / cand;
-    if (ct * 4 <= sms || cand == 256) {
+    long long S = std::max<long long>(1, slots / ct);
+    S = std::min<long long>(S, std::max<long long>(1, (K + 31) / 32));
+    const long long ctas = ct * S;
+    const long long waves = (ctas + slots - 1) / slots;
+    const double util = (double)ctas / (double)(waves * slots);
+    if (util >= 0.9) {
       nt = cand;
       break;
+    }
+    if (util > best) {
+      best = util;
+      nt = cand;
     }
   }
   nt = env_int("SFX_GEMV_NT", nt);
   p.NT = nt;
   p.col_tiles = (int)((N + nt - 1) / nt);
-  // K splits: fill the SMs once, with at least 64 rows per split.
-  long long S = std::max<long long>(1, sms / p.col_tiles);
-  S = std::min<long long>(S, std::max<long long>(1, K / 64));
+  long long S = std::max<long long>(1, slots / p.col_tiles);
+  S = std::min<long long>(S, std::max<long long>(1, (K + 31) / 32));
   S = env_int("SFX_GEMV_S", (int)S);
   const size_t per_row = 4 * (size_t)(1 + p.BMAX);
   const long long cap_max = (long long)(kListBudget / per_row) / 32 * 32;
@@ -73,13 +84,11 @@ GemvPlan plan_gemv(long long K, long long N, int B, bool idx_mode) {
     p.list_cap = (int)round_up((K + S - 1) / S, 32);
   }
   p.S = (int)S;
-  const size_t list_bytes = (size_t)p.list_cap * per_row;
-  const size_t bar_bytes = 2 * 8 * 16;
-  int nstage = (int)((kSmemBudget - list_bytes - bar_bytes) / kStageBytes);
-  nstage = std::max(2, std::min(nstage, 8));
-  nstage = env_int("SFX_GEMV_STAGES", nstage);
-  p.nstage = nstage;
-  p.smem = (size_t)nstage * kStageBytes + list_bytes + 2 * 8 * (size_t)nstage;
+  // shared memory: warp-reduction buffer (warps x 256 floats) + list; the
+  // split-K tail reuses the front as 4 x NT floats
+  const size_t main_bytes =
+      (size_t)(gemv_threads(p.BMAX) / 32) * 256 * 4 + (size_t)p.list_cap * per_row;
+  p.smem = std::max(main_bytes, (size_t)16 * nt);
   return p;
 }
 
@@ -101,13 +110,16 @@ SFX_DECL(gemv_f16_f16_small) SFX_DECL(gemv_f16_f16_large)
 SFX_DECL(gemv_f16_f32_small) SFX_DECL(gemv_f16_f32_large)
 #undef SFX_DECL
 
-int launch_sparse_gemv(int wdt, int xdt, const GemvPlan& p, GemvArgs a, cudaStream_t s,
-                       bool pdl) {
+// Every launch is a programmatic dependent grid: the kernel waits
+// (griddepcontrol.wait) before it reads any input or workspace, so it is
+// correct after any predecessor, and its CTAs get scheduled while the
+// previous kernel finishes its tail.
+int launch_sparse_gemv(int wdt, int xdt, const GemvPlan& p, GemvArgs a, cudaStream_t s, bool) {
+  const bool pdl = true;
   if (p.col_tiles > kCounterSlots) return SFX_ERR_UNSUPPORTED;
   a.S = p.S;
   a.slice = p.slice;
   a.list_cap = p.list_cap;
-  a.nstage = p.nstage;
   const bool large = p.NT >= 1024;
   if (wdt == SFX_BF16) {
     if (xdt == SFX_BF16) return large ? gemv_bf16_bf16_large(p, a, s, pdl) : gemv_bf16_bf16_small(p, a, s, pdl);

@@ -6,21 +6,27 @@
 // and only the needed weights are loaded; "Activation sparsity (LLM)"
 // glossary: a zero input skips one weight row).
 //
-// Grid = (column tiles) x (K splits). Each CTA
+// Grid = (column tiles of NT columns) x (K splits), 512 threads, two CTAs per
+// SM for batch 1. Each CTA
 //   1. builds the active list of its K-slice in shared memory: |x| > t per
 //      token, warp ballots + popc + a block prefix give ascending positions
-//      (or it reads its share of a caller list in the top-k modes);
-//   2. streams the active rows' segments W[i, n0:n0+NT] into a ring of 16 KB
-//      shared-memory stages with 1-D bulk copies (TMA) issued by a producer
-//      warp, each stage guarded by a full/empty mbarrier pair, weights marked
-//      L2 evict-first;
-//   3. eight consumer warps read 128-bit words from the stages and accumulate
-//      x * w in fp32 registers;
-//   4. reduces across row groups in shared memory, then across K splits: each
-//      CTA writes its fp32 partial tile, and the last CTA to arrive at the
-//      tile's counter sums the S partials in split order (deterministic) and
-//      applies the epilogue (store, GeLU, or SiLU(g) * u for interleaved
-//      gate|up columns).
+//      (or it reads its share of a caller-provided list);
+//   2. streams the active rows' segments W[i, n0:n0+NT] with 128-bit loads
+//      that bypass L1 and carry an L2 evict-first policy: each warp owns one
+//      256-column chunk of the tile (32 lanes x 8 bf16/fp16) and keeps four
+//      rows in flight, so an SM holds ~64 KB of weight reads in flight,
+//      enough to cover HBM latency; products accumulate in fp32 registers;
+//   3. reduces the warps of each chunk in shared memory, then across K
+//      splits: every CTA writes its fp32 partial tile and the last CTA to
+//      arrive at the tile's counter sums the S partials in split order
+//      (deterministic; the sum is spread over all threads, four split groups
+//      at a time) and applies the epilogue (store, GeLU, or SiLU(g) * u for
+//      interleaved gate|up columns).
+//
+// Why plain loads rather than bulk (TMA) copies into a shared-memory ring: on
+// this GPU a CTA issues 1-D bulk copies at a few million per second, so the
+// 0.5-4 KB row segments of a sparse GEMV top out at 1-4 TB/s that way,
+// while 128-bit loads with enough rows in flight reach the HBM peak.
 #pragma once
 
 #include "sfx_common.cuh"
@@ -28,11 +34,10 @@
 
 namespace sfx {
 
-constexpr int kConsumerThreads = 256;
-constexpr int kProducerWarp = kConsumerThreads / 32;  // warp 8
-constexpr int kThreads = kConsumerThreads + 32;
-constexpr int kWarps = kThreads / 32;
-constexpr int kStageBytes = 16384;
+// 512 threads (two CTAs per SM) up to 4 batch slots; 256 threads with the
+// register room for 8 x BMAX accumulators above that.
+__host__ __device__ constexpr int gemv_threads(int bmax) { return bmax >= 8 ? 256 : 512; }
+constexpr int kRowsInFlight = 4;  // independent row loads per warp
 
 __device__ __forceinline__ float apply_epi(int epi, float v) {
   if (epi == EPI_GELU) return gelu_erf_f(v);
@@ -40,25 +45,34 @@ __device__ __forceinline__ float apply_epi(int epi, float v) {
   return v;
 }
 
-template <typename TW, typename TX, int NT, int BMAX>
-__global__ void __launch_bounds__(kThreads, 1) sparse_gemv_kernel(const GemvArgs a) {
-  constexpr int TPR = NT / 8;                 // threads per row segment (8 columns each)
-  constexpr int RG = kConsumerThreads / TPR;  // row groups working in parallel
-  constexpr int SR = kStageBytes / (NT * 2);  // rows per stage
-  constexpr int RPT = SR / RG;                // rows per thread per stage
-  static_assert(TPR <= kConsumerThreads && SR % RG == 0, "tile shape");
+// 16-byte weight load: skip L1, L2 evict-first (weights are read once).
+__device__ __forceinline__ uint4 ldg_stream(const void* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
 
-  extern __shared__ __align__(1024) unsigned char smem[];
-  unsigned char* stage_mem = smem;
-  int32_t* list_row = reinterpret_cast<int32_t*>(smem + (size_t)a.nstage * kStageBytes);
-  float* list_x = reinterpret_cast<float*>(list_row + a.list_cap);
-  uint64_t* full = reinterpret_cast<uint64_t*>(list_x + (size_t)a.list_cap * BMAX);
-  uint64_t* empty = full + a.nstage;
+template <typename TW, typename TX, int NT, int BMAX>
+__global__ void __launch_bounds__(gemv_threads(BMAX), (BMAX == 1) ? 2 : 1)
+    sparse_gemv_kernel(const GemvArgs a) {
+  constexpr int kThreads = gemv_threads(BMAX);
+  constexpr int kWarps = kThreads / 32;
+  constexpr int C = NT / 256;          // 256-column chunks per tile
+  constexpr int WPC = kWarps / C;      // warps per chunk
+  static_assert(NT % 256 == 0 && kWarps % C == 0, "tile shape");
+
+  // shared memory: [warp-reduction buffer, kWarps x 256 floats][active list:
+  // rows, x values]; the split-K tail reuses the front as 4 x NT floats
+  extern __shared__ __align__(16) unsigned char smem[];
+  float* red = reinterpret_cast<float*>(smem);                       // [WPC][NT] floats
+  int32_t* list_row = reinterpret_cast<int32_t*>(smem + (size_t)kWarps * 256 * 4);
+  float* list_x = reinterpret_cast<float*>(list_row + a.list_cap);   // [cap][BMAX]
 
   __shared__ int s_warp_tot[kWarps];
   __shared__ int s_count;
   __shared__ int s_last;
-  __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -68,14 +82,6 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_gemv_kernel(const GemvArgs
   const long long n0 = (long long)tile * NT;
   const int ncols = (int)min((long long)NT, a.N - n0);
 
-  if (tid == 0) {
-    for (int s = 0; s < a.nstage; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kConsumerThreads / 32);
-    }
-    fence_barrier_init();
-    s_abort = 0;
-  }
   // Inputs (x, caller lists) and the workspace may be written by the
   // previous kernel on the stream when launched as a dependent grid.
   pdl_wait();
@@ -86,9 +92,21 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_gemv_kernel(const GemvArgs
     const long long k1 = min(a.K, k0 + a.slice);
     const TX* xp = reinterpret_cast<const TX*>(a.x);
     int base = 0;
+    // x of the next chunk is loaded while the current chunk is compacted
+    float xnext[BMAX];
+#pragma unroll
+    for (int b = 0; b < BMAX; ++b)
+      xnext[b] = (b < a.B && k0 + tid < k1) ? to_f32(xp[(long long)b * a.K + k0 + tid]) : 0.f;
     for (long long c0 = k0; c0 < k1; c0 += kThreads) {
       const long long i = c0 + tid;
       const bool in = i < k1;
+      float xcur[BMAX];
+#pragma unroll
+      for (int b = 0; b < BMAX; ++b) {
+        xcur[b] = xnext[b];
+        const long long inext = i + kThreads;
+        xnext[b] = (b < a.B && inext < k1) ? to_f32(xp[(long long)b * a.K + inext]) : 0.f;
+      }
       float xv[BMAX];
       bool act = false;
 #pragma unroll
@@ -97,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_gemv_kernel(const GemvArgs
         bool m = false;
         if (b < a.B) {
           if (in) {
-            v = to_f32(xp[(long long)b * a.K + i]);
+            v = xcur[b];
             m = fabsf(v) > a.t;
           }
           if (a.bitmap_out != nullptr && tile == 0) {
@@ -108,8 +126,7 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_gemv_kernel(const GemvArgs
           }
         }
         act |= m;
-        xv[b] = m ? v : 0.f;
-        if (a.union_mask) xv[b] = v;  // fixed below once the union is known
+        xv[b] = (m || a.union_mask) ? v : 0.f;
       }
       if (a.union_mask && !act) {
 #pragma unroll
@@ -160,131 +177,85 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_gemv_kernel(const GemvArgs
   }
   __syncthreads();
 
-  // ---------------------------------------------------------------- 2/3. stream + FMA
+  // ---------------------------------------------------------------- 2. stream + FMA
   const int nrows = s_count;
-  const int nst = (nrows + SR - 1) / SR;
-  const uint32_t seg_bytes = (uint32_t)ncols * (uint32_t)sizeof(TW);
-  const int rg = tid / TPR;
-  const int tc = tid % TPR;
+  const int chunk = warp % C;      // which 256-column chunk this warp reads
+  const int wrow = warp / C;       // row phase of this warp within the chunk
+  const int col = chunk * 256 + lane * 8;
+  const bool col_ok = col < ncols;
+  const uint64_t pol = l2_evict_first_policy();
+  const TW* Wc = reinterpret_cast<const TW*>(a.W) + n0 + col;
   float acc[BMAX][8];
 #pragma unroll
   for (int b = 0; b < BMAX; ++b)
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[b][j] = 0.f;
 
-  if (warp == kProducerWarp) {
-    const uint64_t pol = l2_evict_first_policy();
-    const TW* Wp = reinterpret_cast<const TW*>(a.W);
-    for (int st = 0; st < nst; ++st) {
-      const int slot = st % a.nstage;
-      const int use = st / a.nstage;
-      if (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1, &s_abort)) {
-        s_abort = 1;
-        raise_status(a.status, SFX_DEV_TIMEOUT);
-        break;
-      }
-      const int r0 = st * SR;
-      const int rows = min(SR, nrows - r0);
-      if (lane == 0) mbar_arrive_expect_tx(&full[slot], (uint32_t)rows * seg_bytes);
-      __syncwarp();
-      unsigned char* dst = stage_mem + (size_t)slot * kStageBytes;
-      for (int r = lane; r < rows; r += 32) {
-        const TW* src = Wp + (long long)list_row[r0 + r] * a.N + n0;
-        bulk_g2s(dst + (size_t)r * NT * sizeof(TW), src, seg_bytes, &full[slot], pol);
-      }
-    }
-  } else {
-    const bool col_ok = tc * 8 < ncols;
-    for (int st = 0; st < nst; ++st) {
-      const int slot = st % a.nstage;
-      const int use = st / a.nstage;
-      if (!mbar_wait(&full[slot], use & 1, &s_abort)) {
-        s_abort = 1;
-        raise_status(a.status, SFX_DEV_TIMEOUT);
-        break;
-      }
-      const int r0 = st * SR;
-      const int rows = min(SR, nrows - r0);
-      const unsigned char* src = stage_mem + (size_t)slot * kStageBytes;
-      if (col_ok) {
+  if (col_ok) {
+    // rows wrow, wrow + WPC, wrow + 2 WPC, ... ; kRowsInFlight of them per step
+    for (int r0 = wrow; r0 < nrows; r0 += WPC * kRowsInFlight) {
+      uint4 q[kRowsInFlight];
 #pragma unroll
-        for (int rr = 0; rr < RPT; ++rr) {
-          const int r = rg + rr * RG;
-          if (r < rows) {
-            const uint4 q = *reinterpret_cast<const uint4*>(src + (size_t)r * NT * 2 + tc * 16);
-            float w[8];
-            unpack8(q, w, TW());
-            const float* xr = list_x + (size_t)(r0 + r) * BMAX;
+      for (int u = 0; u < kRowsInFlight; ++u) {
+        const int r = r0 + u * WPC;
+        if (r < nrows) q[u] = ldg_stream(Wc + (long long)list_row[r] * a.N, pol);
+      }
 #pragma unroll
-            for (int b = 0; b < BMAX; ++b) {
-              const float xv = xr[b];
+      for (int u = 0; u < kRowsInFlight; ++u) {
+        const int r = r0 + u * WPC;
+        if (r < nrows) {
+          float w[8];
+          unpack8(q[u], w, TW());
+          const float* xr = list_x + (size_t)r * BMAX;
 #pragma unroll
-              for (int j = 0; j < 8; ++j) acc[b][j] = fmaf(xv, w[j], acc[b][j]);
-            }
+          for (int b = 0; b < BMAX; ++b) {
+            const float xv = xr[b];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[b][j] = fmaf(xv, w[j], acc[b][j]);
           }
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
     }
   }
   pdl_launch_dependents();
-  __syncthreads();
-  if (s_abort) {
-    // Bounded drain of copies that may still be in flight, then leave.
-    if (tid == 0) {
-      for (int s = 0; s < a.nstage; ++s) {
-        mbar_wait(&full[s], 0, nullptr, kDrainLimitNs);
-        mbar_wait(&full[s], 1, nullptr, kDrainLimitNs);
-      }
-    }
-    __syncthreads();
-    return;
-  }
 
-  // ---------------------------------------------------------------- 4. reductions
-  float* red = reinterpret_cast<float*>(stage_mem);  // [RG][NT], stages are drained
+  // ---------------------------------------------------------------- 3. reductions
   const bool swiglu = a.epi == EPI_SWIGLU;
   const long long N = a.N;
 #pragma unroll
   for (int b = 0; b < BMAX; ++b) {
     if (b >= a.B) break;
-    if (tid < kConsumerThreads && tc * 8 < ncols) {
-      float4* dst = reinterpret_cast<float4*>(red + rg * NT + tc * 8);
+    __syncthreads();  // red is free (previous token done, list reads done)
+    if (col_ok) {
+      float4* dst = reinterpret_cast<float4*>(red + wrow * NT + col);
       dst[0] = make_float4(acc[b][0], acc[b][1], acc[b][2], acc[b][3]);
       dst[1] = make_float4(acc[b][4], acc[b][5], acc[b][6], acc[b][7]);
     }
     __syncthreads();
-    if (a.S == 1) {
-      if (swiglu) {
-        float* h = reinterpret_cast<float*>(a.y);
-        for (int p = tid; p < ncols / 2; p += kThreads) {
-          float g = 0.f, u = 0.f;
+    // sum the WPC warps of each chunk: thread handles 4 columns
+    for (int v = tid; v < ncols / 4; v += kThreads) {
+      float4 s = reinterpret_cast<const float4*>(red)[v];
 #pragma unroll
-          for (int r = 0; r < RG; ++r) {
-            g += red[r * NT + 2 * p];
-            u += red[r * NT + 2 * p + 1];
-          }
-          h[(long long)b * (N / 2) + n0 / 2 + p] = silu_f(g) * u;
+      for (int r = 1; r < WPC; ++r) {
+        const float4 t4 = reinterpret_cast<const float4*>(red + r * NT)[v];
+        s.x += t4.x; s.y += t4.y; s.z += t4.z; s.w += t4.w;
+      }
+      if (a.S == 1) {
+        if (swiglu) {
+          float* h = reinterpret_cast<float*>(a.y) + (long long)b * (N / 2) + n0 / 2;
+          *reinterpret_cast<float2*>(h + 2 * v) = make_float2(silu_f(s.x) * s.y, silu_f(s.z) * s.w);
+        } else {
+          const long long o = (long long)b * N + n0 + 4 * v;
+          store_as(a.y, o + 0, a.ydt, apply_epi(a.epi, s.x));
+          store_as(a.y, o + 1, a.ydt, apply_epi(a.epi, s.y));
+          store_as(a.y, o + 2, a.ydt, apply_epi(a.epi, s.z));
+          store_as(a.y, o + 3, a.ydt, apply_epi(a.epi, s.w));
         }
       } else {
-        for (int c = tid; c < ncols; c += kThreads) {
-          float v = 0.f;
-#pragma unroll
-          for (int r = 0; r < RG; ++r) v += red[r * NT + c];
-          store_as(a.y, (long long)b * N + n0 + c, a.ydt, apply_epi(a.epi, v));
-        }
-      }
-    } else {
-      float* part = a.partials + ((long long)split * a.B + b) * N + n0;
-      for (int c = tid; c < ncols; c += kThreads) {
-        float v = 0.f;
-#pragma unroll
-        for (int r = 0; r < RG; ++r) v += red[r * NT + c];
-        part[c] = v;
+        float* part = a.partials + ((long long)split * a.B + b) * N + n0;
+        reinterpret_cast<float4*>(part)[v] = s;
       }
     }
-    __syncthreads();
   }
   if (a.S == 1) return;
 
@@ -298,31 +269,57 @@ __global__ void __launch_bounds__(kThreads, 1) sparse_gemv_kernel(const GemvArgs
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  // thread = (column group of 4, split group g of 4); split group g sums the
+  // splits s = g, g + 4, g + 8, ... in order; the four group sums are then
+  // added in group order.
+  const long long vs = (long long)a.B * N / 4;  // float4 stride between splits
+  const int nv = ncols / 4;
+  float4* gsum = reinterpret_cast<float4*>(red);  // [4][nv]
   for (int b = 0; b < a.B; ++b) {
-    const float* part = a.partials + (long long)b * N + n0;
-    const long long sstride = (long long)a.B * N;
-    if (swiglu) {
-      float* h = reinterpret_cast<float*>(a.y);
-      for (int p = tid; p < ncols / 2; p += kThreads) {
-        float g = 0.f, u = 0.f;
-        for (int s = 0; s < a.S; ++s) {
-          const float2 gu = __ldcg(reinterpret_cast<const float2*>(part + s * sstride) + p);
-          g += gu.x;
-          u += gu.y;
-        }
-        h[(long long)b * (N / 2) + n0 / 2 + p] = silu_f(g) * u;
+    __syncthreads();
+    const float4* pb = reinterpret_cast<const float4*>(a.partials + (long long)b * N + n0);
+    for (int e = tid; e < 4 * nv; e += kThreads) {
+      const int g = e / nv, v = e - g * nv;
+      float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      int s = g;
+      for (; s + 12 < a.S; s += 16) {
+        const float4 q0 = __ldcg(pb + (long long)(s + 0) * vs + v);
+        const float4 q1 = __ldcg(pb + (long long)(s + 4) * vs + v);
+        const float4 q2 = __ldcg(pb + (long long)(s + 8) * vs + v);
+        const float4 q3 = __ldcg(pb + (long long)(s + 12) * vs + v);
+        acc4.x += q0.x; acc4.y += q0.y; acc4.z += q0.z; acc4.w += q0.w;
+        acc4.x += q1.x; acc4.y += q1.y; acc4.z += q1.z; acc4.w += q1.w;
+        acc4.x += q2.x; acc4.y += q2.y; acc4.z += q2.z; acc4.w += q2.w;
+        acc4.x += q3.x; acc4.y += q3.y; acc4.z += q3.z; acc4.w += q3.w;
       }
-    } else {
-      for (int c = tid; c < ncols; c += kThreads) {
-        float v = 0.f;
-        for (int s = 0; s < a.S; ++s) v += __ldcg(part + s * sstride + c);
-        store_as(a.y, (long long)b * N + n0 + c, a.ydt, apply_epi(a.epi, v));
+      for (; s < a.S; s += 4) {
+        const float4 q0 = __ldcg(pb + (long long)s * vs + v);
+        acc4.x += q0.x; acc4.y += q0.y; acc4.z += q0.z; acc4.w += q0.w;
+      }
+      gsum[g * nv + v] = acc4;
+    }
+    __syncthreads();
+    for (int v = tid; v < nv; v += kThreads) {
+      float4 s4 = gsum[v];
+#pragma unroll
+      for (int g = 1; g < 4; ++g) {
+        const float4 t4 = gsum[g * nv + v];
+        s4.x += t4.x; s4.y += t4.y; s4.z += t4.z; s4.w += t4.w;
+      }
+      if (swiglu) {
+        float* h = reinterpret_cast<float*>(a.y) + (long long)b * (N / 2) + n0 / 2;
+        *reinterpret_cast<float2*>(h + 2 * v) = make_float2(silu_f(s4.x) * s4.y, silu_f(s4.z) * s4.w);
+      } else {
+        const long long o = (long long)b * N + n0 + 4 * v;
+        store_as(a.y, o + 0, a.ydt, apply_epi(a.epi, s4.x));
+        store_as(a.y, o + 1, a.ydt, apply_epi(a.epi, s4.y));
+        store_as(a.y, o + 2, a.ydt, apply_epi(a.epi, s4.z));
+        store_as(a.y, o + 3, a.ydt, apply_epi(a.epi, s4.w));
       }
     }
   }
   if (tid == 0) a.counters[tile] = 0;  // leave the workspace ready for the next call
 }
-
 
 template <typename TW, typename TX, int NT, int BMAX>
 inline int launch_t(const GemvPlan& p, const GemvArgs& a, cudaStream_t stream, bool pdl) {
@@ -336,7 +333,7 @@ inline int launch_t(const GemvPlan& p, const GemvArgs& a, cudaStream_t stream, b
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.col_tiles, (unsigned)p.S, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(gemv_threads(BMAX), 1, 1);
   cfg.dynamicSmemBytes = p.smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];

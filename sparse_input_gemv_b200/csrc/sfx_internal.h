@@ -35,7 +35,6 @@ struct GemvArgs {
   int S;                  // number of K splits
   int slice;              // rows of K per split (threshold mode), multiple of 32
   int list_cap;           // capacity of the per-CTA active list
-  int nstage;             // bulk-copy ring depth (16 KB per stage)
   int ydt;                // output dtype (ignored for EPI_SWIGLU: fp32)
   int epi;                // Epi
   int union_mask;         // every token uses the batch-union mask
@@ -48,7 +47,6 @@ struct GemvPlan {
   int S = 1;         // K splits
   int slice = 0;     // rows per split
   int list_cap = 0;
-  int nstage = 0;
   int col_tiles = 0;
   size_t smem = 0;
 };
