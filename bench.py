@@ -107,6 +107,46 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
+KERNEL_SOURCES = ("sparse_input_gemv_b200/csrc/sfx_gemv_kernel.cuh",
+                  "sparse_input_gemv_b200/csrc/sfx_gemv.cu",
+                  "sparse_input_gemv_b200/csrc/sfx_common.cuh")
+PROFILE_SUMMARIES = {"ffn_gate_up": "profiles/sparse_gemv_gate_up_llama3_8b.md"}
+
+
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, sparsity: float):
+    """DRAM traffic per launch from the committed ncu summary of `kernel`.
+
+    The summary records `traffic_bytes_per_launch`, the `sparsity` it was
+    taken at and `kernel_source_sha256_16` of the GEMV sources; the figure is
+    used only while those sources are unchanged (else None).
+    """
+    path = PROFILE_SUMMARIES.get(kernel)
+    if not path or not os.path.exists(os.path.join(ROOT, path)):
+        return None, "no ncu summary for this kernel"
+    fields = {}
+    for line in open(os.path.join(ROOT, path)):
+        if ":" in line and line.strip().startswith("- `"):
+            k, v = line.strip()[3:].split("`", 1)[0], line.split(":", 1)[1].strip().strip("`")
+            fields[k] = v
+    try:
+        if fields.get("kernel_source_sha256_16") != kernel_source_hash():
+            return None, "kernel changed since the ncu capture"
+        if abs(float(fields.get("sparsity", "nan")) - sparsity) > 1e-9:
+            return None, "ncu capture taken at another sparsity"
+        return int(fields["traffic_bytes_per_launch"]), f"ncu capture, {path}"
+    except (KeyError, ValueError):
+        return None, "ncu summary unreadable"
+
+
 def time_graph(graph, reps, stream):
     """Device time of `reps` replays of a captured graph (CUDA events, ms)."""
     start = torch.cuda.Event(enable_timing=True)
@@ -481,15 +521,7 @@ def main():
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"], "peak": peak,
                 "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak, "peak_source": peak_src,
                 "traffic": None}
-    traffic_file = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(traffic_file):
-        try:
-            tr = json.load(open(traffic_file))
-            if tr.get("kernel") == dom and tr.get("sparsity") == args.sparsity:
-                roofline["traffic"] = tr.get("bytes_per_launch")
-                roofline["traffic_note"] = tr.get("note")
-        except Exception:
-            pass
+    roofline["traffic"], roofline["traffic_note"] = profiled_traffic(dom, args.sparsity)
 
     # sweep over sparsity (shorter runs, graph replay only)
     sweep = []

@@ -266,26 +266,30 @@ int sfx_pack_gate_up(const void* W_g, const void* W_u, int dt, int d, int ffn,
  * Per token t: p = softmax(logits[t]) over E experts; the top_k experts by p
  * (ties to the lower index) with weights w = p / sum(p_selected)
  * (SFX_FLAG_NO_RENORM: raw p). For each selected expert e:
- *   a = SiLU(x_t W_g[e])            (dense gate projection)
- *   m_j = |a_j| > t_e[e]            (one threshold pass)
+ *   a_j = SiLU(W_gT[e][j, :] . x_t)  (dense gate projection)
+ *   m_j = |a_j| > t_e[e]             (one threshold pass)
  *   y_t += w_e * sum_{j: m_j} a_j (W_upT[e][j, :] . x_t) W_d[e][j, :]
  * reading only rows j of W_upT[e] and W_d[e] with m_j = 1. If Ws_gu is not
  * NULL, a dense shared SwiGLU expert (always on) is added:
  * y_t += SwiGLU(x_t; Ws_gu [d x 2 ffn_shared] interleaved, Ws_d [ffn_shared x d]).
+ * All three expert matrices are stored one row per intermediate neuron
+ * ([ffn x d] per expert), so each neuron's gate, up and down weights are
+ * contiguous 2d-byte rows. Experts are combined into an fp32 accumulator with
+ * atomics, so the last bits of y may differ between runs.
  *
- *  x       (dev) [B x d] dtype dt (bf16 or f16)
+ *  x       (dev) [B x d] dtype dt (bf16 or f16), 16-byte aligned
  *  logits  (dev) [B x E] f32
- *  W_g     (dev) [E x d x ffn]   W_upT (dev) [E x ffn x d]   W_d (dev) [E x ffn x d]
+ *  W_gT    (dev) [E x ffn x d]   W_upT (dev) [E x ffn x d]   W_d (dev) [E x ffn x d]
  *  t_e     (dev) [E] f32 per-expert thresholds (-INFINITY: dense expert)
  *  y       (dev) [B x d] dtype ydt
  *  a_out   (dev, optional) [B x top_k x ffn] f32 gate activations a, in each
  *          token's selection order; sel_out (dev, optional) [B x top_k] int32
  *          selected experts
  *  ws      (dev) sfx_workspace_bytes(SFX_OP_MOE, B, d, E, ffn, top_k, ffn_shared)
- * Limits: 1 <= B <= 64, 1 <= top_k <= E <= 1024, d % 8 == 0, ffn % 8 == 0.
+ * Limits: 1 <= B <= 16, 1 <= top_k <= E <= 1024, d % 8 == 0, ffn % 8 == 0.
  * ---------------------------------------------------------------------- */
 int sfx_moe_expert_sparse(const void* x, int dt, const float* logits, int B, int d, int E,
-                          int ffn, int top_k, const void* W_g, const void* W_upT,
+                          int ffn, int top_k, const void* W_gT, const void* W_upT,
                           const void* W_d, const float* t_e, const void* Ws_gu,
                           const void* Ws_d, int ffn_shared, void* y, int ydt,
                           float* a_out, int32_t* sel_out, int flags,

@@ -285,16 +285,20 @@ def sfx_sparse_ffn_swiglu(x, W_gu, W_d, t_in=-math.inf, t_h=-math.inf, out_dtype
     return out
 
 
-def sfx_moe_expert_sparse(x, logits, W_g, W_upT, W_d, t_e, top_k, Ws_gu=None, Ws_d=None,
+def sfx_moe_expert_sparse(x, logits, W_gT, W_upT, W_d, t_e, top_k, Ws_gu=None, Ws_d=None,
                           out_dtype=None, flags=0, want_a=False, y=None,
                           ws: Workspace | None = None, stream=None):
-    """MoE layer with intra-expert magnitude masks; returns dict(y[, a, sel])."""
+    """MoE layer with intra-expert magnitude masks; returns dict(y[, a, sel]).
+
+    W_gT, W_upT, W_d: [E x ffn x d] (one row per intermediate neuron).
+    """
     squeeze = x.dim() == 1
     x2 = x[None] if squeeze else x
     lg = logits[None] if logits.dim() == 1 else logits
-    _need_cuda(x2, lg, W_g, W_upT, W_d, t_e, Ws_gu, Ws_d)
+    _need_cuda(x2, lg, W_gT, W_upT, W_d, t_e, Ws_gu, Ws_d)
     B, d = x2.shape
-    E, _, ffn = W_g.shape
+    E, ffn, _ = W_gT.shape
+    W_g = W_gT
     ffn_s = Ws_d.shape[0] if Ws_d is not None else 0
     dev = x2.device
     out_dtype = out_dtype or x2.dtype

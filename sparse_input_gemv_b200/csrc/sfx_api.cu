@@ -279,7 +279,7 @@ int sfx_moe_expert_sparse(const void* x, int dt, const float* logits, int B, int
                           void* y, int ydt, float* a_out, int32_t* sel_out, int flags, void* ws,
                           size_t ws_bytes, void* stream) {
   if (!x || !logits || !W_g || !W_upT || !W_d || !t_e || !y) return SFX_ERR_ARG;
-  if (B < 1 || B > 64 || E < 1 || E > 1024 || top_k < 1 || top_k > E || d < 8 || ffn < 8)
+  if (B < 1 || B > 16 || E < 1 || E > 1024 || top_k < 1 || top_k > E || d < 8 || ffn < 8)
     return SFX_ERR_ARG;
   if ((Ws_gu == nullptr) != (Ws_d == nullptr) || (Ws_gu && ffn_shared < 4)) return SFX_ERR_ARG;
   if (!(dt == SFX_F16 || dt == SFX_BF16) || !valid_dtype(ydt)) return SFX_ERR_DTYPE;

@@ -1,0 +1,115 @@
+"""MoE layer with intra-expert activation sparsity: CUDA path vs the fp64 oracle.
+
+Routing (selected experts) is compared exactly; the output within the float
+tolerance; the gate activations a within tolerance, and a neuron's mask may
+differ between the fp32 GPU gate and the fp64 oracle only where a lies within
+rounding distance of the expert's threshold.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from helpers import assert_close, to64
+from sparse_input_gemv_b200 import binding as sb
+from sparse_input_gemv_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    sb.load()
+
+
+def make_moe(name, E, d, ffn, ffn_s, dtype="bf16"):
+    dev = "cuda"
+    Wg = synth.normal((E, d, ffn), synth.seed_of(name, "Wg"), 0.02, dtype, dev)
+    WuT = synth.normal((E, ffn, d), synth.seed_of(name, "WuT"), 0.02, dtype, dev)
+    Wd = synth.normal((E, ffn, d), synth.seed_of(name, "Wd"), 0.02, dtype, dev)
+    sh = None
+    if ffn_s:
+        Sg = synth.normal((d, ffn_s), synth.seed_of(name, "Sg"), 0.02, dtype, dev)
+        Su = synth.normal((d, ffn_s), synth.seed_of(name, "Su"), 0.02, dtype, dev)
+        Sd = synth.normal((ffn_s, d), synth.seed_of(name, "Sd"), 0.02, dtype, dev)
+        sh = (Sg, Su, Sd)
+    return Wg, WuT, Wd, sh
+
+
+def expert_thresholds(name, Wg64, experts, p, d, dtype):
+    """Per-expert t_e: the oracle's calibration on |SiLU(x W_g[e])| over 64 draws.
+
+    Only the experts the batch routes to get one (the others are never read).
+    """
+    E = Wg64.shape[0]
+    if p <= 0:
+        return np.full(E, -np.inf, dtype=np.float32)
+    xc = to64(synth.calib_draws(name, "x", 64, d, dtype))
+    te = np.full(E, np.inf, dtype=np.float32)
+    for e in experts:
+        te[e] = np.float32(O.calibrate_threshold(O.silu(xc @ Wg64[e]), p))
+    return te
+
+
+def run_case(name, B, E, d, ffn, top_k, ffn_s, p, flags=0, expert_subset=None):
+    dtype = "bf16"
+    Wg, WuT, Wd, sh = make_moe(name, E, d, ffn, ffn_s, dtype)
+    x = synth.eval_draw(name, "x", B, d, dtype)
+    logits = synth.normal((B, E), synth.seed_of(name, "logits", B), 1.0, "f32")
+    # oracle routing first: which experts' weights need to come to the host
+    renorm = not (flags & sb.SFX_FLAG_NO_RENORM)
+    routes = [O.moe_route(logits.numpy()[t].astype(np.float64), top_k, renorm) for t in range(B)]
+    used = sorted({int(e) for ex, _ in routes for e in ex})
+    Wg64 = np.zeros((E, d, ffn))
+    WuT64 = np.zeros((E, ffn, d))
+    Wd64 = np.zeros((E, ffn, d))
+    for e in used:
+        Wg64[e], WuT64[e], Wd64[e] = to64(Wg[e]), to64(WuT[e]), to64(Wd[e])
+    te = expert_thresholds(name, Wg64, used, p, d, dtype)
+    WgT = Wg.transpose(1, 2).contiguous()
+    Sgu = sb.sfx_pack_gate_up(sh[0], sh[1]) if sh else None
+    out = sb.sfx_moe_expert_sparse(x.cuda(), logits.cuda(), WgT, WuT, Wd,
+                                   torch.from_numpy(te).cuda(), top_k, Ws_gu=Sgu,
+                                   Ws_d=sh[2] if sh else None, flags=flags, want_a=True)
+    sh64 = (to64(sh[0]), to64(sh[1]), to64(sh[2])) if sh else (None, None, None)
+    want = O.moe_layer(to64(x), logits.numpy().astype(np.float64), Wg64, WuT64, Wd64,
+                       te.astype(np.float64), top_k, *sh64, renormalize=renorm)
+    # routing is exact
+    sel = out["sel"].cpu().numpy()
+    for t in range(B):
+        assert sel[t].tolist() == routes[t][0].tolist(), (t, sel[t], routes[t][0])
+    # gate activations within tolerance; mask flips only at the threshold
+    a_gpu = out["a"].cpu().numpy().astype(np.float64)
+    for t in range(B):
+        for k, e in enumerate(routes[t][0]):
+            _, a_ref, m_ref = O.moe_expert(to64(x)[t], Wg64[e], WuT64[e], Wd64[e], float(te[e]))
+            assert_close(a_gpu[t, k], O.round_to(a_ref, "f32"), f"a t={t} e={e}")
+            flips = np.flatnonzero((np.abs(a_gpu[t, k]) > te[e]) != m_ref)
+            for j in flips:
+                assert abs(abs(a_ref[j]) - te[e]) <= 1e-4 * np.abs(a_ref).max()
+            assert flips.size <= 2
+    assert_close(to64(out["y"]), O.round_to(want, dtype), f"y B={B} p={p}")
+    return out
+
+
+@pytest.mark.parametrize("B,p", [(1, 0.5), (3, 0.8), (16, 0.9), (2, 0.0)])
+def test_moe_small_ragged(B, p):
+    run_case("moe-small", B, 16, 264, 72, 4, 136, p)
+
+
+def test_moe_without_shared_expert_and_raw_weights():
+    run_case("moe-noshared", 5, 12, 256, 64, 3, 0, 0.5, flags=sb.SFX_FLAG_NO_RENORM)
+
+
+def test_moe_top1_of_1():
+    run_case("moe-one", 4, 1, 128, 32, 1, 0, 0.5)
+
+
+@pytest.mark.parametrize("B,p", [(1, 0.5), (4, 0.8)])
+def test_moe_128_experts_full_size(B, p):
+    # 128 experts, d = 2048, expert ffn = 768 SwiGLU, top-8, shared ffn = 2048
+    run_case("moe-config", B, 128, 2048, 768, 8, 2048, p)
