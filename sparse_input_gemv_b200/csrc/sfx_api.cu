@@ -213,6 +213,7 @@ int sfx_sparse_gemv(const void* x, int xdt, int B, int K, const void* W, int wdt
         : (flags & SFX_FLAG_GELU_TANH) ? EPI_GELU_TANH
                                        : EPI_NONE;
   a.union_mask = (flags & SFX_FLAG_UNION_MASK) ? 1 : 0;
+  a.no_tc = (flags & SFX_FLAG_CUDA_CORES) ? 1 : 0;
   a.t = t;
   return launch_sparse_gemv(wdt, xdt, plan, a, as_stream(stream), false);
 }
@@ -244,6 +245,7 @@ int sfx_sparse_ffn_swiglu(const void* x, int dt, int B, int d, int ffn, const vo
   a.ydt = SFX_F32;
   a.epi = EPI_SWIGLU;
   a.union_mask = umask;
+  a.no_tc = (flags & SFX_FLAG_CUDA_CORES) ? 1 : 0;
   a.t = t_in;
   carve_gemv(ws, gbody, a);
   int rc = launch_sparse_gemv(dt, dt, plan_gemv(a.K, a.N, B, false), a, s, false);
@@ -261,6 +263,7 @@ int sfx_sparse_ffn_swiglu(const void* x, int dt, int B, int d, int ffn, const vo
   b.ydt = ydt;
   b.epi = EPI_NONE;
   b.union_mask = umask;
+  b.no_tc = a.no_tc;
   b.t = t_h;
   carve_gemv(ws, gbody, b);
   return launch_sparse_gemv(dt, SFX_F32, plan_gemv(b.K, b.N, B, false), b, s, true);

@@ -38,6 +38,7 @@ struct GemvArgs {
   int ydt;                // output dtype (ignored for EPI_SWIGLU: fp32)
   int epi;                // Epi
   int union_mask;         // every token uses the batch-union mask
+  int no_tc;              // keep B >= 4 on the CUDA-core kernel
   float t;                // magnitude threshold (threshold mode)
 };
 
@@ -56,6 +57,12 @@ GemvPlan plan_gemv(long long K, long long N, int B, bool idx_mode);
 size_t gemv_workspace_bytes(long long K, long long N, int B);  // excludes the header
 int launch_sparse_gemv(int wdt, int xdt, const GemvPlan& plan, GemvArgs a, cudaStream_t stream,
                        bool pdl);
+
+// batch-union GEMM on tcgen05 (sfx_union_tc.cu), used for B >= kTcMinBatch
+constexpr int kTcMinBatch = 5;  // measured: CUDA cores win up to 4 tokens
+GemvPlan plan_union_tc(long long K, long long N);
+size_t union_tc_workspace_bytes(long long K, long long N, int B);
+int launch_union_tc(int wdt, int xdt, const GemvPlan& plan, const GemvArgs& a, cudaStream_t stream);
 
 // mask / selection kernels (sfx_mask.cu)
 size_t mask_workspace_bytes(int B, int K, int sel);

@@ -99,6 +99,7 @@ extern "C" int sfx_sparse_gemv_noalloc(const void* x, int xdt, int B, int K, con
         : (flags & SFX_FLAG_GELU_TANH) ? EPI_GELU_TANH
                                        : EPI_NONE;
   a.union_mask = (flags & SFX_FLAG_UNION_MASK) ? 1 : 0;
+  a.no_tc = (flags & SFX_FLAG_CUDA_CORES) ? 1 : 0;
   a.t = t;
   return launch_sparse_gemv(wdt, xdt, plan, a, s, false);
 }

@@ -1,0 +1,562 @@
+// Batch-union skinny GEMM on the 5th-generation tensor cores (tcgen05).
+//
+// For a batch of B <= 16 tokens with per-token magnitude masks ("TEAL:
+// Training-Free Activation Sparsity in Large Language Models", slide 8),
+// y[b, n] = sum_i (x[b, i] m[b, i]) W[i, n]. The rows any token keeps (the
+// union) are fetched once and multiplied as a dense tile: with B tokens the
+// product has B FLOPs per weight byte, more than CUDA cores sustain at HBM
+// speed once B grows, so it runs as tcgen05.mma:
+//
+//   D[m, b] (TMEM, fp32)  +=  A[m, k] * B[k, b]
+//   A = W[union rows, n0 : n0+128]   (M = 128 output columns, MN-major)
+//   B = x[b, union rows] * m[b, row] (N = 16 padded tokens, K-major)
+//
+// Two kernels:
+//  1. union_pack_kernel, one CTA per K-split: compacts the split's union rows
+//     (warp ballots, ascending) into a row list in the workspace, and writes
+//     the B operand for them -- already in the canonical K-major no-swizzle
+//     layout of 16-row K-steps (8 x 8 core matrices, SBO = 128 B between token
+//     groups, LBO = 256 B between row halves), bf16/f16, plus a "lo" copy
+//     holding x - hi when x is fp32 (two MMAs per K-step keep ~16 bits).
+//     Rows past the list are zero, padded to whole 64-row stages.
+//  2. union_gemm_tc_kernel, grid (128-column tiles) x (K-splits), warp
+//     specialised: 8 producer warps copy A (64 rows x 256 B per stage, 16-byte
+//     cp.async straight into the canonical MN-major layout: SBO = 128 B
+//     between column groups, LBO = 2 KB between row halves; L2 evict-first)
+//     and B (the packed tiles) into a 4-stage ring and signal each stage's
+//     "full" mbarrier with cp.async.mbarrier.arrive.noinc; one MMA warp waits
+//     on it, issues the stage's four K-steps as tcgen05.mma into a TMEM
+//     accumulator and commits them to the stage's "empty" mbarrier, on which
+//     the producers wait before refilling. No CTA-wide barrier in the loop.
+//     Epilogue: tcgen05.ld (warps 0-3 own TMEM lanes 32w..32w+31), then the
+//     deterministic split-K reduction shared with the CUDA-core kernel.
+// Every mbarrier wait is bounded; on timeout the kernel raises
+// SFX_DEV_TIMEOUT, drains its copies, frees its TMEM and returns.
+#include "sfx_common.cuh"
+#include "sfx_internal.h"
+
+#include <algorithm>
+
+namespace sfx {
+
+namespace {
+
+constexpr int kTcM = 128;          // output columns per CTA (MMA M)
+constexpr int kTcN = 16;           // padded tokens (MMA N)
+constexpr int kTcK = 16;           // rows per MMA K-step (16-bit inputs)
+constexpr int kSub = 4;            // K-steps per stage
+constexpr int kRowsPerStage = kSub * kTcK;  // 64
+constexpr int kStages = 4;
+constexpr int kProducers = 256;    // warps 0-7
+constexpr int kTcThreads = kProducers + 32;  // + the MMA warp
+constexpr int kABytes = kTcM * kTcK * 2;    // 4 KB per K-step
+constexpr int kBBytes = kTcN * kTcK * 2;    // 512 B per K-step (hi or lo)
+constexpr int kSubBytes = kABytes + 2 * kBBytes;
+constexpr int kStageBytes = kSub * kSubBytes;  // 20 KB
+constexpr int kTmemCols = 64;         // four 16-column accumulators (one per K-step of a stage)
+constexpr int kPackThreads = 256;
+
+struct TcArgs {
+  GemvArgs g;
+  int32_t* rows;      // [S x slice] union rows per split
+  int32_t* counts;    // [S] union rows per split
+  int32_t* chunk_counts;  // [ceil(K / 256)] union rows per 256-row chunk
+  uint16_t* pack;     // [S x slice/16 x (hi, lo) x 256] B tiles per split
+  int split_b;        // 1 if x is fp32 (hi + lo tiles)
+};
+
+__device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid,
+                                                 uint64_t pol) {
+  const int n = valid ? 16 : 0;
+  asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2, %3;" ::"r"(dst),
+               "l"(src), "r"(n), "l"(pol)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+// arrive on `bar` once this thread's earlier cp.async copies have landed
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor, no swizzle (version 1 for this architecture).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+// Instruction descriptor for kind::f16: fp32 accumulate, A and B of the same
+// 16-bit type, A MN-major, B K-major, N = 16, M = 128.
+__host__ __device__ constexpr uint32_t instr_desc(bool bf16) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | (1u << 15) |
+         (0u << 16) | ((uint32_t)(kTcN >> 3) << 17) | ((uint32_t)(kTcM >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f16(uint32_t tmem, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n\t}\n" ::"r"(tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0), "r"(0), "r"(0), "r"(0)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+template <typename T> __device__ __forceinline__ uint16_t to_bits16(float v);
+template <> __device__ __forceinline__ uint16_t to_bits16<__nv_bfloat16>(float v) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+}
+template <> __device__ __forceinline__ uint16_t to_bits16<__half>(float v) {
+  return __half_as_ushort(__float2half_rn(v));
+}
+template <typename T> __device__ __forceinline__ float from_bits16(uint16_t b);
+template <> __device__ __forceinline__ float from_bits16<__nv_bfloat16>(uint16_t b) {
+  return __bfloat162float(__ushort_as_bfloat16(b));
+}
+template <> __device__ __forceinline__ float from_bits16<__half>(uint16_t b) {
+  return __half2float(__ushort_as_half(b));
+}
+
+// offset (in elements) of (token b, row kk) inside one 16 x 16 K-major B tile
+__device__ __forceinline__ int btile_off(int b, int kk) {
+  return ((b & 7) * 16 + (b >> 3) * 128 + (kk & 7) * 2 + (kk >> 3) * 256) / 2;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------- 1. union + pack
+
+// Token bits of row i: bit b set iff |x[b, i]| > t (xv receives the values).
+template <typename TX>
+__device__ __forceinline__ uint32_t row_bits(const GemvArgs& a, long long i, bool in, float (&xv)[kTcN]) {
+  const TX* xp = reinterpret_cast<const TX*>(a.x);
+  uint32_t bits = 0;
+#pragma unroll
+  for (int b = 0; b < kTcN; ++b) {
+    xv[b] = (in && b < a.B) ? to_f32(xp[(long long)b * a.K + i]) : 0.f;
+    bits |= ((in && b < a.B && fabsf(xv[b]) > a.t) ? 1u : 0u) << b;
+  }
+  return bits;
+}
+
+// Pass 1, one CTA per 256-row chunk of K: the number of union rows in the
+// chunk (and the fused-mask bitmap words, if requested).
+template <typename TX>
+__global__ void __launch_bounds__(kPackThreads) union_count_kernel(const TcArgs t) {
+  const GemvArgs& a = t.g;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long i = (long long)blockIdx.x * kPackThreads + tid;
+  const bool in = i < a.K;
+  pdl_wait();
+  float xv[kTcN];
+  const uint32_t bits = row_bits<TX>(a, i, in, xv);
+  if (a.bitmap_out != nullptr) {
+    const long long w0 = (long long)blockIdx.x * kPackThreads + warp * 32;
+    for (int b = 0; b < a.B; ++b) {
+      const unsigned bal = __ballot_sync(0xffffffffu, (bits >> b) & 1u);
+      if (lane == 0 && w0 < a.K) a.bitmap_out[(long long)b * ((a.K + 31) >> 5) + (w0 >> 5)] = bal;
+    }
+  }
+  const int n = __syncthreads_count(bits != 0);
+  if (tid == 0) t.chunk_counts[blockIdx.x] = n;
+  pdl_launch_dependents();
+}
+
+// Pass 2, one CTA per 256-row chunk: the chunk's union rows go to positions
+// base + (rank within the chunk) of its split's list, base = union rows of the
+// split's earlier chunks; the matching B operand values go into the packed
+// K-major tiles. The split's last chunk records the split's count and zeroes
+// the B rows up to the end of the last 64-row stage.
+template <typename TW, typename TX>
+__global__ void __launch_bounds__(kPackThreads) union_pack_kernel(const TcArgs t) {
+  const GemvArgs& a = t.g;
+  __shared__ int s_warp_tot[kPackThreads / 32];
+  __shared__ int s_base;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int chunk = blockIdx.x;
+  const long long i = (long long)chunk * kPackThreads + tid;
+  const bool in = i < a.K;
+  const int per_split = a.slice / kPackThreads;
+  const int split = chunk / per_split;
+  const int first = split * per_split;
+  const int last = min((int)((a.K + kPackThreads - 1) / kPackThreads), first + per_split) - 1;
+  int32_t* rows = t.rows + (long long)split * a.slice;
+  const int tile_elems = 256 * (t.split_b ? 2 : 1);  // per 16-row K-step
+  uint16_t* pack = t.pack + (long long)split * (a.slice / kTcK) * tile_elems;
+  pdl_wait();  // chunk counts of pass 1
+  if (warp == 0) {
+    int s = 0;
+    for (int c = first + lane; c < chunk; c += 32) s += t.chunk_counts[c];
+    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0) s_base = s;
+  }
+  float xv[kTcN];
+  uint32_t bits = row_bits<TX>(a, i, in, xv);
+  const bool act = bits != 0;
+  const unsigned bal = __ballot_sync(0xffffffffu, act);
+  if (lane == 0) s_warp_tot[warp] = __popc(bal);
+  __syncthreads();
+  int woff = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kPackThreads / 32; ++w) {
+    const int c = s_warp_tot[w];
+    woff += (w < warp) ? c : 0;
+    tot += c;
+  }
+  const int base = s_base;
+  if (act) {
+    const int pos = base + woff + __popc(bal & lanemask_lt());
+    rows[pos] = (int32_t)i;
+    uint16_t* tl = pack + (long long)(pos / kTcK) * tile_elems;
+    const int kk = pos % kTcK;
+    if (a.union_mask) bits = (1u << a.B) - 1u;
+#pragma unroll
+    for (int b = 0; b < kTcN; ++b) {
+      const float v = ((bits >> b) & 1u) ? xv[b] : 0.f;
+      const uint16_t hi = to_bits16<TW>(v);
+      tl[btile_off(b, kk)] = hi;
+      if (t.split_b) tl[256 + btile_off(b, kk)] = to_bits16<TW>(v - from_bits16<TW>(hi));
+    }
+  }
+  if (chunk == last) {
+    const int n = base + tot;
+    if (tid == 0) t.counts[split] = n;
+    const int padded = (n + kRowsPerStage - 1) / kRowsPerStage * kRowsPerStage;
+    for (int e = n * kTcN + tid; e < padded * kTcN; e += kPackThreads) {
+      const int pos = e / kTcN, b = e % kTcN;
+      uint16_t* tl = pack + (long long)(pos / kTcK) * tile_elems;
+      tl[btile_off(b, pos % kTcK)] = 0;
+      if (t.split_b) tl[256 + btile_off(b, pos % kTcK)] = 0;
+    }
+  }
+  pdl_launch_dependents();
+}
+
+// ---------------------------------------------------------------- 2. tcgen05 GEMM
+
+template <typename TW>
+__global__ void __launch_bounds__(kTcThreads, 2) union_gemm_tc_kernel(const TcArgs t) {
+  const GemvArgs& a = t.g;
+  extern __shared__ __align__(1024) unsigned char smem[];
+  unsigned char* stages = smem;
+  int32_t* list_row = reinterpret_cast<int32_t*>(smem + (size_t)kStages * kStageBytes);
+  __shared__ __align__(8) uint64_t s_full[kStages];
+  __shared__ __align__(8) uint64_t s_empty[kStages];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_last;
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x, split = blockIdx.y;
+  const long long n0 = (long long)tile * kTcM;
+  const int ncols = (int)min((long long)kTcM, a.N - n0);
+
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&s_full[s], kProducers);
+      mbar_init(&s_empty[s], 1);
+    }
+    fence_barrier_init();
+    s_abort = 0;
+  }
+  if (warp == 8) {  // TMEM: four fp32 accumulators of 128 lanes x 16 columns
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s_tmem)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  pdl_wait();  // the pack kernel's rows, counts and B tiles
+  const int nrows = min(max(t.counts[split], 0), a.slice);
+  for (int r = tid; r < nrows; r += kTcThreads) list_row[r] = t.rows[(long long)split * a.slice + r];
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const int nit = (nrows + kRowsPerStage - 1) / kRowsPerStage;
+  const uint32_t sbase = smem_u32(stages);
+  const int tile_elems = 256 * (t.split_b ? 2 : 1);
+  const uint16_t* pack = t.pack + (long long)split * (a.slice / kTcK) * tile_elems;
+
+  if (warp < 8) {
+    // ------------------------------------------------ producers
+    const uint64_t pol = l2_evict_first_policy();
+    const TW* Wp = reinterpret_cast<const TW*>(a.W);
+    for (int c = 0; c < nit; ++c) {
+      const int s = c % kStages, use = c / kStages;
+      if (use > 0 && !mbar_wait(&s_empty[s], (use - 1) & 1, &s_abort)) {
+        s_abort = 1;
+        raise_status(a.status, SFX_DEV_TIMEOUT);
+        break;
+      }
+      const uint32_t sa = sbase + s * kStageBytes;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {  // A: 64 rows x 16 groups of 16 bytes
+        const int idx = tid + q * kProducers;
+        const int r = idx >> 4, g = idx & 15;
+        const int row = c * kRowsPerStage + r;
+        const bool valid = row < nrows && g * 8 < ncols;
+        const TW* src = Wp + (valid ? (long long)list_row[row] * a.N + n0 + g * 8 : 0);
+        const int sub = r >> 4, rr = r & 15;
+        cp_async16_zfill(sa + sub * kSubBytes + (rr >> 3) * 2048 + g * 128 + (rr & 7) * 16, src,
+                         valid, pol);
+      }
+      {  // B: the packed tiles of the stage's 4 K-steps (hi [, lo])
+        const int per_sub = t.split_b ? 64 : 32;  // 16-byte chunks per K-step
+        if (tid < kSub * per_sub) {
+          const int sub = tid / per_sub, ch = tid % per_sub;
+          const uint16_t* src = pack + (long long)(c * kSub + sub) * tile_elems + ch * 8;
+          cp_async16(sa + sub * kSubBytes + kABytes + ch * 16, src);
+        }
+      }
+      cp_async_arrive_noinc(&s_full[s]);
+    }
+  } else if (lane == 0) {
+    // ------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = instr_desc(DT<TW>::id == SFX_BF16);
+    for (int c = 0; c < nit; ++c) {
+      const int s = c % kStages;
+      if (!mbar_wait(&s_full[s], (c / kStages) & 1, &s_abort)) {
+        s_abort = 1;
+        raise_status(a.status, SFX_DEV_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t sa = sbase + s * kStageBytes;
+#pragma unroll
+      for (int q = 0; q < kSub; ++q) {
+        const uint32_t st = sa + q * kSubBytes;
+        const uint64_t adesc = smem_desc(st, 2048, 128);
+        // K-step q accumulates into its own 16 columns: four independent
+        // accumulation chains instead of one serial chain of MMAs
+        const uint32_t dq = tmem + (uint32_t)(q * kTcN);
+        mma_f16(dq, adesc, smem_desc(st + kABytes, 256, 128), idesc, c > 0 ? 1u : 0u);
+        if (t.split_b) mma_f16(dq, adesc, smem_desc(st + kABytes + kBBytes, 256, 128), idesc, 1u);
+      }
+      mma_commit(&s_empty[s]);
+    }
+  }
+  // all MMAs done: the last commit covers every earlier MMA
+  if (nit > 0 && !s_abort) {
+    const int c = nit - 1;
+    if (!mbar_wait(&s_empty[c % kStages], (c / kStages) & 1, &s_abort)) {
+      s_abort = 1;
+      raise_status(a.status, SFX_DEV_TIMEOUT);
+    }
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pdl_launch_dependents();
+
+  // ---------------------------------------------------------------- epilogue
+  float d[kTcN];
+#pragma unroll
+  for (int b = 0; b < kTcN; ++b) d[b] = 0.f;
+  if (warp < 4 && nit > 0 && !s_abort) {
+    // sum the four accumulators in K-step order
+#pragma unroll
+    for (int q = 0; q < kSub; ++q) {
+      uint32_t r[16];
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+          "%14,%15}, [%16];"
+          : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+            "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+            "=r"(r[14]), "=r"(r[15])
+          : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(q * kTcN)));
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+      for (int b = 0; b < kTcN; ++b) d[b] += __uint_as_float(r[b]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kTmemCols)
+                 : "memory");
+  }
+  if (s_abort) return;
+
+  const long long N = a.N;
+  const bool swiglu = a.epi == EPI_SWIGLU;
+  const int m = tid;  // output column within the tile (threads 0..127)
+  if (a.S == 1) {
+    if (warp < 4) {
+#pragma unroll
+      for (int b = 0; b < kTcN; ++b) {
+        if (b >= a.B) break;
+        if (swiglu) {
+          const float up = __shfl_down_sync(0xffffffffu, d[b], 1);
+          if ((m & 1) == 0 && m < ncols)
+            reinterpret_cast<float*>(a.y)[(long long)b * (N / 2) + (n0 + m) / 2] = silu_f(d[b]) * up;
+        } else if (m < ncols) {
+          float v = d[b];
+          if (a.epi == EPI_GELU) v = gelu_erf_f(v);
+          else if (a.epi == EPI_GELU_TANH) v = gelu_tanh_f(v);
+          store_as(a.y, (long long)b * N + n0 + m, a.ydt, v);
+        }
+      }
+    }
+    return;
+  }
+  if (warp < 4 && m < ncols) {
+#pragma unroll
+    for (int b = 0; b < kTcN; ++b)
+      if (b < a.B) a.partials[((long long)split * a.B + b) * N + n0 + m] = d[b];
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(&a.counters[tile], 1) == a.S - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const long long vs = (long long)a.B * N;
+  // pairs of columns so the SwiGLU epilogue sees (gate, up) together
+  for (int e = tid; e < a.B * (kTcM / 2); e += kTcThreads) {
+    const int b = e / (kTcM / 2), c2 = 2 * (e % (kTcM / 2));
+    if (c2 >= ncols) continue;
+    const float* pb = a.partials + (long long)b * N + n0 + c2;
+    float s0 = 0.f, s1 = 0.f;
+    for (int s = 0; s < a.S; ++s) {
+      const float2 q = __ldcg(reinterpret_cast<const float2*>(pb + s * vs));
+      s0 += q.x;
+      s1 += q.y;
+    }
+    if (swiglu) {
+      reinterpret_cast<float*>(a.y)[(long long)b * (N / 2) + (n0 + c2) / 2] = silu_f(s0) * s1;
+    } else {
+      if (a.epi == EPI_GELU) { s0 = gelu_erf_f(s0); s1 = gelu_erf_f(s1); }
+      else if (a.epi == EPI_GELU_TANH) { s0 = gelu_tanh_f(s0); s1 = gelu_tanh_f(s1); }
+      store_as(a.y, (long long)b * N + n0 + c2, a.ydt, s0);
+      store_as(a.y, (long long)b * N + n0 + c2 + 1, a.ydt, s1);
+    }
+  }
+  if (tid == 0) a.counters[tile] = 0;
+}
+
+// ------------------------------------------------------------------ host
+
+static long long rup(long long v, long long m) { return (v + m - 1) / m * m; }
+static constexpr long long kMaxSlice = 6144;  // 24 KB row list in shared memory
+
+GemvPlan plan_union_tc(long long K, long long N) {
+  GemvPlan p;
+  p.NT = kTcM;
+  p.BMAX = kTcN;
+  p.col_tiles = (int)((N + kTcM - 1) / kTcM);
+  // one wave of resident CTAs (two per SM); K splits only to fill it (at
+  // least 256 rows each) or to keep a split's list within kMaxSlice rows
+  const long long slots = 2LL * sm_count();
+  long long S = std::max<long long>(1, slots / p.col_tiles);
+  S = std::min<long long>(S, std::max<long long>(1, K / 256));
+  long long slice = rup((K + S - 1) / S, kPackThreads);  // whole 256-row pack chunks
+  if (slice > kMaxSlice) slice = kMaxSlice;
+  p.S = (int)((K + slice - 1) / slice);
+  p.slice = (int)slice;
+  p.list_cap = (int)slice;
+  p.smem = (size_t)kStages * kStageBytes + (size_t)slice * 4;
+  return p;
+}
+
+// workspace after the header: [partials S x B x N f32] then, 256-aligned,
+// [rows S x slice][split counts][chunk counts][B tiles S x slice/16 x (hi, lo)]
+struct TcAux {
+  size_t rows, counts, chunk_counts, pack, total;
+};
+static TcAux tc_aux(const GemvPlan& p, long long K) {
+  TcAux x;
+  x.rows = 0;
+  x.counts = x.rows + (size_t)p.S * p.slice * 4;
+  x.chunk_counts = x.counts + rup((long long)p.S * 4, 256);
+  x.pack = x.chunk_counts + rup((K + kPackThreads - 1) / kPackThreads * 4, 256);
+  x.total = x.pack + (size_t)p.S * (p.slice / kTcK) * 256 * 2 * 2;  // hi + lo, bytes
+  return x;
+}
+
+size_t union_tc_workspace_bytes(long long K, long long N, int B) {
+  const GemvPlan p = plan_union_tc(K, N);
+  return (size_t)(p.S > 1 ? p.S : 0) * B * N * 4 + 256 /* alignment */ + tc_aux(p, K).total;
+}
+
+// One opt-in per kernel (shared by the bf16/f16 and fp32 activation paths):
+// the largest dynamic shared memory any plan asks for.
+template <typename TW>
+static int configure_tc_kernel() {
+  static int rc = cudaFuncSetAttribute(union_gemm_tc_kernel<TW>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)((size_t)kStages * kStageBytes + kMaxSlice * 4)) ==
+                          cudaSuccess
+                      ? SFX_OK
+                      : SFX_ERR_CUDA;
+  return rc;
+}
+
+template <typename TW, typename TX>
+static int launch_tc(const GemvPlan& p, TcArgs t, cudaStream_t s) {
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((t.g.K + kPackThreads - 1) / kPackThreads), 1, 1);
+  cfg.blockDim = dim3(kPackThreads, 1, 1);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, union_count_kernel<TX>, t) != cudaSuccess) return SFX_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, union_pack_kernel<TW, TX>, t) != cudaSuccess) return SFX_ERR_CUDA;
+
+  auto kern = union_gemm_tc_kernel<TW>;
+  if (configure_tc_kernel<TW>() != SFX_OK) return SFX_ERR_CUDA;
+  cfg.gridDim = dim3((unsigned)p.col_tiles, (unsigned)p.S, 1);
+  cfg.blockDim = dim3(kTcThreads, 1, 1);
+  cfg.dynamicSmemBytes = p.smem;
+  return cudaLaunchKernelEx(&cfg, kern, t) == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
+}
+
+int launch_union_tc(int wdt, int xdt, const GemvPlan& p, const GemvArgs& a, cudaStream_t s) {
+  if (p.col_tiles > kCounterSlots) return SFX_ERR_UNSUPPORTED;
+  TcArgs t;
+  t.g = a;
+  t.g.S = p.S;
+  t.g.slice = p.slice;
+  t.g.list_cap = p.list_cap;
+  // auxiliary buffers follow the split-K partials in the workspace
+  unsigned char* aux = reinterpret_cast<unsigned char*>(a.partials) +
+                       (size_t)(p.S > 1 ? p.S : 0) * a.B * a.N * 4;
+  aux = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(aux) + 255) & ~uintptr_t(255));
+  const TcAux lay = tc_aux(p, a.K);
+  t.rows = reinterpret_cast<int32_t*>(aux + lay.rows);
+  t.counts = reinterpret_cast<int32_t*>(aux + lay.counts);
+  t.chunk_counts = reinterpret_cast<int32_t*>(aux + lay.chunk_counts);
+  t.pack = reinterpret_cast<uint16_t*>(aux + lay.pack);
+  t.split_b = xdt == SFX_F32 ? 1 : 0;
+  if (wdt == SFX_BF16) {
+    if (xdt == SFX_BF16) return launch_tc<__nv_bfloat16, __nv_bfloat16>(p, t, s);
+    if (xdt == SFX_F32) return launch_tc<__nv_bfloat16, float>(p, t, s);
+  } else if (wdt == SFX_F16) {
+    if (xdt == SFX_F16) return launch_tc<__half, __half>(p, t, s);
+    if (xdt == SFX_F32) return launch_tc<__half, float>(p, t, s);
+  }
+  return SFX_ERR_DTYPE;
+}
+
+}  // namespace sfx

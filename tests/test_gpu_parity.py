@@ -317,3 +317,44 @@ def test_workspace_shared_across_operations():
         want = O.masked_gemv(to64(x), O.magnitude_mask(to64(x), 0.7), to64(W))
         assert_close(to64(y), O.round_to(want, "f32"), f"gemv after other ops ({rep})")
     assert ws.status() == 0
+
+
+# ---------------------------------------------------------------- batch union on tensor cores
+
+@pytest.mark.parametrize("B,K,N,p,wdt,xdt,out", [
+    (4, 4096, 2048, 0.5, "bf16", "bf16", "bf16"),
+    (16, 1000, 264, 0.3, "f16", "f16", "f32"),     # ragged K and N (N % 128 != 0)
+    (8, 14336, 4096, 0.65, "bf16", "f32", "bf16"),  # fp32 inputs: hi + lo bf16 split
+    (5, 33, 136, 0.0, "bf16", "bf16", "f32"),       # tiny, dense
+    (16, 8192, 1024, 0.9, "bf16", "bf16", "bf16"),  # sparse union (1 - 0.9^16 = 81% rows)
+])
+def test_union_tensor_core_matches_oracle(B, K, N, p, wdt, xdt, out):
+    gemv_case(B, K, N, p, wdt, xdt=xdt, seed="tc", out=out)
+
+
+def test_union_tensor_core_equals_cuda_core_path():
+    B, K, N = 16, 4096, 3072
+    x = synth.eval_draw("tc-vs-cc", "x", B, K, "bf16")
+    W = dev(weights(K, N, "tc-vs-cc", "bf16"))
+    t = 0.9
+    y_tc = sb.sfx_sparse_gemv(dev(x), W, t=t, out_dtype=torch.float32)
+    y_cc = sb.sfx_sparse_gemv(dev(x), W, t=t, out_dtype=torch.float32,
+                              flags=sb.SFX_FLAG_CUDA_CORES)
+    assert_close(to64(y_tc), to64(y_cc), "tensor cores vs CUDA cores")
+
+
+def test_union_tensor_core_epilogues():
+    gemv_case(4, 2560, 1024, 0.4, "f16", out="f32", flags=sb.SFX_FLAG_GELU, seed="tc-gelu")
+    B, K, N = 6, 1024, 512
+    x = synth.eval_draw("tc-umask", "x", B, K, "bf16")
+    W = weights(K, N, "tc-umask", "bf16")
+    y = sb.sfx_sparse_gemv(dev(x), dev(W), t=1.1, flags=sb.SFX_FLAG_UNION_MASK,
+                           out_dtype=torch.float32)
+    u = O.union_mask(O.magnitude_mask(to64(x), 1.1))
+    want = O.masked_gemv(to64(x), np.broadcast_to(u, (B, K)), to64(W))
+    assert_close(to64(y), O.round_to(want, "f32"), "tc union-mask reading")
+
+
+@pytest.mark.parametrize("B", [4, 16])
+def test_ffn_swiglu_batched_tensor_cores(B):
+    ffn_case(B, 1024, 3584, 0.5, seed=f"ffn-b{B}")
