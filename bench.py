@@ -281,6 +281,185 @@ def capture(fn, stream):
     return g
 
 
+def graph_us(fns, stream, reps=5):
+    """Mean device time (us) of one call of `fns` (a list of callables replayed
+    round-robin, one per weight copy) captured in a CUDA graph."""
+    for f in fns:
+        f()
+    torch.cuda.synchronize()
+    g = capture(lambda: [f() for f in fns], stream)
+    g.replay()
+    ms = time_graph(g, reps, stream)
+    del g
+    return ms * 1e3 / (reps * len(fns))
+
+
+def copies_for(nbytes, floor=2):
+    """Weight copies needed so that one pass over them is >= 3x the 126 MB L2."""
+    return max(floor, math.ceil(400e6 / max(nbytes, 1)))
+
+
+def bench_other_workloads(stream, dev):
+    """The other workloads of the path, short graph-timed runs (not the headline)."""
+    from sparse_input_gemv_b200 import binding as sb
+    from sparse_input_gemv_b200 import synth
+    out = {}
+    ws = sb.Workspace(dev)
+    ws.reserve(256 << 20)
+
+    # single input-sparse GEMV: x fp16 [1 x 256], W fp16 [256 x 512], t_p for 50%
+    calib = synth.calib_draws("single", "x", 64, 256, "f16").to(dev)
+    t = sb.sfx_calibrate_thresholds(calib, [0.5], ws=ws)[0]
+    n = copies_for(256 * 512 * 2, floor=2)
+    Ws = [synth.normal((256, 512), synth.seed_of("single", "W", c), 0.02, "f16", dev) for c in range(n)]
+    x = synth.eval_draw("single", "x", 1, 256, "f16").to(dev)
+    y = torch.empty((1, 512), dtype=torch.float16, device=dev)
+    us = graph_us([lambda W=W: sb.sfx_sparse_gemv(x, W, t=t, y=y, ws=ws) for W in Ws[:64]], stream)
+    act = int((x.float().abs() > t).sum())
+    out["single_gemv_fp16_256x512_p50"] = {
+        "us": us, "active_rows": act, "gbs": (act * 1024 + 512 + 1024) / (us * 1e-6) / 1e9,
+        "note": "latency-bound: 128 KB of active weights; 64 distinct weight copies per graph"}
+    del Ws
+
+    # Phi-2-shaped GeLU FFN d=2560, ffn=10240, fp16: dense up + GeLU, top-k of |g h|
+    # (or a static GLASS mask), sparse down
+    d, f = 2560, 10240
+    n = copies_for(2 * d * f * 2)
+    W1 = [synth.normal((d, f), synth.seed_of("phi2", "W1", c), 0.02, "f16", dev) for c in range(n)]
+    W2 = [synth.normal((f, d), synth.seed_of("phi2", "W2", c), 0.02, "f16", dev) for c in range(n)]
+    x = synth.eval_draw("phi2", "x", 1, d, "f16").to(dev)
+    g = synth.normal((1, f), synth.seed_of("phi2", "g"), 1.0, "f32", dev)
+    sl = synth.abs_normal((1, f), synth.seed_of("phi2", "local"), device=dev)
+    sgl = synth.abs_normal((1, f), synth.seed_of("phi2", "global"), device=dev)
+    h = torch.empty((1, f), dtype=torch.float32, device=dev)
+    y = torch.empty((1, d), dtype=torch.float16, device=dev)
+    bitmap = torch.zeros((1, (f + 31) // 32), dtype=torch.int32, device=dev)
+    idx = torch.zeros((1, f), dtype=torch.int32, device=dev)
+    cnt = torch.zeros((1,), dtype=torch.int32, device=dev)
+    lib = sb.load()
+    import ctypes
+    P = lambda tns: ctypes.c_void_p(tns.data_ptr())
+
+    def select_gxo(k):
+        lib.sfx_mask_compact(P(h), sb.SFX_F32, 1, f, sb.SFX_SEL_TOPK_GXO, 0.0, k, P(g), None, 0.5,
+                             P(bitmap), P(idx), P(cnt), None, None, P(ws.buf), ws.buf.numel(),
+                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    phi = {}
+    for keep in (0.3, 0.5, 0.7):
+        k = int(keep * f + 0.5)
+        steps = []
+        for c in range(n):
+            def step(c=c, k=k):
+                sb.sfx_sparse_gemv(x, W1[c], flags=sb.SFX_FLAG_GELU, y=h, ws=ws)
+                select_gxo(k)
+                sb.sfx_sparse_gemv(h[0], W2[c], idx=idx[0], cnt=cnt, y=y[0], ws=ws)
+            steps.append(step)
+        us = graph_us(steps, stream)
+        nbytes = d * f * 2 + k * d * 2 + d * 2 + f * 4 * 3 + d * 2
+        # GLASS: the mask is fixed after prefill, so a decode step is up + down only
+        sb.sfx_mask_compact(None, sb.SFX_SEL_TOPK_GLASS, k=k, score_l=sl, score_g=sgl, lam=0.5, ws=ws)
+        gl = sb.sfx_mask_compact(None, sb.SFX_SEL_TOPK_GLASS, k=k, score_l=sl, score_g=sgl, lam=0.5,
+                                 ws=ws)
+        us_gl = graph_us([lambda c=c: (sb.sfx_sparse_gemv(x, W1[c], flags=sb.SFX_FLAG_GELU, y=h, ws=ws),
+                                       sb.sfx_sparse_gemv(h[0], W2[c], idx=gl["idx"][0],
+                                                          cnt=gl["cnt"], y=y[0], ws=ws))
+                          for c in range(n)], stream)
+        phi[f"keep{int(keep * 100)}"] = {"us_gxo": us, "us_glass_static_mask": us_gl,
+                                         "gbs_gxo": nbytes / (us * 1e-6) / 1e9}
+    out["phi2_gelu_ffn_fp16_topk"] = phi
+    del W1, W2
+
+    # MoE: 128 experts, d=2048, expert ffn=768, top-8, shared expert ffn=2048, bf16
+    E, d, f, fs, top = 128, 2048, 768, 2048, 8
+    WgT = synth.normal((E, f, d), synth.seed_of("moe", "WgT"), 0.02, "bf16", dev)
+    WuT = synth.normal((E, f, d), synth.seed_of("moe", "WuT"), 0.02, "bf16", dev)
+    Wd = synth.normal((E, f, d), synth.seed_of("moe", "Wd"), 0.02, "bf16", dev)
+    Sg = synth.normal((d, fs), synth.seed_of("moe", "Sg"), 0.02, "bf16", dev)
+    Su = synth.normal((d, fs), synth.seed_of("moe", "Su"), 0.02, "bf16", dev)
+    Sgu = sb.sfx_pack_gate_up(Sg, Su)
+    Sd = synth.normal((fs, d), synth.seed_of("moe", "Sd"), 0.02, "bf16", dev)
+    del Sg, Su
+    # per-expert thresholds from 16 calibration tokens routed to every expert
+    xc = synth.calib_draws("moe", "x", 16, d, "bf16").to(dev)
+    zl = torch.zeros((16, E), dtype=torch.float32, device=dev)
+    ninf = torch.full((E,), -math.inf, dtype=torch.float32, device=dev)
+    a_all = sb.sfx_moe_expert_sparse(xc, zl, WgT, WuT, Wd, ninf, E, want_a=True, ws=ws)["a"]
+    a_e = a_all.permute(1, 0, 2).contiguous()  # [E x 16 x ffn], experts in index order
+    moe = {}
+    for p in (0.5, 0.8, 0.9):
+        te = torch.tensor([sb.sfx_calibrate_thresholds(a_e[e], [p], ws=ws)[0] for e in range(E)],
+                          dtype=torch.float32, device=dev)
+        for B in (1, 4, 16):
+            xb = synth.eval_draw("moe", "x", B, d, "bf16").to(dev)
+            lg = synth.normal((B, E), synth.seed_of("moe", "logits", B), 1.0, "f32", dev)
+            yb = torch.empty((B, d), dtype=torch.bfloat16, device=dev)
+            r = sb.sfx_moe_expert_sparse(xb, lg, WgT, WuT, Wd, te, top, Ws_gu=Sgu, Ws_d=Sd, y=yb,
+                                         want_a=True, ws=ws)
+            sel = r["sel"].cpu().numpy()
+            a = r["a"]
+            experts = sorted({int(e) for e in sel.ravel()})
+            # bytes: dense gate rows of every active expert, kept up/down rows
+            # (union over the expert's tokens), shared expert, activations
+            kept = 0
+            for e in experts:
+                mask = torch.zeros(f, dtype=torch.bool, device=dev)
+                for t_ in range(B):
+                    for k_ in range(top):
+                        if sel[t_, k_] == e:
+                            mask |= a[t_, k_].abs() > te[e]
+                kept += int(mask.sum())
+            nbytes = len(experts) * f * d * 2 + kept * 2 * d * 2 + 3 * d * fs * 2 + 2 * B * d * 2
+            us = graph_us([lambda: sb.sfx_moe_expert_sparse(xb, lg, WgT, WuT, Wd, te, top, Ws_gu=Sgu,
+                                                            Ws_d=Sd, y=yb, ws=ws)], stream, reps=20)
+            moe[f"p{int(p * 100)}_b{B}"] = {"us": us, "gbs": nbytes / (us * 1e-6) / 1e9,
+                                            "active_experts": len(experts),
+                                            "kept_frac": kept / (len(experts) * f)}
+    out["moe_128x768_top8_shared2048"] = {"results": moe,
+                                          "note": "one MoE layer per graph replay; its 1.2 GB of expert "
+                                                  "weights exceed L2 but an expert's rows can stay "
+                                                  "cached between replays"}
+    del WgT, WuT, Wd, Sgu, Sd, a_all, a_e
+
+    # Llama-3-70B-shaped SwiGLU FFN d=8192, ffn=28672 bf16, batch 1/4/8/16,
+    # per-batch union of magnitude masks, sparsity 0..0.9
+    d, f = 8192, 28672
+    n = 2
+    Wgu = []
+    Wdn = []
+    for c in range(n):
+        Wg = synth.normal((d, f), synth.seed_of("l70", "Wg", c), 0.02, "bf16", dev)
+        Wu = synth.normal((d, f), synth.seed_of("l70", "Wu", c), 0.02, "bf16", dev)
+        Wgu.append(sb.sfx_pack_gate_up(Wg, Wu))
+        del Wg, Wu
+        Wdn.append(synth.normal((f, d), synth.seed_of("l70", "Wd", c), 0.02, "bf16", dev))
+    calib = synth.calib_draws("l70", "x", 64, d, "bf16").to(dev)
+    hc = torch.cat([sb.sfx_sparse_ffn_swiglu(calib[i:i + 16], Wgu[0], Wdn[0], want_h=True, ws=ws)["h"]
+                    for i in range(0, 64, 16)]).contiguous()
+    sweep = []
+    for B in (1, 4, 8, 16):
+        xb = synth.eval_draw("l70", "x", B, d, "bf16").to(dev)
+        yb = torch.empty((B, d), dtype=torch.bfloat16, device=dev)
+        hb = torch.empty((B, f), dtype=torch.float32, device=dev)
+        for p in [i / 10 for i in range(10)]:
+            t_in = sb.sfx_calibrate_thresholds(calib, [p], ws=ws)[0]
+            t_h = sb.sfx_calibrate_thresholds(hc, [p], ws=ws)[0]
+            r = sb.sfx_sparse_ffn_swiglu(xb, Wgu[0], Wdn[0], t_in, t_h, h=hb, y=yb,
+                                         want_bitmaps=True, ws=ws)
+            ux = int(np.unpackbits(r["bitmap_x"].view(torch.uint8).cpu().numpy().reshape(B, -1),
+                                   axis=1).any(0).sum())
+            uh = int(np.unpackbits(r["bitmap_h"].view(torch.uint8).cpu().numpy().reshape(B, -1),
+                                   axis=1).any(0).sum())
+            nbytes = ux * 2 * f * 2 + uh * d * 2 + B * (d * 2 * 2 + f * 4 * 2)
+            us = graph_us([lambda c=c: sb.sfx_sparse_ffn_swiglu(xb, Wgu[c], Wdn[c], t_in, t_h, h=hb,
+                                                                y=yb, ws=ws) for c in range(n)],
+                          stream, reps=3)
+            sweep.append({"batch": B, "sparsity": p, "us": us, "gbs": nbytes / (us * 1e-6) / 1e9,
+                          "union_frac_in": ux / d, "union_frac_h": uh / f})
+    out["llama3_70b_ffn_bf16"] = {"sweep": sweep, "dense_bytes": 3 * d * f * 2,
+                                  "note": "2 weight copies (2.8 GB) alternate between calls"}
+    return out
+
+
 # ---------------------------------------------------------------- CPU oracle leg
 
 def oracle_layer_pass(W, x, t):
@@ -399,6 +578,8 @@ def main():
     ap.add_argument("--sweep-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-other", action="store_true",
+                    help="skip the other workloads (single GEMV, Phi-2, MoE, Llama-3-70B FFN)")
     args = ap.parse_args()
 
     rank, local_rank, world = env_rank()
@@ -554,6 +735,10 @@ def main():
                "sample": f"{reps_o} passes of one layer (qkv, o, SwiGLU FFN) of the fp64 numpy "
                          f"oracle on layer 0 in {el:.1f} s"}
 
+    other = None
+    if rank == 0 and not args.no_other:
+        other = bench_other_workloads(stream, dev)
+
     e2e_val = bytes_step * K * world / (main_res["e2e_ms"] * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
@@ -577,6 +762,8 @@ def main():
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    if other is not None:
+        line["other_workloads"] = other
     del main_res["graph"]
     if rank == 0:
         print(json.dumps(line), flush=True)
