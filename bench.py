@@ -51,6 +51,20 @@ def env_rank():
             int(os.environ.get("WORLD_SIZE", 1)))
 
 
+def max_over_ranks(ms, dist=None, device=None):
+    """The slowest rank's time: replicas finish when the last one does."""
+    if dist is None:
+        return float(ms)
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_gbs(bytes_per_step, steps, world, ms):
+    """Whole-job GB/s of `world` replicas that each ran `steps` steps, the slowest in `ms`."""
+    return bytes_per_step * steps * world / (ms * 1e-3) / 1e9
+
+
 class ClockSampler:
     """Samples SM clock, max clock and clock-event reasons with NVML in a thread."""
 
@@ -369,56 +383,66 @@ def bench_other_workloads(stream, dev):
     out["phi2_gelu_ffn_fp16_topk"] = phi
     del W1, W2
 
-    # MoE: 128 experts, d=2048, expert ffn=768, top-8, shared expert ffn=2048, bf16
-    E, d, f, fs, top = 128, 2048, 768, 2048, 8
-    WgT = synth.normal((E, f, d), synth.seed_of("moe", "WgT"), 0.02, "bf16", dev)
-    WuT = synth.normal((E, f, d), synth.seed_of("moe", "WuT"), 0.02, "bf16", dev)
-    Wd = synth.normal((E, f, d), synth.seed_of("moe", "Wd"), 0.02, "bf16", dev)
-    Sg = synth.normal((d, fs), synth.seed_of("moe", "Sg"), 0.02, "bf16", dev)
-    Su = synth.normal((d, fs), synth.seed_of("moe", "Su"), 0.02, "bf16", dev)
-    Sgu = sb.sfx_pack_gate_up(Sg, Su)
-    Sd = synth.normal((fs, d), synth.seed_of("moe", "Sd"), 0.02, "bf16", dev)
-    del Sg, Su
-    # per-expert thresholds from 16 calibration tokens routed to every expert
+    # MoE: 128 experts, d=2048, expert ffn=768, top-8, shared expert ffn=2048, bf16.
+    # Four layers with their own weights (1.2 GB each) are replayed round-robin,
+    # so a replay reads its active experts from HBM, not from the 126 MB L2.
+    E, d, f, fs, top, L = 128, 2048, 768, 2048, 8, 4
+    layers = []
     xc = synth.calib_draws("moe", "x", 16, d, "bf16").to(dev)
     zl = torch.zeros((16, E), dtype=torch.float32, device=dev)
     ninf = torch.full((E,), -math.inf, dtype=torch.float32, device=dev)
-    a_all = sb.sfx_moe_expert_sparse(xc, zl, WgT, WuT, Wd, ninf, E, want_a=True, ws=ws)["a"]
-    a_e = a_all.permute(1, 0, 2).contiguous()  # [E x 16 x ffn], experts in index order
+    for li in range(L):
+        WgT = synth.normal((E, f, d), synth.seed_of("moe", "WgT", li), 0.02, "bf16", dev)
+        WuT = synth.normal((E, f, d), synth.seed_of("moe", "WuT", li), 0.02, "bf16", dev)
+        Wd = synth.normal((E, f, d), synth.seed_of("moe", "Wd", li), 0.02, "bf16", dev)
+        SgT = synth.normal((fs, d), synth.seed_of("moe", "SgT", li), 0.02, "bf16", dev)
+        SuT = synth.normal((fs, d), synth.seed_of("moe", "SuT", li), 0.02, "bf16", dev)
+        Sd = synth.normal((fs, d), synth.seed_of("moe", "Sd", li), 0.02, "bf16", dev)
+        # per-expert gate activations of 16 calibration tokens routed to every expert
+        a_all = sb.sfx_moe_expert_sparse(xc, zl, WgT, WuT, Wd, ninf, E, want_a=True, ws=ws)["a"]
+        a_e = a_all.permute(1, 0, 2).contiguous()  # [E x 16 x ffn], experts in index order
+        te = {p: torch.tensor([sb.sfx_calibrate_thresholds(a_e[e], [p], ws=ws)[0]
+                               for e in range(E)], dtype=torch.float32, device=dev)
+              for p in (0.5, 0.8, 0.9)}
+        layers.append((WgT, WuT, Wd, SgT, SuT, Sd, te))
+        del a_all, a_e
     moe = {}
     for p in (0.5, 0.8, 0.9):
-        te = torch.tensor([sb.sfx_calibrate_thresholds(a_e[e], [p], ws=ws)[0] for e in range(E)],
-                          dtype=torch.float32, device=dev)
         for B in (1, 4, 16):
             xb = synth.eval_draw("moe", "x", B, d, "bf16").to(dev)
-            lg = synth.normal((B, E), synth.seed_of("moe", "logits", B), 1.0, "f32", dev)
+            lgs = [synth.normal((B, E), synth.seed_of("moe", "logits", B, li), 1.0, "f32", dev)
+                   for li in range(L)]
             yb = torch.empty((B, d), dtype=torch.bfloat16, device=dev)
-            r = sb.sfx_moe_expert_sparse(xb, lg, WgT, WuT, Wd, te, top, Ws_gu=Sgu, Ws_d=Sd, y=yb,
-                                         want_a=True, ws=ws)
-            sel = r["sel"].cpu().numpy()
-            a = r["a"]
-            experts = sorted({int(e) for e in sel.ravel()})
-            # bytes: dense gate rows of every active expert, kept up/down rows
-            # (union over the expert's tokens), shared expert, activations
-            kept = 0
-            for e in experts:
-                mask = torch.zeros(f, dtype=torch.bool, device=dev)
-                for t_ in range(B):
-                    for k_ in range(top):
-                        if sel[t_, k_] == e:
-                            mask |= a[t_, k_].abs() > te[e]
-                kept += int(mask.sum())
-            nbytes = len(experts) * f * d * 2 + kept * 2 * d * 2 + 3 * d * fs * 2 + 2 * B * d * 2
-            us = graph_us([lambda: sb.sfx_moe_expert_sparse(xb, lg, WgT, WuT, Wd, te, top, Ws_gu=Sgu,
-                                                            Ws_d=Sd, y=yb, ws=ws)], stream, reps=20)
-            moe[f"p{int(p * 100)}_b{B}"] = {"us": us, "gbs": nbytes / (us * 1e-6) / 1e9,
-                                            "active_experts": len(experts),
-                                            "kept_frac": kept / (len(experts) * f)}
+            nbytes, n_exp, kept_all = 0, 0, 0
+            for li, (WgT, WuT, Wd, SgT, SuT, Sd, te) in enumerate(layers):
+                r = sb.sfx_moe_expert_sparse(xb, lgs[li], WgT, WuT, Wd, te[p], top, Ws_gT=SgT,
+                                             Ws_upT=SuT, Ws_d=Sd, y=yb, want_a=True, ws=ws)
+                sel = r["sel"].cpu().numpy()
+                a = r["a"]
+                experts = sorted({int(e) for e in sel.ravel()})
+                # bytes: dense gate rows of every active expert, kept up/down rows
+                # (union over the expert's tokens), shared expert, activations
+                kept = 0
+                for e in experts:
+                    mask = torch.zeros(f, dtype=torch.bool, device=dev)
+                    for t_ in range(B):
+                        for k_ in range(top):
+                            if sel[t_, k_] == e:
+                                mask |= a[t_, k_].abs() > te[p][e]
+                    kept += int(mask.sum())
+                nbytes += len(experts) * f * d * 2 + kept * 2 * d * 2 + 3 * d * fs * 2 + 2 * B * d * 2
+                n_exp += len(experts)
+                kept_all += kept
+            us = graph_us([lambda li=li, l=l: sb.sfx_moe_expert_sparse(
+                xb, lgs[li], l[0], l[1], l[2], l[6][p], top, Ws_gT=l[3], Ws_upT=l[4], Ws_d=l[5],
+                y=yb, ws=ws) for li, l in enumerate(layers)], stream, reps=20)
+            moe[f"p{int(p * 100)}_b{B}"] = {"us": us, "gbs": nbytes / L / (us * 1e-6) / 1e9,
+                                            "active_experts": n_exp / L,
+                                            "kept_frac": kept_all / (n_exp * f)}
     out["moe_128x768_top8_shared2048"] = {"results": moe,
-                                          "note": "one MoE layer per graph replay; its 1.2 GB of expert "
-                                                  "weights exceed L2 but an expert's rows can stay "
-                                                  "cached between replays"}
-    del WgT, WuT, Wd, Sgu, Sd, a_all, a_e
+                                          "note": "us per MoE layer; 4 layers with distinct "
+                                                  "weights replayed round-robin (HBM-resident)"}
+    del layers
 
     # Llama-3-70B-shaped SwiGLU FFN d=8192, ffn=28672 bf16, batch 1/4/8/16,
     # per-batch union of magnitude masks, sparsity 0..0.9
@@ -628,11 +652,7 @@ def main():
         if sampler:
             sampler.__exit__()
             res["clocks"] = sampler.summary()
-        if dist is not None:
-            tmax = torch.tensor([ms], device=dev)
-            dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-            ms = float(tmax.item())
-        res["ms"] = ms
+        res["ms"] = max_over_ranks(ms, dist, dev)
         res["bytes_step"] = stack.step_bytes()
         res["graph"] = g
         if e2e:
@@ -656,11 +676,7 @@ def main():
             end.record(stream)
             end.synchronize()
             ems = start.elapsed_time(end)
-            if dist is not None:
-                tmax = torch.tensor([ems], device=dev)
-                dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
-                ems = float(tmax.item())
-            res["e2e_ms"] = ems
+            res["e2e_ms"] = max_over_ranks(ems, dist, dev)
             res["h2d"] = sum(x.numel() * x.element_size() for x in xs)
             res["d2h"] = sum(y.numel() * y.element_size() for y in ys)
         return res
@@ -670,7 +686,7 @@ def main():
     ms = main_res["ms"]
     K = args.steps
     bytes_step = main_res["bytes_step"]
-    value = bytes_step * K * world / (ms * 1e-3) / 1e9
+    value = replica_gbs(bytes_step, K, world, ms)
     us_layer = ms * 1e3 / (K * args.layers)
 
     # per-kernel device times: each kernel alone, replayed over the 32 layers
@@ -739,7 +755,7 @@ def main():
     if rank == 0 and not args.no_other:
         other = bench_other_workloads(stream, dev)
 
-    e2e_val = bytes_step * K * world / (main_res["e2e_ms"] * 1e-3) / 1e9
+    e2e_val = replica_gbs(bytes_step, K, world, main_res["e2e_ms"])
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,

@@ -269,29 +269,33 @@ int sfx_pack_gate_up(const void* W_g, const void* W_u, int dt, int d, int ffn,
  *   a_j = SiLU(W_gT[e][j, :] . x_t)  (dense gate projection)
  *   m_j = |a_j| > t_e[e]             (one threshold pass)
  *   y_t += w_e * sum_{j: m_j} a_j (W_upT[e][j, :] . x_t) W_d[e][j, :]
- * reading only rows j of W_upT[e] and W_d[e] with m_j = 1. If Ws_gu is not
- * NULL, a dense shared SwiGLU expert (always on) is added:
- * y_t += SwiGLU(x_t; Ws_gu [d x 2 ffn_shared] interleaved, Ws_d [ffn_shared x d]).
- * All three expert matrices are stored one row per intermediate neuron
- * ([ffn x d] per expert), so each neuron's gate, up and down weights are
- * contiguous 2d-byte rows. Experts are combined into an fp32 accumulator with
- * atomics, so the last bits of y may differ between runs.
+ * reading only rows j of W_upT[e] and W_d[e] with m_j = 1. If Ws_gT is not
+ * NULL, a dense shared SwiGLU expert (always on, weight 1) is added:
+ * y_t += sum_j SiLU(Ws_gT[j, :] . x_t) (Ws_upT[j, :] . x_t) Ws_d[j, :].
+ * Every expert matrix, routed or shared, is stored one row per intermediate
+ * neuron ([ffn x d] per expert), so each neuron's gate, up and down weights
+ * are contiguous 2d-byte rows. Experts are combined into an fp32 accumulator
+ * with atomics, so the last bits of y may differ between runs.
  *
  *  x       (dev) [B x d] dtype dt (bf16 or f16), 16-byte aligned
  *  logits  (dev) [B x E] f32
  *  W_gT    (dev) [E x ffn x d]   W_upT (dev) [E x ffn x d]   W_d (dev) [E x ffn x d]
  *  t_e     (dev) [E] f32 per-expert thresholds (-INFINITY: dense expert)
+ *  Ws_gT, Ws_upT, Ws_d (dev, optional, all or none) [ffn_shared x d] dtype dt
  *  y       (dev) [B x d] dtype ydt
  *  a_out   (dev, optional) [B x top_k x ffn] f32 gate activations a, in each
  *          token's selection order; sel_out (dev, optional) [B x top_k] int32
  *          selected experts
  *  ws      (dev) sfx_workspace_bytes(SFX_OP_MOE, B, d, E, ffn, top_k, ffn_shared)
- * Limits: 1 <= B <= 16, 1 <= top_k <= E <= 1024, d % 8 == 0, ffn % 8 == 0.
+ * Limits: 1 <= B <= 16, 1 <= top_k <= E <= 1024, d % 8 == 0, ffn % 8 == 0,
+ * ffn_shared % 8 == 0,
+ * B * d <= 98304 (the expert kernel holds x of the batch in shared memory);
+ * violations return SFX_ERR_ARG / SFX_ERR_ALIGN before any launch.
  * ---------------------------------------------------------------------- */
 int sfx_moe_expert_sparse(const void* x, int dt, const float* logits, int B, int d, int E,
                           int ffn, int top_k, const void* W_gT, const void* W_upT,
-                          const void* W_d, const float* t_e, const void* Ws_gu,
-                          const void* Ws_d, int ffn_shared, void* y, int ydt,
+                          const void* W_d, const float* t_e, const void* Ws_gT,
+                          const void* Ws_upT, const void* Ws_d, int ffn_shared, void* y, int ydt,
                           float* a_out, int32_t* sel_out, int flags,
                           void* ws, size_t ws_bytes, void* stream);
 

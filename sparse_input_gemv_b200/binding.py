@@ -49,7 +49,7 @@ _SIGS = {
                                    _I, _VP, _SZ, _VP]),
     "sfx_pack_gate_up": (_I, [_VP, _VP, _I, _I, _I, _VP, _VP]),
     "sfx_moe_expert_sparse": (_I, [_VP, _I, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP,
-                                   _I, _VP, _I, _VP, _VP, _I, _VP, _SZ, _VP]),
+                                   _VP, _I, _VP, _I, _VP, _VP, _I, _VP, _SZ, _VP]),
 }
 EXPORTED = tuple(_SIGS)
 
@@ -285,17 +285,18 @@ def sfx_sparse_ffn_swiglu(x, W_gu, W_d, t_in=-math.inf, t_h=-math.inf, out_dtype
     return out
 
 
-def sfx_moe_expert_sparse(x, logits, W_gT, W_upT, W_d, t_e, top_k, Ws_gu=None, Ws_d=None,
-                          out_dtype=None, flags=0, want_a=False, y=None,
+def sfx_moe_expert_sparse(x, logits, W_gT, W_upT, W_d, t_e, top_k, Ws_gT=None, Ws_upT=None,
+                          Ws_d=None, out_dtype=None, flags=0, want_a=False, y=None,
                           ws: Workspace | None = None, stream=None):
     """MoE layer with intra-expert magnitude masks; returns dict(y[, a, sel]).
 
-    W_gT, W_upT, W_d: [E x ffn x d] (one row per intermediate neuron).
+    W_gT, W_upT, W_d: [E x ffn x d]; the optional shared expert Ws_gT, Ws_upT,
+    Ws_d: [ffn_shared x d] (every matrix one row per intermediate neuron).
     """
     squeeze = x.dim() == 1
     x2 = x[None] if squeeze else x
     lg = logits[None] if logits.dim() == 1 else logits
-    _need_cuda(x2, lg, W_gT, W_upT, W_d, t_e, Ws_gu, Ws_d)
+    _need_cuda(x2, lg, W_gT, W_upT, W_d, t_e, Ws_gT, Ws_upT, Ws_d)
     B, d = x2.shape
     E, ffn, _ = W_gT.shape
     W_g = W_gT
@@ -309,7 +310,8 @@ def sfx_moe_expert_sparse(x, logits, W_gT, W_upT, W_d, t_e, top_k, Ws_gu=None, W
     ws, buf = _ws(ws, sfx_workspace_bytes(SFX_OP_MOE, B, d, E, ffn, top_k, ffn_s), dev)
     _check("sfx_moe_expert_sparse", load().sfx_moe_expert_sparse(
         _ptr(x2), _DT[x2.dtype], _ptr(lg), B, d, E, ffn, top_k, _ptr(W_g), _ptr(W_upT), _ptr(W_d),
-        _ptr(t_e), _ptr(Ws_gu), _ptr(Ws_d), ffn_s, _ptr(y), _DT[y.dtype], _ptr(a), _ptr(sel),
+        _ptr(t_e), _ptr(Ws_gT), _ptr(Ws_upT), _ptr(Ws_d), ffn_s, _ptr(y), _DT[y.dtype], _ptr(a),
+        _ptr(sel),
         int(flags), _ptr(buf), buf.numel(), _stream(stream)))
     out = {"y": y[0] if squeeze else y}
     if want_a:

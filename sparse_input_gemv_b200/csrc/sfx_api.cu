@@ -277,25 +277,30 @@ int sfx_pack_gate_up(const void* W_g, const void* W_u, int dt, int d, int ffn, v
 }
 
 int sfx_moe_expert_sparse(const void* x, int dt, const float* logits, int B, int d, int E,
-                          int ffn, int top_k, const void* W_g, const void* W_upT, const void* W_d,
-                          const float* t_e, const void* Ws_gu, const void* Ws_d, int ffn_shared,
-                          void* y, int ydt, float* a_out, int32_t* sel_out, int flags, void* ws,
-                          size_t ws_bytes, void* stream) {
-  if (!x || !logits || !W_g || !W_upT || !W_d || !t_e || !y) return SFX_ERR_ARG;
-  if (B < 1 || B > 16 || E < 1 || E > 1024 || top_k < 1 || top_k > E || d < 8 || ffn < 8)
+                          int ffn, int top_k, const void* W_gT, const void* W_upT,
+                          const void* W_d, const float* t_e, const void* Ws_gT,
+                          const void* Ws_upT, const void* Ws_d, int ffn_shared, void* y, int ydt,
+                          float* a_out, int32_t* sel_out, int flags, void* ws, size_t ws_bytes,
+                          void* stream) {
+  if (!x || !logits || !W_gT || !W_upT || !W_d || !t_e || !y) return SFX_ERR_ARG;
+  if (B < 1 || B > 16 || E < 1 || E > 1024 || top_k < 1 || top_k > E || d < 8 || ffn < 8 ||
+      (long long)B * d > 98304)
     return SFX_ERR_ARG;
-  if ((Ws_gu == nullptr) != (Ws_d == nullptr) || (Ws_gu && ffn_shared < 4)) return SFX_ERR_ARG;
+  const bool shared = Ws_gT != nullptr;
+  if ((Ws_upT != nullptr) != shared || (Ws_d != nullptr) != shared || (shared && ffn_shared < 8))
+    return SFX_ERR_ARG;
   if (!(dt == SFX_F16 || dt == SFX_BF16) || !valid_dtype(ydt)) return SFX_ERR_DTYPE;
-  if (d % 8 != 0 || ffn % 8 != 0 || !aligned16(W_g) || !aligned16(W_upT) || !aligned16(W_d) ||
-      !aligned16(x) || (Ws_gu && (!aligned16(Ws_gu) || !aligned16(Ws_d) || ffn_shared % 4 != 0)))
+  if (d % 8 != 0 || ffn % 8 != 0 || !aligned16(W_gT) || !aligned16(W_upT) || !aligned16(W_d) ||
+      !aligned16(x) ||
+      (shared && (!aligned16(Ws_gT) || !aligned16(Ws_upT) || !aligned16(Ws_d) ||
+                  ffn_shared % 8 != 0)))
     return SFX_ERR_ALIGN;
-  const size_t need =
-      sfx_workspace_bytes(SFX_OP_MOE, B, d, E, ffn, top_k, Ws_gu ? ffn_shared : 0);
+  const size_t need = sfx_workspace_bytes(SFX_OP_MOE, B, d, E, ffn, top_k, shared ? ffn_shared : 0);
   if (!ws || ws_bytes < need) return SFX_ERR_WORKSPACE;
-  return run_moe(x, dt, logits, B, d, E, ffn, top_k, W_g, W_upT, W_d, t_e, Ws_gu, Ws_d,
-                 Ws_gu ? ffn_shared : 0, y, ydt, a_out, sel_out, flags,
+  return run_moe(x, dt, logits, B, d, E, ffn, top_k, W_gT, W_upT, W_d, t_e, Ws_gT, Ws_upT, Ws_d,
+                 shared ? ffn_shared : 0, y, ydt, a_out, sel_out, flags,
                  reinterpret_cast<unsigned char*>(ws) + kWsHeader, need - kWsHeader,
-                 reinterpret_cast<unsigned*>(ws), as_stream(stream));
+                 as_stream(stream));
 }
 
 }  // extern "C"

@@ -80,10 +80,10 @@ int run_calibrate(const void* calib, int dt, long long n, const long long* ranks
 // MoE (sfx_moe.cu)
 size_t moe_workspace_bytes(int B, int d, int E, int ffn, int top_k, int ffn_shared);
 int run_moe(const void* x, int dt, const float* logits, int B, int d, int E, int ffn, int top_k,
-            const void* W_g, const void* W_upT, const void* W_d, const float* t_e,
-            const void* Ws_gu, const void* Ws_d, int ffn_shared, void* y, int ydt,
-            float* a_out, int32_t* sel_out, int flags, unsigned char* ws_body, size_t body_bytes,
-            unsigned* status, cudaStream_t stream);
+            const void* W_gT, const void* W_upT, const void* W_d, const float* t_e,
+            const void* Ws_gT, const void* Ws_upT, const void* Ws_d, int ffn_shared, void* y,
+            int ydt, float* a_out, int32_t* sel_out, int flags, unsigned char* ws_body,
+            size_t body_bytes, cudaStream_t stream);
 
 // gate/up interleave (sfx_api.cu)
 int launch_pack_gate_up(const void* W_g, const void* W_u, int dt, int d, int ffn, void* W_gu,

@@ -103,9 +103,15 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* x, con
     for (int shift = 24; shift >= 0; shift -= 8) {
       for (int j = tid; j < 256; j += kMaskThreads) hist[j] = 0;
       __syncthreads();
-      for (int i = tid; i < K; i += kMaskThreads) {
-        const uint32_t key = keys[i];
-        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1u);
+      // warp-aggregated: the scores share a few leading bytes, so most lanes of a
+      // warp hit the same bin; one lane per distinct bin adds its group's count
+      for (int i0 = 0; i0 < K; i0 += kMaskThreads) {
+        const int i = i0 + tid;
+        const uint32_t key = i < K ? keys[i] : 0u;
+        const bool cand = i < K && (key & pmask) == prefix;
+        const uint32_t bin = cand ? ((key >> shift) & 255u) : 256u;
+        const unsigned same = __match_any_sync(0xffffffffu, bin);
+        if (cand && lane == __ffs(same) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(same));
       }
       __syncthreads();
       if (warp == 0) {

@@ -7,55 +7,63 @@
 // weights of active neurons; the router and the always-on shared expert are
 // unchanged.
 //
-// Launches per call:
-//  1. moe_route_kernel (one CTA): per token softmax over E logits, top-k by
-//     probability (ties to the lower expert index), weights renormalised over
-//     the selection (or raw); groups the selected (token, slot) pairs by
-//     expert (experts ascending, tokens ascending) and zeroes the fp32 output
-//     accumulator.
-//  2. moe_expert_kernel, grid (ffn / 32 neuron chunks) x (active experts):
-//       gate:  g_tj = W_gT[e][j, :] . x_t for the chunk's 32 neurons (dense,
-//              one warp per neuron row, 4 KB contiguous rows), a = SiLU(g);
-//       mask:  m_tj = |a_tj| > t_e[e];
-//       up:    u_tj = W_upT[e][j, :] . x_t, only for neurons some token keeps;
+// Every expert matrix, routed or shared, is stored one row per intermediate
+// neuron ([ffn x d]), so a neuron's gate, up and down weights are three
+// contiguous 2d-byte rows.
+//
+// Launches per call (the second with programmatic dependent launch):
+//  1. moe_route_kernel (one CTA, one warp per token): softmax over E logits,
+//     top-k by probability (ties to the lower expert index), weights
+//     renormalised over the selection (or raw); the selected (token, slot)
+//     pairs grouped by expert (experts ascending, tokens ascending); the fp32
+//     output accumulator zeroed.
+//  2. moe_expert_kernel, one persistent CTA per SM taking work items (the
+//     first by block index, the rest from an atomic counter): a chunk of the
+//     shared expert's neurons (all tokens, weight 1, no threshold; these items
+//     come first and do their gate and up work while routing still runs), or
+//     of one active routed expert's (its tokens, at most 16):
+//       gate:  g_tj = W_gT[e][j, :] . x_t for the chunk's neurons (dense; a
+//              16-neuron x 8-token tensor-core tile per warp and K slice; the
+//              chunk's rows are one contiguous block, prefetched to L2 when
+//              the item starts), a = SiLU(g);
+//       mask:  m_tj = |a_tj| > t_e[e] (then the kept up/down rows and the
+//              next item's gate block are prefetched to L2);
+//       up:    u_tj = W_upT[e][j, :] . x_t, only for neurons some token keeps
+//              (tensor-core tiles over the kept rows);
 //       down:  y_t += sum_j (w_te m_tj a_tj u_tj) W_d[e][j, :], reading only
-//              those rows; the CTA's contribution is added to the fp32
-//              accumulator with atomics (the combine order, hence the last
-//              bits of y, may vary between runs).
-//  3. the shared expert (if any): dense SwiGLU through the sparse GEMV path
-//     with threshold -inf (gate|up with the SiLU epilogue, then down), fp32.
-//  4. moe_finalize_kernel: y = accumulator (+ shared) in the output dtype.
+//              those rows; each warp adds its 256-column partial to the
+//              accumulator with 16-byte atomics (the combine order, hence the
+//              last bits of y, may vary between runs).
+//  3. moe_finalize_kernel: y = accumulator in the output dtype.
 #include "sfx_common.cuh"
 #include "sfx_internal.h"
 
 namespace sfx {
 
-constexpr int kMoeChunk = 32;        // intermediate neurons per CTA
-constexpr int kMaxMoeTokens = 16;    // tokens per call (each expert sees at most this many)
+constexpr int kMaxMoeTokens = 16;  // tokens per call (each expert sees at most this many)
+// the expert kernel stages x of all tokens of an item in shared memory
+constexpr long long kMaxMoeTokenElems = 98304;  // B * d (192 KB of bf16)
 
-__host__ __device__ constexpr int moe_threads(int be) { return be >= 8 ? 256 : 512; }
+constexpr int kMoeThreads = 256;  // expert CTAs: two per SM where shared memory allows
+constexpr int kMoeChunkMax = 64;  // intermediate neurons per work item, at most
 
 // ---------------------------------------------------------------- workspace layout
 
 struct MoeWs {
-  int32_t* sel;       // [B x top_k] selected experts, selection order
-  float* wsel;        // [B x top_k] routing weights
-  int32_t* n_active;  // [1]
+  int32_t* n_active;   // [1]
+  int32_t* next_item;  // [1] work-item counter of the expert grid
   int32_t* active;    // [max_active] active experts, ascending
   int32_t* tok_off;   // [max_active + 1]
   int32_t* tok;       // [B x top_k] token of each grouped pair
   int32_t* slot;      // [B x top_k] selection slot of each grouped pair
   float* tokw;        // [B x top_k] routing weight of each grouped pair
   float* acc;         // [B x d] fp32 output accumulator
-  float* hs;          // [B x ffn_shared] shared-expert h
-  float* ys;          // [B x d] shared-expert output
-  unsigned char* gemv;  // partial sums of the shared-expert GEMVs
 };
 
 static size_t al256(size_t v) { return (v + 255) / 256 * 256; }
 
-// Carves the layout from `body`; returns the bytes used before the GEMV area.
-static size_t carve_moe(unsigned char* body, int B, int d, int E, int top_k, int ffn_s, MoeWs* w) {
+// Carves the layout from `body`; returns the bytes it takes.
+static size_t carve_moe(unsigned char* body, int B, int d, int E, int top_k, MoeWs* w) {
   const int pairs = B * top_k;
   const int max_active = pairs < E ? pairs : E;
   size_t off = 0;
@@ -65,77 +73,70 @@ static size_t carve_moe(unsigned char* body, int B, int d, int E, int top_k, int
     return body ? body + at : nullptr;
   };
   MoeWs v;
-  v.sel = reinterpret_cast<int32_t*>(take((size_t)pairs * 4));
-  v.wsel = reinterpret_cast<float*>(take((size_t)pairs * 4));
   v.n_active = reinterpret_cast<int32_t*>(take(4));
+  v.next_item = reinterpret_cast<int32_t*>(take(4));
   v.active = reinterpret_cast<int32_t*>(take((size_t)max_active * 4));
   v.tok_off = reinterpret_cast<int32_t*>(take((size_t)(max_active + 1) * 4));
   v.tok = reinterpret_cast<int32_t*>(take((size_t)pairs * 4));
   v.slot = reinterpret_cast<int32_t*>(take((size_t)pairs * 4));
   v.tokw = reinterpret_cast<float*>(take((size_t)pairs * 4));
   v.acc = reinterpret_cast<float*>(take((size_t)B * d * 4));
-  v.hs = reinterpret_cast<float*>(take((size_t)B * (ffn_s > 0 ? ffn_s : 1) * 4));
-  v.ys = reinterpret_cast<float*>(take((size_t)B * d * 4));
-  v.gemv = body ? body + off : nullptr;
   if (w) *w = v;
   return off;
 }
 
 size_t moe_workspace_bytes(int B, int d, int E, int ffn, int top_k, int ffn_shared) {
   (void)ffn;
-  const size_t head = carve_moe(nullptr, B, d, E, top_k, ffn_shared, nullptr);
-  size_t g = 0;
-  if (ffn_shared > 0) {
-    const size_t g1 = gemv_workspace_bytes(d, 2LL * ffn_shared, B);
-    const size_t g2 = gemv_workspace_bytes(ffn_shared, d, B);
-    g = g1 > g2 ? g1 : g2;
-  }
-  return head + g;
+  (void)ffn_shared;
+  return carve_moe(nullptr, B, d, E, top_k, nullptr);
 }
 
 // ---------------------------------------------------------------- 1. routing
 
-__global__ void __launch_bounds__(1024) moe_route_kernel(const float* logits, int B, int E,
-                                                         int top_k, int renorm, int d, MoeWs w) {
-  extern __shared__ float s_z[];  // [E]
-  __shared__ float s_red[32];
-  __shared__ int s_redi[32];
-  __shared__ int s_cnt[1024];     // per-expert pair counts (E <= 1024)
-  __shared__ int s_off[1025];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+// One warp per token keeps the token's logits in shared memory, reduces max and
+// softmax denominator with shuffles and takes the top-k by repeated warp
+// arg-max (largest logit, then lowest index -- softmax is monotone in the
+// logit, so this is the top-k by probability). The grouping by expert then
+// runs on shared memory: per-expert counts and token masks, one warp's scan
+// over experts, and each pair's rank among the earlier tokens of its expert.
+__global__ void __launch_bounds__(512) moe_route_kernel(const float* logits, int B, int E,
+                                                        int top_k, int renorm, int d, MoeWs w,
+                                                        int32_t* sel_out) {
+  extern __shared__ __align__(16) unsigned char s_raw[];
+  float* s_z = reinterpret_cast<float*>(s_raw);                  // [B x E] logits
+  int* s_sel = reinterpret_cast<int*>(s_z + (size_t)B * E);     // [B x top_k]
+  float* s_wsel = reinterpret_cast<float*>(s_sel + B * top_k);  // [B x top_k]
+  __shared__ int s_cnt[1024];  // per-expert pair counts (E <= 1024)
+  __shared__ int s_off[1024];  // first grouped position of each expert
+  __shared__ unsigned s_tokmask[1024];  // tokens (B <= 16) that selected each expert
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nthr = blockDim.x, pairs = B * top_k;
+  pdl_launch_dependents();  // the expert grid waits for this grid's results where it needs them
 
-  for (int i = tid; i < B * d; i += blockDim.x) w.acc[i] = 0.f;
-  for (int e = tid; e < E; e += blockDim.x) s_cnt[e] = 0;
-
-  for (int t = 0; t < B; ++t) {
-    __syncthreads();
-    for (int e = tid; e < E; e += blockDim.x) s_z[e] = logits[(long long)t * E + e];
-    __syncthreads();
-    // max logit and the softmax denominator over all experts
+  for (int i = tid; i < B * d; i += nthr) w.acc[i] = 0.f;
+  if (tid == 0) *w.next_item = 0;
+  for (int e = tid; e < E; e += nthr) {
+    s_cnt[e] = 0;
+    s_tokmask[e] = 0u;
+  }
+  if (warp < B) {
+    const int t = warp;
+    float* z = s_z + (size_t)t * E;
     float m = -INFINITY;
-    for (int e = tid; e < E; e += blockDim.x) m = fmaxf(m, s_z[e]);
+    for (int e = lane; e < E; e += 32) {
+      z[e] = logits[(size_t)t * E + e];
+      m = fmaxf(m, z[e]);
+    }
     for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (lane == 0) s_red[warp] = m;
-    __syncthreads();
-    m = s_red[0];
-    for (int i = 1; i < nw; ++i) m = fmaxf(m, s_red[i]);
-    __syncthreads();
     float den = 0.f;
-    for (int e = tid; e < E; e += blockDim.x) den += expf(s_z[e] - m);
+    for (int e = lane; e < E; e += 32) den += expf(z[e] - m);
     for (int o = 16; o; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    if (lane == 0) s_red[warp] = den;
-    __syncthreads();
-    den = 0.f;
-    for (int i = 0; i < nw; ++i) den += s_red[i];
-    __syncthreads();
-    // top-k by repeated arg-max (largest logit, then lowest index); softmax is
-    // monotone in the logit, so this is the top-k by probability
     float selsum = 0.f;
     for (int k = 0; k < top_k; ++k) {
       float bv = -INFINITY;
       int bi = 0x7fffffff;
-      for (int e = tid; e < E; e += blockDim.x) {
-        const float v = s_z[e];
+      for (int e = lane; e < E; e += 32) {
+        const float v = z[e];
         if (v > bv || (v == bv && e < bi)) { bv = v; bi = e; }
       }
       for (int o = 16; o; o >>= 1) {
@@ -143,309 +144,533 @@ __global__ void __launch_bounds__(1024) moe_route_kernel(const float* logits, in
         const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
         if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
       }
-      if (lane == 0) { s_red[warp] = bv; s_redi[warp] = bi; }
-      __syncthreads();
-      bv = s_red[0];
-      bi = s_redi[0];
-      for (int i = 1; i < nw; ++i) {
-        if (s_red[i] > bv || (s_red[i] == bv && s_redi[i] < bi)) { bv = s_red[i]; bi = s_redi[i]; }
-      }
       const float pe = expf(bv - m);
       selsum += pe;
-      if (tid == 0) {
-        w.sel[t * top_k + k] = bi;
-        w.wsel[t * top_k + k] = pe;  // scaled below
-        s_cnt[bi] += 1;
-        s_z[bi] = -INFINITY;  // taken
+      if (lane == 0) {
+        s_sel[t * top_k + k] = bi;
+        s_wsel[t * top_k + k] = pe;  // scaled below
+        z[bi] = -INFINITY;           // taken
       }
-      __syncthreads();
+      __syncwarp();
     }
-    if (tid < top_k) w.wsel[t * top_k + tid] /= (renorm ? selsum : den);
+    const float norm = renorm ? selsum : den;
+    for (int k = lane; k < top_k; k += 32) {
+      s_wsel[t * top_k + k] /= norm;
+      if (sel_out) sel_out[t * top_k + k] = s_sel[t * top_k + k];
+    }
   }
   __syncthreads();
-  // group pairs by expert: ascending experts, tokens ascending within one
-  if (tid == 0) {
+  for (int q = tid; q < pairs; q += nthr) {
+    atomicAdd(&s_cnt[s_sel[q]], 1);
+    atomicOr(&s_tokmask[s_sel[q]], 1u << (q / top_k));
+  }
+  __syncthreads();
+  // active experts ascending and their first grouped positions (warp scan)
+  if (warp == 0) {
     int na = 0, off = 0;
-    for (int e = 0; e < E; ++e) {
-      if (s_cnt[e] > 0) {
-        w.active[na] = e;
-        w.tok_off[na] = off;
-        s_off[e] = off;
-        off += s_cnt[e];
-        ++na;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const int c = (e < E) ? s_cnt[e] : 0;
+      const unsigned act = __ballot_sync(0xffffffffu, c > 0);
+      int v = c;  // inclusive scan of the counts
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
       }
+      const int excl = off + v - c;
+      if (c > 0) {
+        const int ai = na + __popc(act & lanemask_lt());
+        w.active[ai] = e;
+        w.tok_off[ai] = excl;
+      }
+      if (e < E) s_off[e] = excl;
+      off += __shfl_sync(0xffffffffu, v, 31);
+      na += __popc(act);
     }
-    w.tok_off[na] = off;
-    *w.n_active = na;
-    for (int t = 0; t < B; ++t)
-      for (int k = 0; k < top_k; ++k) {
-        const int e = w.sel[t * top_k + k];
-        const int q = s_off[e]++;
-        w.tok[q] = t;
-        w.slot[q] = k;
-        w.tokw[q] = w.wsel[t * top_k + k];
-      }
+    if (lane == 0) {
+      w.tok_off[na] = off;
+      *w.n_active = na;
+    }
+  }
+  __syncthreads();
+  // pair q = (token t, slot k) goes after the earlier tokens of its expert (a
+  // token selects an expert at most once)
+  for (int q = tid; q < pairs; q += nthr) {
+    const int e = s_sel[q], t = q / top_k;
+    const int pos = s_off[e] + __popc(s_tokmask[e] & ((1u << t) - 1u));
+    w.tok[pos] = t;
+    w.slot[pos] = q % top_k;
+    w.tokw[pos] = s_wsel[q];
   }
 }
 
 // ---------------------------------------------------------------- 2. experts
 
+// Pointers of one expert kind: the routed stack [E x ffn x d] or the shared expert.
 template <typename TW>
-__device__ __forceinline__ void load_x8(const TW* x, float (&v)[8]) {
-  const uint4 q = __ldg(reinterpret_cast<const uint4*>(x));
-  unpack8(q, v, TW());
+struct ExpertMats {
+  const TW* gT;
+  const TW* upT;
+  const TW* d;
+};
+
+// Work items: 0 .. n_shared-1 are the shared expert's chunks of ch_s neurons,
+// then (active expert p, chunk c) with ch neurons, in order of p. A routed
+// neuron costs its gate row plus, at about half kept, one up and one down row;
+// a shared neuron costs all three rows, so shared chunks are 2/3 as long.
+struct MoeItems {
+  int ch, ch_s;    // neurons per routed / shared item
+  int n_chunks;    // items per routed expert
+  int n_shared;    // shared-expert items
+  int n_total;     // n_shared + max_active * n_chunks
+};
+
+struct MoeItem {
+  bool shared;
+  int p, e, j0, nj;
+};
+
+// Decodes item `it`; false for a routed item past the active experts (all
+// later items are past them too). Routed items need the routing results.
+__device__ __forceinline__ bool decode_item(int it, const MoeItems& I, int ffn, int ffn_s,
+                                            const MoeWs& w, MoeItem* out) {
+  MoeItem m;
+  m.shared = it < I.n_shared;
+  if (m.shared) {
+    m.p = -1;
+    m.e = 0;
+    m.j0 = it * I.ch_s;
+    m.nj = ffn_s - m.j0 < I.ch_s ? ffn_s - m.j0 : I.ch_s;
+  } else {
+    const int k = it - I.n_shared;
+    m.p = k / I.n_chunks;
+    if (m.p >= *w.n_active) return false;
+    m.e = w.active[m.p];
+    m.j0 = (k - m.p * I.n_chunks) * I.ch;
+    m.nj = ffn - m.j0 < I.ch ? ffn - m.j0 : I.ch;
+  }
+  *out = m;
+  return true;
 }
 
-template <typename TW, int BE>
-__global__ void __launch_bounds__(moe_threads(BE), BE == 1 ? 2 : 1)
-    moe_expert_kernel(const TW* __restrict__ x, int d, int ffn, int top_k,
-                      const TW* __restrict__ WgT, const TW* __restrict__ WupT,
-                      const TW* __restrict__ Wd, const float* __restrict__ t_e, float* a_out,
-                      MoeWs w) {
-  constexpr int kThreads = moe_threads(BE);
-  constexpr int kWarps = kThreads / 32;
-  __shared__ int s_tok[BE];
-  __shared__ int s_slot[BE];
-  __shared__ float s_w[BE];
-  __shared__ float s_a[kMoeChunk][BE];
-  __shared__ float s_v[kMoeChunk][BE];
-  __shared__ int s_list[kMoeChunk];
-  __shared__ int s_n;
+// D (16 x 8, f32) += A (16 x 16) B (16 x 8) on the tensor cores, A and B in the
+// storage dtype (both bf16 or both f16), one warp.
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1, __nv_bfloat16) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1, __half) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
 
-  const int p = blockIdx.y;
-  if (p >= *w.n_active) return;
-  const int e = w.active[p];
-  const int q0 = w.tok_off[p];
-  const int ne = w.tok_off[p + 1] - q0;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  if (tid < ne) {
-    s_tok[tid] = w.tok[q0 + tid];
-    s_slot[tid] = w.slot[q0 + tid];
-    s_w[tid] = w.tokw[q0 + tid];
+constexpr int kMoeTok = 16;           // tokens of one item: two 8-token MMA tiles
+constexpr int kXPad = 32;             // staged x row stride d + 32 elements (bank spread)
+
+// S[r][t] = W[row(r), :] . x_t for r < nrows (<= 64) and the item's ne tokens,
+// on the tensor cores: warps take (16-row tile, slice of K) pairs. Lane
+// (g = lane / 4, q = lane % 4) loads 16 bytes at k0 + 8q of rows g and g + 8 of
+// its tile and of tokens g and g + 8; the contraction runs over physical k, so
+// the fragment's logical k order need not match memory (A and B use the same
+// assignment). Partial sums go to s_part; the caller reduces them.
+template <typename TW, typename RowFn>
+__device__ __forceinline__ void mma_rows(const TW* __restrict__ Wm, RowFn row_of, int nrows,
+                                         int d, const TW* xs, int xstride, int ne,
+                                         float (*s_part)[16][kMoeTok], int* n_tiles_out,
+                                         int* ksplit_out) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, q = lane & 3;
+  constexpr int kWarps = kMoeThreads / 32;
+  const int n_tiles = (nrows + 15) >> 4;
+  const int ksplit = n_tiles > 0 ? kWarps / n_tiles : 0;
+  *n_tiles_out = n_tiles;
+  *ksplit_out = ksplit;
+  const int rt = n_tiles > 0 ? warp % n_tiles : 0, ks = n_tiles > 0 ? warp / n_tiles : kWarps;
+  if (ks >= ksplit) return;
+  const int nblk = (d + 31) >> 5;
+  const int per = (nblk + ksplit - 1) / ksplit;
+  const int blk0 = ks * per, blk1 = blk0 + per < nblk ? blk0 + per : nblk;
+  const int r0 = rt * 16 + g, r1 = r0 + 8;
+  const TW* p0 = r0 < nrows ? Wm + row_of(r0) * (long long)d : nullptr;
+  const TW* p1 = r1 < nrows ? Wm + row_of(r1) * (long long)d : nullptr;
+  const bool t0 = g < ne, t1 = g + 8 < ne, two = ne > 8;
+  const TW* x0 = xs + (long long)g * xstride;
+  const TW* x1 = xs + (long long)(g + 8) * xstride;
+  float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  constexpr int U = 4;  // 32-element blocks in flight per lane (2 rows x 16 B each)
+  for (int b = blk0; b < blk1; b += U) {
+    uint4 wa[U], wb[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int k = (b + u) * 32 + 8 * q;
+      const bool ok = b + u < blk1 && k < d;
+      wa[u] = (ok && p0) ? __ldcs(reinterpret_cast<const uint4*>(p0 + k)) : z;
+      wb[u] = (ok && p1) ? __ldcs(reinterpret_cast<const uint4*>(p1 + k)) : z;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int k = (b + u) * 32 + 8 * q;
+      if (b + u < blk1) {
+        const bool kin = k < d;
+        const uint4 xa = (kin && t0) ? *reinterpret_cast<const uint4*>(x0 + k) : z;
+        mma_16816(c0, wa[u].x, wb[u].x, wa[u].y, wb[u].y, xa.x, xa.y, TW());
+        mma_16816(c0, wa[u].z, wb[u].z, wa[u].w, wb[u].w, xa.z, xa.w, TW());
+        if (two) {
+          const uint4 xb = (kin && t1) ? *reinterpret_cast<const uint4*>(x1 + k) : z;
+          mma_16816(c1, wa[u].x, wb[u].x, wa[u].y, wb[u].y, xb.x, xb.y, TW());
+          mma_16816(c1, wa[u].z, wb[u].z, wa[u].w, wb[u].w, xb.z, xb.w, TW());
+        }
+      }
+    }
   }
-  __syncthreads();
-  const int j0 = blockIdx.x * kMoeChunk;
-  const long long erow = (long long)e * ffn;  // first row of expert e in [E x ffn x d]
-  const float te = t_e[e];
+  // D fragment: c[0], c[1] = (row g, tokens 2q, 2q+1); c[2], c[3] = (row g+8, same)
+  float(*sp)[kMoeTok] = s_part[warp];
+  sp[g][2 * q] = c0[0];
+  sp[g][2 * q + 1] = c0[1];
+  sp[g + 8][2 * q] = c0[2];
+  sp[g + 8][2 * q + 1] = c0[3];
+  sp[g][8 + 2 * q] = c1[0];
+  sp[g][8 + 2 * q + 1] = c1[1];
+  sp[g + 8][8 + 2 * q] = c1[2];
+  sp[g + 8][8 + 2 * q + 1] = c1[3];
+}
 
-  // dot products W[j, :] . x_t for the tokens of this expert, one warp per row
-  auto dot_rows = [&](const TW* Wm, int j, float (&out)[BE]) {
+// Sum of the K-slice partials of row r, token t (after mma_rows and a barrier).
+__device__ __forceinline__ float sum_parts(const float (*s_part)[16][kMoeTok], int n_tiles,
+                                           int ksplit, int r, int t) {
+  const int rt = r >> 4, rr = r & 15;
+  float s = 0.f;
+  for (int ks = 0; ks < ksplit; ++ks) s += s_part[ks * n_tiles + rt][rr][t];
+  return s;
+}
+
+// y_t += sum_k v[k][t] W_d[row(k), :] for NTOK tokens starting at t0, the
+// warps taking (256-column chunk, row phase) tasks; 16-byte atomics into acc.
+template <typename TW, int NTOK>
+__device__ __forceinline__ void down_pass(const TW* __restrict__ Wd, long long erow, int j0,
+                                          const int* s_list, int na, const float (*s_v)[kMoeTok],
+                                          int t0, const int* s_tok, int d, float* acc_out) {
+  constexpr int kWarps = kMoeThreads / 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nch = (d + 255) / 256;
+  const int nsplit = kWarps >= nch ? kWarps / nch : 1;
+  for (int task = warp; task < nch * nsplit; task += kWarps) {
+    const int chk = task % nch, par = task / nch;
+    const int col = chk * 256 + lane * 8;
+    if (col >= d) continue;
+    float acc[NTOK][8];
 #pragma unroll
-    for (int b = 0; b < BE; ++b) out[b] = 0.f;
-    const TW* row = Wm + (erow + j) * d;
-    for (int c0 = lane * 8; c0 < d; c0 += 256 * 4) {
-      uint4 wq[4];
+    for (int b = 0; b < NTOK; ++b)
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        if (c0 + u * 256 < d) wq[u] = __ldcs(reinterpret_cast<const uint4*>(row + c0 + u * 256));
+      for (int k = 0; k < 8; ++k) acc[b][k] = 0.f;
+    constexpr int L = NTOK <= 2 ? 4 : 2;  // rows in flight (registers: acc grows with NTOK)
+    for (int k0 = par; k0 < na; k0 += L * nsplit) {
+      uint4 wq[L];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = c0 + u * 256;
-        if (c < d) {
+      for (int u = 0; u < L; ++u) {
+        const int k = k0 + u * nsplit;
+        if (k < na)
+          wq[u] = __ldcs(reinterpret_cast<const uint4*>(Wd + (erow + j0 + s_list[k]) * d + col));
+      }
+#pragma unroll
+      for (int u = 0; u < L; ++u) {
+        const int k = k0 + u * nsplit;
+        if (k < na) {
           float wv[8];
           unpack8(wq[u], wv, TW());
 #pragma unroll
-          for (int b = 0; b < BE; ++b) {
-            if (b < ne) {
-              float xv[8];
-              load_x8(x + (long long)s_tok[b] * d + c, xv);
+          for (int b = 0; b < NTOK; ++b) {
+            const float vv = s_v[k][t0 + b];
 #pragma unroll
-              for (int k = 0; k < 8; ++k) out[b] = fmaf(wv[k], xv[k], out[b]);
-            }
+            for (int kk = 0; kk < 8; ++kk) acc[b][kk] = fmaf(vv, wv[kk], acc[b][kk]);
           }
         }
       }
     }
 #pragma unroll
-    for (int b = 0; b < BE; ++b)
-      for (int o = 16; o; o >>= 1) out[b] += __shfl_xor_sync(0xffffffffu, out[b], o);
-  };
-
-  // gate (dense) and SiLU
-  for (int jl = warp; jl < kMoeChunk; jl += kWarps) {
-    const int j = j0 + jl;
-    float g[BE];
-    if (j < ffn) {
-      dot_rows(WgT, j, g);
-    } else {
-#pragma unroll
-      for (int b = 0; b < BE; ++b) g[b] = 0.f;
-    }
-    if (lane == 0) {
-#pragma unroll
-      for (int b = 0; b < BE; ++b) {
-        if (b < ne) {
-          const float av = silu_f(g[b]);
-          s_a[jl][b] = av;
-          if (a_out && j < ffn)
-            a_out[((long long)s_tok[b] * top_k + s_slot[b]) * ffn + j] = av;
-        }
-      }
-    }
-  }
-  __syncthreads();
-  // threshold mask; neurons some token keeps, ascending
-  if (warp == 0) {
-    bool keep = false;
-    const int j = j0 + lane;
-    if (lane < kMoeChunk && j < ffn)
-      for (int b = 0; b < ne; ++b) keep |= fabsf(s_a[lane][b]) > te;
-    const unsigned bal = __ballot_sync(0xffffffffu, keep);
-    if (keep) s_list[__popc(bal & lanemask_lt())] = lane;
-    if (lane == 0) s_n = __popc(bal);
-  }
-  __syncthreads();
-  const int na = s_n;
-  // up projection for kept neurons; v = w_te * m * a * u
-  for (int k = warp; k < na; k += kWarps) {
-    const int jl = s_list[k];
-    float u[BE];
-    dot_rows(WupT, j0 + jl, u);
-    if (lane == 0) {
-#pragma unroll
-      for (int b = 0; b < BE; ++b) {
-        if (b < ne) {
-          const float av = s_a[jl][b];
-          s_v[k][b] = (fabsf(av) > te) ? s_w[b] * av * u[b] : 0.f;
-        }
-      }
-    }
-  }
-  __syncthreads();
-  if (na == 0) return;
-  // down projection over the kept rows: warps own 256-column chunks
-  const int nch = (d + 255) / 256;
-  for (int ch0 = 0; ch0 < nch; ch0 += kWarps) {
-    // one pass covers kWarps chunks (each warp one chunk, all kept rows)
-    const int ch = ch0 + warp;
-    const int col = ch * 256 + lane * 8;
-    float acc[BE][8];
-#pragma unroll
-    for (int b = 0; b < BE; ++b)
-#pragma unroll
-      for (int k = 0; k < 8; ++k) acc[b][k] = 0.f;
-    if (ch < nch && col < d) {
-      for (int k0 = 0; k0 < na; k0 += 4) {
-        uint4 wq[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (k0 + u < na)
-            wq[u] = __ldcs(reinterpret_cast<const uint4*>(Wd + (erow + j0 + s_list[k0 + u]) * d + col));
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (k0 + u < na) {
-            float wv[8];
-            unpack8(wq[u], wv, TW());
-#pragma unroll
-            for (int b = 0; b < BE; ++b) {
-              const float vv = (b < ne) ? s_v[k0 + u][b] : 0.f;
-#pragma unroll
-              for (int k = 0; k < 8; ++k) acc[b][k] = fmaf(vv, wv[k], acc[b][k]);
-            }
-          }
-        }
-      }
-#pragma unroll
-      for (int b = 0; b < BE; ++b) {
-        if (b < ne) {
-          float* dst = w.acc + (long long)s_tok[b] * d + col;
-#pragma unroll
-          for (int k = 0; k < 8; ++k) atomicAdd(dst + k, acc[b][k]);
-        }
-      }
+    for (int b = 0; b < NTOK; ++b) {
+      float4* dst = reinterpret_cast<float4*>(acc_out + (long long)s_tok[t0 + b] * d + col);
+      atomicAdd(dst, make_float4(acc[b][0], acc[b][1], acc[b][2], acc[b][3]));
+      atomicAdd(dst + 1, make_float4(acc[b][4], acc[b][5], acc[b][6], acc[b][7]));
     }
   }
 }
 
-// ---------------------------------------------------------------- 4. finalize
+// Persistent CTAs (as many as fit on the SMs): the first item is blockIdx.x, later ones come
+// from an atomic counter (gridDim.x + counter), so SMs that finish early take
+// more. While an item runs its up and down phases, the next item's gate block
+// is already on its way to L2.
+template <typename TW>
+__global__ void __launch_bounds__(kMoeThreads, 2)
+    moe_expert_kernel(const TW* __restrict__ x, int B, int d, int ffn, int ffn_s, MoeItems I,
+                      int top_k, ExpertMats<TW> R, ExpertMats<TW> S,
+                      const float* __restrict__ t_e, float* a_out, MoeWs w) {
+  constexpr int CH = kMoeChunkMax;
+  constexpr int kWarps = kMoeThreads / 32;
+  extern __shared__ __align__(16) unsigned char s_xraw[];  // [ne][d + kXPad] x of the item's tokens
+  __shared__ float s_part[kWarps][16][kMoeTok];             // K-slice partial sums
+  __shared__ float s_a[CH][kMoeTok];
+  __shared__ float s_v[CH][kMoeTok];
+  __shared__ int s_tok[kMoeTok];
+  __shared__ float s_w[kMoeTok];
+  __shared__ int s_slot[kMoeTok];
+  __shared__ int s_list[CH];
+  __shared__ int s_wcnt[CH / 32];
+  __shared__ int s_next;
 
-__global__ void moe_finalize_kernel(const float* acc, const float* ys, long long n, void* y, int ydt) {
-  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (long long)gridDim.x * blockDim.x) {
-    float v = acc[i];
-    if (ys) v += ys[i];
-    store_as(y, i, ydt, v);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const long long row_bytes = (long long)d * sizeof(TW);
+  const int xstride = d + kXPad;
+  TW* xs = reinterpret_cast<TW*>(s_xraw);
+  // routing results, the zeroed accumulator and the item counter come from the
+  // previous grid; every thread takes the same branches, so the wait is CTA-uniform
+  bool waited = false;
+  auto wait_routing = [&]() {
+    if (!waited) {
+      pdl_wait();
+      waited = true;
+    }
+  };
+  // the item's gate rows are one contiguous block: 16 KB bulk prefetches to L2
+  auto prefetch_gate = [&](const MoeItem& m) {
+    const TW* gm = m.shared ? S.gT : R.gT;
+    const char* base = reinterpret_cast<const char*>(
+        gm + ((long long)m.e * (m.shared ? ffn_s : ffn) + m.j0) * d);
+    const long long total = m.nj * row_bytes;
+    constexpr long long kPiece = 16384;
+    for (long long off = (long long)tid * kPiece; off < total; off += kMoeThreads * kPiece)
+      prefetch_l2_bulk(base + off, (uint32_t)(total - off < kPiece ? total - off : kPiece));
+  };
+
+  int it = blockIdx.x;
+  if (it >= I.n_total) return;
+  if (it >= I.n_shared) wait_routing();
+  MoeItem cur;
+  if (!decode_item(it, I, ffn, ffn_s, w, &cur)) return;
+  prefetch_gate(cur);
+
+  for (;;) {
+    const ExpertMats<TW> M = cur.shared ? S : R;
+    const int nf = cur.shared ? ffn_s : ffn;
+    const long long erow = (long long)cur.e * nf;  // first row of the expert in its stack
+    const int j0 = cur.j0, nj = cur.nj;
+    int ne;
+    float te;
+    __syncthreads();  // the previous item is done with the shared arrays
+    if (cur.shared) {
+      ne = B;
+      te = -INFINITY;
+      if (tid < B) {
+        s_tok[tid] = tid;
+        s_slot[tid] = -1;
+        s_w[tid] = 1.f;
+      }
+    } else {
+      const int q0 = w.tok_off[cur.p];
+      ne = w.tok_off[cur.p + 1] - q0;
+      te = t_e[cur.e];
+      if (tid < ne) {
+        s_tok[tid] = w.tok[q0 + tid];
+        s_slot[tid] = w.slot[q0 + tid];
+        s_w[tid] = w.tokw[q0 + tid];
+      }
+    }
+    __syncthreads();
+    // stage x of the item's tokens (d % 8 == 0: whole 16-byte words)
+    for (int i = tid; i < ne * (d / 8); i += kMoeThreads) {
+      const int b = i / (d / 8), c = i - b * (d / 8);
+      *reinterpret_cast<uint4*>(xs + (long long)b * xstride + c * 8) =
+          __ldg(reinterpret_cast<const uint4*>(x + (long long)s_tok[b] * d) + c);
+    }
+    __syncthreads();
+
+    // gate (dense) on the tensor cores, then SiLU
+    int n_tiles, ksplit;
+    mma_rows(M.gT, [&](int r) { return erow + j0 + r; }, nj, d, xs, xstride, ne, s_part,
+             &n_tiles, &ksplit);
+    __syncthreads();
+    for (int i = tid; i < nj * ne; i += kMoeThreads) {
+      const int r = i / ne, t = i - r * ne;
+      const float av = silu_f(sum_parts(s_part, n_tiles, ksplit, r, t));
+      s_a[r][t] = av;
+      if (a_out && !cur.shared)
+        a_out[((long long)s_tok[t] * top_k + s_slot[t]) * ffn + j0 + r] = av;
+    }
+    __syncthreads();
+    // threshold mask; the chunk's neurons some token keeps, ascending
+    bool keep = false;
+    unsigned bal = 0;
+    if (warp < CH / 32) {
+      if (tid < nj)
+        for (int t = 0; t < ne; ++t) keep |= fabsf(s_a[tid][t]) > te;
+      bal = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0) s_wcnt[warp] = __popc(bal);
+    }
+    __syncthreads();
+    int na = 0, woff = 0;
+#pragma unroll
+    for (int q = 0; q < CH / 32; ++q) {
+      woff += (q < warp) ? s_wcnt[q] : 0;
+      na += s_wcnt[q];
+    }
+    if (keep) s_list[woff + __popc(bal & lanemask_lt())] = tid;
+    // start the kept up and down rows towards L2, one bulk prefetch per row
+    __syncthreads();
+    for (int k = tid; k < 2 * na; k += kMoeThreads) {
+      const TW* m = (k < na) ? M.upT : M.d;
+      const int kk = (k < na) ? k : k - na;
+      prefetch_l2_bulk(m + (erow + j0 + s_list[kk]) * d, (uint32_t)row_bytes);
+    }
+    // the next item: take one from the counter, start its gate block too
+    wait_routing();
+    if (tid == 0) s_next = (int)gridDim.x + atomicAdd(w.next_item, 1);
+    // up projection for the kept neurons on the tensor cores
+    mma_rows(M.upT, [&](int r) { return erow + j0 + s_list[r]; }, na, d, xs, xstride, ne, s_part,
+             &n_tiles, &ksplit);
+    __syncthreads();
+    const int nxt_it = s_next;
+    MoeItem nxt;
+    const bool has_next = nxt_it < I.n_total && decode_item(nxt_it, I, ffn, ffn_s, w, &nxt);
+    if (has_next) prefetch_gate(nxt);
+    // v = w_te * m * a * u
+    for (int i = tid; i < na * ne; i += kMoeThreads) {
+      const int k = i / ne, t = i - k * ne;
+      const float av = s_a[s_list[k]][t];
+      s_v[k][t] = (fabsf(av) > te) ? s_w[t] * av * sum_parts(s_part, n_tiles, ksplit, k, t) : 0.f;
+    }
+    __syncthreads();
+    // down projection over the kept rows, four tokens per pass
+    for (int t0 = 0; t0 < ne && na > 0; t0 += 4) {
+      switch (ne - t0 < 4 ? ne - t0 : 4) {
+        case 1: down_pass<TW, 1>(M.d, erow, j0, s_list, na, s_v, t0, s_tok, d, w.acc); break;
+        case 2: down_pass<TW, 2>(M.d, erow, j0, s_list, na, s_v, t0, s_tok, d, w.acc); break;
+        case 3: down_pass<TW, 3>(M.d, erow, j0, s_list, na, s_v, t0, s_tok, d, w.acc); break;
+        default: down_pass<TW, 4>(M.d, erow, j0, s_list, na, s_v, t0, s_tok, d, w.acc); break;
+      }
+    }
+    if (!has_next) break;
+    cur = nxt;
+    it = nxt_it;
   }
+}
+
+// ---------------------------------------------------------------- 3. finalize
+
+__global__ void moe_finalize_kernel(const float* acc, long long n, void* y, int ydt) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x)
+    store_as(y, i, ydt, acc[i]);
 }
 
 // ---------------------------------------------------------------- host
 
-template <typename TW, int BE>
-static int launch_experts(const void* x, int d, int ffn, int top_k, int max_active,
-                          const void* WgT, const void* WupT, const void* Wd, const float* t_e,
-                          float* a_out, const MoeWs& w, cudaStream_t s) {
-  const dim3 grid((ffn + kMoeChunk - 1) / kMoeChunk, max_active);
-  moe_expert_kernel<TW, BE><<<grid, moe_threads(BE), 0, s>>>(
-      reinterpret_cast<const TW*>(x), d, ffn, top_k, reinterpret_cast<const TW*>(WgT),
-      reinterpret_cast<const TW*>(WupT), reinterpret_cast<const TW*>(Wd), t_e, a_out, w);
-  return cudaGetLastError() == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
+// Item sizes: the smallest routed chunk (>= 16 neurons) whose items fit one
+// per resident CTA; when even 64-neuron chunks need several rounds, 64.
+static MoeItems moe_items(int ffn, int ffn_s, int max_active, int slots) {
+  MoeItems I;
+  auto build = [&](int ch) {
+    I.ch = ch;
+    I.ch_s = (2 * ch + 1) / 3;
+    I.n_chunks = (ffn + ch - 1) / ch;
+    I.n_shared = ffn_s > 0 ? (ffn_s + I.ch_s - 1) / I.ch_s : 0;
+    I.n_total = I.n_shared + max_active * I.n_chunks;
+  };
+  for (int ch = 16; ch <= kMoeChunkMax; ++ch) {
+    build(ch);
+    if (I.n_total <= slots) return I;
+  }
+  build(kMoeChunkMax);
+  return I;
 }
 
 template <typename TW>
-static int launch_experts_t(int B, const void* x, int d, int ffn, int top_k, int max_active,
-                            const void* WgT, const void* WupT, const void* Wd, const float* t_e,
-                            float* a_out, const MoeWs& w, cudaStream_t s) {
-  if (B <= 1) return launch_experts<TW, 1>(x, d, ffn, top_k, max_active, WgT, WupT, Wd, t_e, a_out, w, s);
-  if (B <= 4) return launch_experts<TW, 4>(x, d, ffn, top_k, max_active, WgT, WupT, Wd, t_e, a_out, w, s);
-  if (B <= 8) return launch_experts<TW, 8>(x, d, ffn, top_k, max_active, WgT, WupT, Wd, t_e, a_out, w, s);
-  return launch_experts<TW, 16>(x, d, ffn, top_k, max_active, WgT, WupT, Wd, t_e, a_out, w, s);
+static int launch_experts(int B, const void* x, int d, int ffn, int ffn_s, int top_k,
+                          int max_active, const void* W_gT, const void* W_upT, const void* W_d,
+                          const void* Ws_gT, const void* Ws_upT, const void* Ws_d,
+                          const float* t_e, float* a_out, const MoeWs& w, cudaStream_t s) {
+  const ExpertMats<TW> R = {reinterpret_cast<const TW*>(W_gT), reinterpret_cast<const TW*>(W_upT),
+                            reinterpret_cast<const TW*>(W_d)};
+  const ExpertMats<TW> S = {reinterpret_cast<const TW*>(Ws_gT),
+                            reinterpret_cast<const TW*>(Ws_upT), reinterpret_cast<const TW*>(Ws_d)};
+  auto kern = moe_expert_kernel<TW>;
+  const size_t smem = (size_t)B * (d + kXPad) * sizeof(TW);  // x of an item's tokens (<= B)
+  static size_t configured = 0;  // one opt-in per kernel instantiation
+  if (smem > 48 * 1024 && smem > configured) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return SFX_ERR_CUDA;
+    configured = smem;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kMoeThreads, smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    return SFX_ERR_CUDA;
+  const int slots = sm_count() * per_sm;
+  const MoeItems I = moe_items(ffn, ffn_s, max_active, slots);
+  const int grid = I.n_total < slots ? I.n_total : slots;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(kMoeThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, reinterpret_cast<const TW*>(x), B, d, ffn, ffn_s, I, top_k,
+                         R, S, t_e, a_out, w) != cudaSuccess)
+    return SFX_ERR_CUDA;
+  return SFX_OK;
 }
 
 int run_moe(const void* x, int dt, const float* logits, int B, int d, int E, int ffn, int top_k,
             const void* W_gT, const void* W_upT, const void* W_d, const float* t_e,
-            const void* Ws_gu, const void* Ws_d, int ffn_shared, void* y, int ydt, float* a_out,
-            int32_t* sel_out, int flags, unsigned char* body, size_t body_bytes, unsigned* status,
-            cudaStream_t s) {
+            const void* Ws_gT, const void* Ws_upT, const void* Ws_d, int ffn_shared, void* y,
+            int ydt, float* a_out, int32_t* sel_out, int flags, unsigned char* body,
+            size_t body_bytes, cudaStream_t s) {
   (void)body_bytes;
-  if (B > kMaxMoeTokens || E > 1024) return SFX_ERR_UNSUPPORTED;
+  if (B > kMaxMoeTokens || E > 1024 || (long long)B * d > kMaxMoeTokenElems)
+    return SFX_ERR_UNSUPPORTED;
   MoeWs w;
-  carve_moe(body, B, d, E, top_k, ffn_shared, &w);
+  carve_moe(body, B, d, E, top_k, &w);
   const int renorm = (flags & SFX_FLAG_NO_RENORM) ? 0 : 1;
-  moe_route_kernel<<<1, 1024, (size_t)E * 4, s>>>(logits, B, E, top_k, renorm, d, w);
+  const size_t route_smem = (size_t)B * E * 4 + (size_t)B * top_k * 8;
+  if (route_smem > 48 * 1024) {
+    static size_t route_configured = 0;
+    if (route_smem > route_configured) {
+      if (cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)route_smem) != cudaSuccess)
+        return SFX_ERR_CUDA;
+      route_configured = route_smem;
+    }
+  }
+  const int route_threads = 32 * (B > 4 ? B : 4);
+  moe_route_kernel<<<1, route_threads, route_smem, s>>>(logits, B, E, top_k, renorm, d, w,
+                                                        sel_out);
   if (cudaGetLastError() != cudaSuccess) return SFX_ERR_CUDA;
-  if (sel_out &&
-      cudaMemcpyAsync(sel_out, w.sel, sizeof(int32_t) * B * top_k, cudaMemcpyDeviceToDevice, s) !=
-          cudaSuccess)
-    return SFX_ERR_CUDA;
   const int pairs = B * top_k;
   const int max_active = pairs < E ? pairs : E;
-  int rc = (dt == SFX_BF16)
-               ? launch_experts_t<__nv_bfloat16>(B, x, d, ffn, top_k, max_active, W_gT, W_upT,
-                                                 W_d, t_e, a_out, w, s)
-               : launch_experts_t<__half>(B, x, d, ffn, top_k, max_active, W_gT, W_upT, W_d,
-                                          t_e, a_out, w, s);
+  const int ffn_s = Ws_gT ? ffn_shared : 0;
+  const int rc = (dt == SFX_BF16)
+                     ? launch_experts<__nv_bfloat16>(B, x, d, ffn, ffn_s, top_k, max_active,
+                                                       W_gT, W_upT, W_d, Ws_gT, Ws_upT, Ws_d,
+                                                       t_e, a_out, w, s)
+                     : launch_experts<__half>(B, x, d, ffn, ffn_s, top_k, max_active, W_gT,
+                                                W_upT, W_d, Ws_gT, Ws_upT, Ws_d, t_e, a_out, w, s);
   if (rc != SFX_OK) return rc;
-  const float* ys = nullptr;
-  if (Ws_gu != nullptr) {
-    // dense shared SwiGLU expert through the GEMV path (threshold -inf)
-    GemvArgs g = {};
-    g.x = x;
-    g.W = Ws_gu;
-    g.y = w.hs;
-    g.status = status;
-    g.counters = reinterpret_cast<int32_t*>(reinterpret_cast<unsigned char*>(status) + kWsStatusBytes);
-    g.partials = reinterpret_cast<float*>(w.gemv);
-    g.K = d;
-    g.N = 2LL * ffn_shared;
-    g.B = B;
-    g.ydt = SFX_F32;
-    g.epi = EPI_SWIGLU;
-    g.t = -INFINITY;
-    rc = launch_sparse_gemv(dt, dt, plan_gemv(g.K, g.N, B, false), g, s, true);
-    if (rc != SFX_OK) return rc;
-    GemvArgs h = g;
-    h.x = w.hs;
-    h.W = Ws_d;
-    h.y = w.ys;
-    h.K = ffn_shared;
-    h.N = d;
-    h.epi = EPI_NONE;
-    rc = launch_sparse_gemv(dt, SFX_F32, plan_gemv(h.K, h.N, B, false), h, s, true);
-    if (rc != SFX_OK) return rc;
-    ys = w.ys;
-  }
   const long long n = (long long)B * d;
-  moe_finalize_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(w.acc, ys, n, y, ydt);
+  moe_finalize_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(w.acc, n, y, ydt);
   return cudaGetLastError() == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
 }
 

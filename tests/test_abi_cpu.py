@@ -110,5 +110,15 @@ def test_other_entry_points_reject_bad_arguments(lib):
     # MoE: top_k > E
     assert lib.sfx_moe_expert_sparse(VP(0x1000), sb.SFX_BF16, VP(0x2000), 1, 64, 4, 64, 5,
                                      VP(0x3000), VP(0x4000), VP(0x5000), VP(0x6000), None, None,
-                                     0, VP(0x7000), sb.SFX_BF16, None, None, 0, VP(0x8000),
+                                     None, 0, VP(0x7000), sb.SFX_BF16, None, None, 0, VP(0x8000),
                                      1 << 24, None) == -1
+    # MoE: the batch's x (B * d elements) must fit the expert kernel's shared memory
+    assert lib.sfx_moe_expert_sparse(VP(0x1000), sb.SFX_BF16, VP(0x2000), 16, 8192, 4, 64, 2,
+                                     VP(0x3000), VP(0x4000), VP(0x5000), VP(0x6000), None, None,
+                                     None, 0, VP(0x7000), sb.SFX_BF16, None, None, 0, VP(0x8000),
+                                     1 << 30, None) == -1
+    # MoE: the shared expert's three matrices come together or not at all
+    assert lib.sfx_moe_expert_sparse(VP(0x1000), sb.SFX_BF16, VP(0x2000), 1, 64, 4, 64, 2,
+                                     VP(0x3000), VP(0x4000), VP(0x5000), VP(0x6000), VP(0x9000),
+                                     None, VP(0xa000), 64, VP(0x7000), sb.SFX_BF16, None, None, 0,
+                                     VP(0x8000), 1 << 24, None) == -1

@@ -71,10 +71,11 @@ def run_case(name, B, E, d, ffn, top_k, ffn_s, p, flags=0, expert_subset=None):
         Wg64[e], WuT64[e], Wd64[e] = to64(Wg[e]), to64(WuT[e]), to64(Wd[e])
     te = expert_thresholds(name, Wg64, used, p, d, dtype)
     WgT = Wg.transpose(1, 2).contiguous()
-    Sgu = sb.sfx_pack_gate_up(sh[0], sh[1]) if sh else None
+    shT = [m.t().contiguous() for m in sh[:2]] if sh else [None, None]
     out = sb.sfx_moe_expert_sparse(x.cuda(), logits.cuda(), WgT, WuT, Wd,
-                                   torch.from_numpy(te).cuda(), top_k, Ws_gu=Sgu,
-                                   Ws_d=sh[2] if sh else None, flags=flags, want_a=True)
+                                   torch.from_numpy(te).cuda(), top_k, Ws_gT=shT[0],
+                                   Ws_upT=shT[1], Ws_d=sh[2] if sh else None, flags=flags,
+                                   want_a=True)
     sh64 = (to64(sh[0]), to64(sh[1]), to64(sh[2])) if sh else (None, None, None)
     want = O.moe_layer(to64(x), logits.numpy().astype(np.float64), Wg64, WuT64, Wd64,
                        te.astype(np.float64), top_k, *sh64, renormalize=renorm)
