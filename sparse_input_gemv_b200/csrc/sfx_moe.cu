@@ -573,8 +573,9 @@ __global__ void moe_finalize_kernel(const float* acc, long long n, void* y, int 
 
 // ---------------------------------------------------------------- host
 
-// Item sizes: the smallest routed chunk (>= 16 neurons) whose items fit one
-// per resident CTA; when even 64-neuron chunks need several rounds, 64.
+// Item sizes: the smallest routed chunk (>= 16 neurons) whose items, with the
+// shared expert's (2/3 as long), fit one round of the resident CTAs; when even
+// 64-neuron chunks need several rounds, 64.
 static MoeItems moe_items(int ffn, int ffn_s, int max_active, int slots) {
   MoeItems I;
   auto build = [&](int ch) {
