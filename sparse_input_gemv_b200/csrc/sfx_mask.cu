@@ -79,99 +79,171 @@ __global__ void __launch_bounds__(kMaskThreads) mask_compact_kernel(
   }
 }
 
-// Exact top-k of s_i = |fl32(x_i * g_i)| for one token per CTA.
+// Block-wide exclusive prefix sum of one int per thread (kMaskThreads threads);
+// *total gets the sum. Uses s_w[kMaskWarps + 1]; ends with a barrier.
+__device__ __forceinline__ int block_excl_scan(int v, int* s_w, int* total) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  if (lane == 31) s_w[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    const int wv = s_w[lane];  // kMaskWarps == 32
+    int winc = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, winc, o);
+      if (lane >= o) winc += n;
+    }
+    s_w[lane] = winc - wv;  // exclusive over warps
+    if (lane == 31) s_w[32] = winc;
+  }
+  __syncthreads();
+  const int r = s_w[warp] + inc - v;
+  *total = s_w[32];
+  __syncthreads();  // s_w may be reused
+  return r;
+}
+
+// Exact top-k of s_i = |fl32(x_i * g_i)| for one token per CTA. Thread t owns
+// the contiguous elements [t kpt, (t + 1) kpt); its j-th key sits in shared
+// memory at j * kMaskThreads + t (conflict-free passes). Three radix passes
+// over the key bits (11, 11 and 10 bits, most significant first; wide digits
+// keep the histogram atomics spread even though the scores share their
+// leading bits) find the k-th largest key T and how many keys equal to T are
+// kept; two block scans then give every thread its ties' ranks and its output
+// position, so the list comes out ascending with ties resolved toward the
+// lower index.
+constexpr int kTopkBins = 2048;  // 2 bins per thread
 template <typename TX>
-__global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* x, const float* g,
+__global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __restrict__ x,
+                                                                const float* __restrict__ g,
                                                                 int K, int k, uint32_t* bitmap,
                                                                 int32_t* idx, int32_t* cnt) {
-  extern __shared__ uint32_t keys[];  // [K]
-  __shared__ uint32_t hist[256];
-  __shared__ int s_tot[kMaskWarps];
-  __shared__ int s_tie[kMaskWarps];
+  extern __shared__ uint32_t keys[];  // [kpt][kMaskThreads], then the bitmap [ceil(K / 32)]
+  __shared__ uint32_t hist[kTopkBins];
+  __shared__ int s_w[kMaskWarps + 1];
   __shared__ uint32_t s_prefix;
   __shared__ uint32_t s_remaining;
   const int b = blockIdx.x;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x;
+  const int kpt = (K + kMaskThreads - 1) / kMaskThreads;
   const TX* xb = x + (long long)b * K;
   const float* gb = g + (long long)b * K;
-  for (int i = tid; i < K; i += kMaskThreads)
-    keys[i] = __float_as_uint(fabsf(__fmul_rn(to_f32(xb[i]), gb[i])));
-  __syncthreads();
+  // coalesced reads, eight per thread in flight; element i belongs to thread
+  // i / kpt, slot i % kpt
+  for (int i0 = 0; i0 < K; i0 += 8 * kMaskThreads) {
+    float xv[8], gv[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kMaskThreads + tid;
+      xv[u] = i < K ? to_f32(xb[i]) : 0.f;
+      gv[u] = i < K ? gb[i] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * kMaskThreads + tid;
+      if (i < K) {
+        const int t = i / kpt, j = i - t * kpt;
+        keys[j * kMaskThreads + t] = __float_as_uint(fabsf(__fmul_rn(xv[u], gv[u])));
+      }
+    }
+  }
+  const int e0 = tid * kpt;
+  const int nt = K - e0 < 0 ? 0 : (K - e0 < kpt ? K - e0 : kpt);  // this thread's elements
+  const int words = (K + 31) >> 5;
+  uint32_t* s_bits = keys + (size_t)kpt * kMaskThreads;
+  for (int w = tid; w < words; w += kMaskThreads) s_bits[w] = 0u;
 
   uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k;
+  // each thread owns bins 2 tid and 2 tid + 1: it zeroes them, and after a pass
+  // reads and re-zeroes them itself
+  hist[2 * tid] = 0u;
+  hist[2 * tid + 1] = 0u;
   if (k > 0) {
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int j = tid; j < 256; j += kMaskThreads) hist[j] = 0;
-      __syncthreads();
-      // warp-aggregated: the scores share a few leading bytes, so most lanes of a
-      // warp hit the same bin; one lane per distinct bin adds its group's count
-      for (int i0 = 0; i0 < K; i0 += kMaskThreads) {
-        const int i = i0 + tid;
-        const uint32_t key = i < K ? keys[i] : 0u;
-        const bool cand = i < K && (key & pmask) == prefix;
-        const uint32_t bin = cand ? ((key >> shift) & 255u) : 256u;
-        const unsigned same = __match_any_sync(0xffffffffu, bin);
-        if (cand && lane == __ffs(same) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(same));
+    constexpr int kShift[3] = {21, 10, 0};
+    constexpr int kBits[3] = {11, 11, 10};
+#pragma unroll
+    for (int ps = 0; ps < 3; ++ps) {
+      const int shift = kShift[ps];
+      const uint32_t dmask = (1u << kBits[ps]) - 1u;
+      __syncthreads();  // keys and zeroed bins (or the previous selection) visible
+      for (int j = 0; j < nt; ++j) {
+        const uint32_t key = keys[j * kMaskThreads + tid];
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
       }
       __syncthreads();
-      if (warp == 0) {
-        uint32_t h[8], local = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          h[j] = hist[lane * 8 + j];
-          local += h[j];
-        }
-        uint32_t incl = local;  // sum over lanes >= lane
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-          const uint32_t v = __shfl_down_sync(0xffffffffu, incl, off);
-          if (lane + off < 32) incl += v;
-        }
-        uint32_t c = incl - local;  // elements in higher bins
-#pragma unroll
-        for (int j = 7; j >= 0; --j) {
-          if (c < remaining && remaining <= c + h[j]) {
-            s_prefix = prefix | ((uint32_t)(lane * 8 + j) << shift);
-            s_remaining = remaining - c;
-          }
-          c += h[j];
-        }
+      // keys in bins above this thread's two: total minus the inclusive prefix
+      const uint32_t h0 = hist[2 * tid], h1 = hist[2 * tid + 1];
+      hist[2 * tid] = 0u;
+      hist[2 * tid + 1] = 0u;
+      const int local = (int)(h0 + h1);
+      int total;
+      const int before = block_excl_scan(local, s_w, &total);
+      uint32_t c = (uint32_t)(total - before - local);
+      if (c < remaining && remaining <= c + h1) {
+        s_prefix = prefix | ((uint32_t)(2 * tid + 1) << shift);
+        s_remaining = remaining - c;
+      }
+      c += h1;
+      if (c < remaining && remaining <= c + h0) {
+        s_prefix = prefix | ((uint32_t)(2 * tid) << shift);
+        s_remaining = remaining - c;
       }
       __syncthreads();
       prefix = s_prefix;
       remaining = s_remaining;
-      pmask |= 255u << shift;
-      __syncthreads();
+      pmask |= dmask << shift;
     }
-  }
-  const uint32_t T = prefix;  // k-th largest key; `remaining` ties at T are kept
-  const int words = (K + 31) >> 5;
-  int base = 0, ties_seen = 0;
-  for (int c0 = 0; c0 < K; c0 += kMaskThreads) {
-    const int i = c0 + tid;
-    const bool in = i < K;
-    const uint32_t key = in ? keys[i] : 0u;
-    const bool gt = in && k > 0 && key > T;
-    const bool eq = in && k > 0 && key == T;
-    const unsigned beq = __ballot_sync(0xffffffffu, eq);
-    if (lane == 0) s_tie[warp] = __popc(beq);
+  } else {
     __syncthreads();
-    int toff = 0, ttot = 0;
-#pragma unroll
-    for (int w = 0; w < kMaskWarps; ++w) {
-      const int c = s_tie[w];
-      toff += (w < warp) ? c : 0;
-      ttot += c;
-    }
-    const int tie_rank = ties_seen + toff + __popc(beq & lanemask_lt());
-    const bool act = gt || (eq && (uint32_t)tie_rank < remaining);
-    unsigned bal;
-    base += compact_chunk(act, i, base, idx ? idx + (long long)b * K : nullptr, s_tot, &bal);
-    ties_seen += ttot;
-    const int w0 = c0 + warp * 32;
-    if (bitmap && lane == 0 && w0 < K) bitmap[(long long)b * words + (w0 >> 5)] = bal;
   }
-  if (tid == 0) cnt[b] = base;
+  const uint32_t T = prefix;  // k-th largest key; `remaining` of the keys equal to T are kept
+  // ties before this thread, then this thread's kept count and output position
+  int n_gt = 0, n_eq = 0;
+  for (int j = 0; j < nt; ++j) {
+    const uint32_t key = keys[j * kMaskThreads + tid];
+    n_gt += (k > 0 && key > T);
+    n_eq += (k > 0 && key == T);
+  }
+  int tot;
+  const int eq_before = block_excl_scan(n_eq, s_w, &tot);
+  int eq_keep = (int)remaining - eq_before;
+  eq_keep = eq_keep < 0 ? 0 : (eq_keep > n_eq ? n_eq : eq_keep);
+  const int pos0 = block_excl_scan(n_gt + eq_keep, s_w, &tot);
+  int32_t* out = idx ? idx + (long long)b * K : nullptr;
+  int pos = pos0, eq_seen = 0;
+  uint32_t word = 0;  // bits of the current bitmap word gathered by this thread
+  int word_id = e0 >> 5;
+  for (int j = 0; j < nt; ++j) {
+    const int i = e0 + j;
+    const uint32_t key = keys[j * kMaskThreads + tid];
+    bool keep = false;
+    if (k > 0) {
+      if (key > T) {
+        keep = true;
+      } else if (key == T) {
+        keep = eq_seen < eq_keep;
+        ++eq_seen;
+      }
+    }
+    if (keep && out) out[pos++] = i;
+    if ((i >> 5) != word_id) {  // flush a finished word (shared with neighbours: OR)
+      if (word) atomicOr(&s_bits[word_id], word);
+      word = 0;
+      word_id = i >> 5;
+    }
+    if (keep) word |= 1u << (i & 31);
+  }
+  if (word) atomicOr(&s_bits[word_id], word);
+  __syncthreads();
+  if (bitmap)
+    for (int w = tid; w < words; w += kMaskThreads) bitmap[(long long)b * words + w] = s_bits[w];
+  if (tid == 0) cnt[b] = tot;
 }
 
 // q_j = #{i : key_i > key_j or (key_i == key_j and i < j)} by counting.
@@ -225,9 +297,11 @@ static int launch_threshold(const void* x, int B, int K, float t, uint32_t* bitm
 template <typename TX>
 static int launch_gxo(const void* x, const float* g, int B, int K, int k, uint32_t* bitmap,
                       int32_t* idx, int32_t* cnt, cudaStream_t s) {
-  const size_t smem = (size_t)K * 4;
+  const int kpt = (K + kMaskThreads - 1) / kMaskThreads;
+  const size_t smem = (size_t)kpt * kMaskThreads * 4 + (size_t)((K + 31) / 32) * 4;
   auto kern = topk_gxo_kernel<TX>;
-  if (smem > 48 * 1024 &&
+  // dynamic + ~8 KB static (the 2048-bin histogram) may pass the 48 KB default
+  if (smem + sizeof(uint32_t) * kTopkBins + 1024 > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
           cudaSuccess)
     return SFX_ERR_CUDA;

@@ -107,7 +107,8 @@ def test_threshold_mask_compact_bit_exact(dtype, B, K, t):
     assert np.array_equal(out["union_idx"][:uc].cpu().numpy(), uidx)
 
 
-@pytest.mark.parametrize("K,keep", [(10240, 0.3), (10240, 0.5), (10240, 0.7), (1000, 0.5), (37, 1.0)])
+@pytest.mark.parametrize("K,keep", [(10240, 0.3), (10240, 0.5), (10240, 0.7), (1000, 0.5), (37, 1.0),
+                                    (32768, 0.5), (32767, 0.1), (1025, 0.0)])
 def test_topk_gxo_bit_exact(K, keep):
     h = synth.normal((1, K), synth.seed_of("gxo", K, "h"), 1.0, "f32")
     g = synth.normal((1, K), synth.seed_of("gxo", K, "g"), 1.0, "f32")
