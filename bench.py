@@ -37,6 +37,7 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+OTHER_WORKLOADS = ("gemv", "phi2", "moe", "ffn70b")
 METRIC = "sparse FFN µs/layer and effective HBM GB/s vs sparsity at batch 1–16"
 D, FFN, NQKV = 4096, 14336, 6144
 WORKLOAD = ("Llama-3-8B-shaped decoder layer at batch 1: q/k/v/o 4096->4096/1024/1024/4096, "
@@ -313,174 +314,182 @@ def copies_for(nbytes, floor=2):
     return max(floor, math.ceil(400e6 / max(nbytes, 1)))
 
 
-def bench_other_workloads(stream, dev):
-    """The other workloads of the path, short graph-timed runs (not the headline)."""
+def bench_other_workloads(stream, dev, which=OTHER_WORKLOADS):
+    """The other workloads of the path, short graph-timed runs (not the headline).
+
+    `which` selects among "gemv" (single input-sparse GEMV), "phi2" (GeLU FFN with
+    GxO top-k / GLASS), "moe" (128-expert MoE) and "ffn70b" (batch sweep).
+    """
     from sparse_input_gemv_b200 import binding as sb
     from sparse_input_gemv_b200 import synth
     out = {}
     ws = sb.Workspace(dev)
     ws.reserve(256 << 20)
 
-    # single input-sparse GEMV: x fp16 [1 x 256], W fp16 [256 x 512], t_p for 50%
-    calib = synth.calib_draws("single", "x", 64, 256, "f16").to(dev)
-    t = sb.sfx_calibrate_thresholds(calib, [0.5], ws=ws)[0]
-    n = copies_for(256 * 512 * 2, floor=2)
-    Ws = [synth.normal((256, 512), synth.seed_of("single", "W", c), 0.02, "f16", dev) for c in range(n)]
-    x = synth.eval_draw("single", "x", 1, 256, "f16").to(dev)
-    y = torch.empty((1, 512), dtype=torch.float16, device=dev)
-    us = graph_us([lambda W=W: sb.sfx_sparse_gemv(x, W, t=t, y=y, ws=ws) for W in Ws[:64]], stream)
-    act = int((x.float().abs() > t).sum())
-    out["single_gemv_fp16_256x512_p50"] = {
-        "us": us, "active_rows": act, "gbs": (act * 1024 + 512 + 1024) / (us * 1e-6) / 1e9,
-        "note": "latency-bound: 128 KB of active weights; 64 distinct weight copies per graph"}
-    del Ws
+    if "gemv" in which:
+        # single input-sparse GEMV: x fp16 [1 x 256], W fp16 [256 x 512], t_p for 50%
+        calib = synth.calib_draws("single", "x", 64, 256, "f16").to(dev)
+        t = sb.sfx_calibrate_thresholds(calib, [0.5], ws=ws)[0]
+        n = copies_for(256 * 512 * 2, floor=2)
+        Ws = [synth.normal((256, 512), synth.seed_of("single", "W", c), 0.02, "f16", dev) for c in range(n)]
+        x = synth.eval_draw("single", "x", 1, 256, "f16").to(dev)
+        y = torch.empty((1, 512), dtype=torch.float16, device=dev)
+        us = graph_us([lambda W=W: sb.sfx_sparse_gemv(x, W, t=t, y=y, ws=ws) for W in Ws[:64]], stream)
+        act = int((x.float().abs() > t).sum())
+        out["single_gemv_fp16_256x512_p50"] = {
+            "us": us, "active_rows": act, "gbs": (act * 1024 + 512 + 1024) / (us * 1e-6) / 1e9,
+            "note": "latency-bound: 128 KB of active weights; 64 distinct weight copies per graph"}
+        del Ws
 
-    # Phi-2-shaped GeLU FFN d=2560, ffn=10240, fp16: dense up + GeLU, top-k of |g h|
-    # (or a static GLASS mask), sparse down
-    d, f = 2560, 10240
-    n = copies_for(2 * d * f * 2)
-    W1 = [synth.normal((d, f), synth.seed_of("phi2", "W1", c), 0.02, "f16", dev) for c in range(n)]
-    W2 = [synth.normal((f, d), synth.seed_of("phi2", "W2", c), 0.02, "f16", dev) for c in range(n)]
-    x = synth.eval_draw("phi2", "x", 1, d, "f16").to(dev)
-    g = synth.normal((1, f), synth.seed_of("phi2", "g"), 1.0, "f32", dev)
-    sl = synth.abs_normal((1, f), synth.seed_of("phi2", "local"), device=dev)
-    sgl = synth.abs_normal((1, f), synth.seed_of("phi2", "global"), device=dev)
-    h = torch.empty((1, f), dtype=torch.float32, device=dev)
-    y = torch.empty((1, d), dtype=torch.float16, device=dev)
-    bitmap = torch.zeros((1, (f + 31) // 32), dtype=torch.int32, device=dev)
-    idx = torch.zeros((1, f), dtype=torch.int32, device=dev)
-    cnt = torch.zeros((1,), dtype=torch.int32, device=dev)
-    lib = sb.load()
-    import ctypes
-    P = lambda tns: ctypes.c_void_p(tns.data_ptr())
+    if "phi2" in which:
+        # Phi-2-shaped GeLU FFN d=2560, ffn=10240, fp16: dense up + GeLU, top-k of |g h|
+        # (or a static GLASS mask), sparse down
+        d, f = 2560, 10240
+        n = copies_for(2 * d * f * 2)
+        W1 = [synth.normal((d, f), synth.seed_of("phi2", "W1", c), 0.02, "f16", dev) for c in range(n)]
+        W2 = [synth.normal((f, d), synth.seed_of("phi2", "W2", c), 0.02, "f16", dev) for c in range(n)]
+        x = synth.eval_draw("phi2", "x", 1, d, "f16").to(dev)
+        g = synth.normal((1, f), synth.seed_of("phi2", "g"), 1.0, "f32", dev)
+        sl = synth.abs_normal((1, f), synth.seed_of("phi2", "local"), device=dev)
+        sgl = synth.abs_normal((1, f), synth.seed_of("phi2", "global"), device=dev)
+        h = torch.empty((1, f), dtype=torch.float32, device=dev)
+        y = torch.empty((1, d), dtype=torch.float16, device=dev)
+        bitmap = torch.zeros((1, (f + 31) // 32), dtype=torch.int32, device=dev)
+        idx = torch.zeros((1, f), dtype=torch.int32, device=dev)
+        cnt = torch.zeros((1,), dtype=torch.int32, device=dev)
+        lib = sb.load()
+        import ctypes
+        P = lambda tns: ctypes.c_void_p(tns.data_ptr())
 
-    def select_gxo(k):
-        lib.sfx_mask_compact(P(h), sb.SFX_F32, 1, f, sb.SFX_SEL_TOPK_GXO, 0.0, k, P(g), None, 0.5,
-                             P(bitmap), P(idx), P(cnt), None, None, P(ws.buf), ws.buf.numel(),
-                             ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
-    phi = {}
-    for keep in (0.3, 0.5, 0.7):
-        k = int(keep * f + 0.5)
-        steps = []
+        def select_gxo(k):
+            lib.sfx_mask_compact(P(h), sb.SFX_F32, 1, f, sb.SFX_SEL_TOPK_GXO, 0.0, k, P(g), None, 0.5,
+                                 P(bitmap), P(idx), P(cnt), None, None, P(ws.buf), ws.buf.numel(),
+                                 ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        phi = {}
+        for keep in (0.3, 0.5, 0.7):
+            k = int(keep * f + 0.5)
+            steps = []
+            for c in range(n):
+                def step(c=c, k=k):
+                    sb.sfx_sparse_gemv(x, W1[c], flags=sb.SFX_FLAG_GELU, y=h, ws=ws)
+                    select_gxo(k)
+                    sb.sfx_sparse_gemv(h[0], W2[c], idx=idx[0], cnt=cnt, y=y[0], ws=ws)
+                steps.append(step)
+            us = graph_us(steps, stream)
+            nbytes = d * f * 2 + k * d * 2 + d * 2 + f * 4 * 3 + d * 2
+            # GLASS: the mask is fixed after prefill, so a decode step is up + down only
+            sb.sfx_mask_compact(None, sb.SFX_SEL_TOPK_GLASS, k=k, score_l=sl, score_g=sgl, lam=0.5, ws=ws)
+            gl = sb.sfx_mask_compact(None, sb.SFX_SEL_TOPK_GLASS, k=k, score_l=sl, score_g=sgl, lam=0.5,
+                                     ws=ws)
+            us_gl = graph_us([lambda c=c: (sb.sfx_sparse_gemv(x, W1[c], flags=sb.SFX_FLAG_GELU, y=h, ws=ws),
+                                           sb.sfx_sparse_gemv(h[0], W2[c], idx=gl["idx"][0],
+                                                              cnt=gl["cnt"], y=y[0], ws=ws))
+                              for c in range(n)], stream)
+            phi[f"keep{int(keep * 100)}"] = {"us_gxo": us, "us_glass_static_mask": us_gl,
+                                             "gbs_gxo": nbytes / (us * 1e-6) / 1e9}
+        out["phi2_gelu_ffn_fp16_topk"] = phi
+        del W1, W2
+
+    if "moe" in which:
+        # MoE: 128 experts, d=2048, expert ffn=768, top-8, shared expert ffn=2048, bf16.
+        # Four layers with their own weights (1.2 GB each) are replayed round-robin,
+        # so a replay reads its active experts from HBM, not from the 126 MB L2.
+        E, d, f, fs, top, L = 128, 2048, 768, 2048, 8, 4
+        layers = []
+        xc = synth.calib_draws("moe", "x", 16, d, "bf16").to(dev)
+        zl = torch.zeros((16, E), dtype=torch.float32, device=dev)
+        ninf = torch.full((E,), -math.inf, dtype=torch.float32, device=dev)
+        for li in range(L):
+            WgT = synth.normal((E, f, d), synth.seed_of("moe", "WgT", li), 0.02, "bf16", dev)
+            WuT = synth.normal((E, f, d), synth.seed_of("moe", "WuT", li), 0.02, "bf16", dev)
+            Wd = synth.normal((E, f, d), synth.seed_of("moe", "Wd", li), 0.02, "bf16", dev)
+            SgT = synth.normal((fs, d), synth.seed_of("moe", "SgT", li), 0.02, "bf16", dev)
+            SuT = synth.normal((fs, d), synth.seed_of("moe", "SuT", li), 0.02, "bf16", dev)
+            Sd = synth.normal((fs, d), synth.seed_of("moe", "Sd", li), 0.02, "bf16", dev)
+            # per-expert gate activations of 16 calibration tokens routed to every expert
+            a_all = sb.sfx_moe_expert_sparse(xc, zl, WgT, WuT, Wd, ninf, E, want_a=True, ws=ws)["a"]
+            a_e = a_all.permute(1, 0, 2).contiguous()  # [E x 16 x ffn], experts in index order
+            te = {p: torch.tensor([sb.sfx_calibrate_thresholds(a_e[e], [p], ws=ws)[0]
+                                   for e in range(E)], dtype=torch.float32, device=dev)
+                  for p in (0.5, 0.8, 0.9)}
+            layers.append((WgT, WuT, Wd, SgT, SuT, Sd, te))
+            del a_all, a_e
+        moe = {}
+        for p in (0.5, 0.8, 0.9):
+            for B in (1, 4, 16):
+                xb = synth.eval_draw("moe", "x", B, d, "bf16").to(dev)
+                lgs = [synth.normal((B, E), synth.seed_of("moe", "logits", B, li), 1.0, "f32", dev)
+                       for li in range(L)]
+                yb = torch.empty((B, d), dtype=torch.bfloat16, device=dev)
+                nbytes, n_exp, kept_all = 0, 0, 0
+                for li, (WgT, WuT, Wd, SgT, SuT, Sd, te) in enumerate(layers):
+                    r = sb.sfx_moe_expert_sparse(xb, lgs[li], WgT, WuT, Wd, te[p], top, Ws_gT=SgT,
+                                                 Ws_upT=SuT, Ws_d=Sd, y=yb, want_a=True, ws=ws)
+                    sel = r["sel"].cpu().numpy()
+                    a = r["a"]
+                    experts = sorted({int(e) for e in sel.ravel()})
+                    # bytes: dense gate rows of every active expert, kept up/down rows
+                    # (union over the expert's tokens), shared expert, activations
+                    kept = 0
+                    for e in experts:
+                        mask = torch.zeros(f, dtype=torch.bool, device=dev)
+                        for t_ in range(B):
+                            for k_ in range(top):
+                                if sel[t_, k_] == e:
+                                    mask |= a[t_, k_].abs() > te[p][e]
+                        kept += int(mask.sum())
+                    nbytes += len(experts) * f * d * 2 + kept * 2 * d * 2 + 3 * d * fs * 2 + 2 * B * d * 2
+                    n_exp += len(experts)
+                    kept_all += kept
+                us = graph_us([lambda li=li, l=l: sb.sfx_moe_expert_sparse(
+                    xb, lgs[li], l[0], l[1], l[2], l[6][p], top, Ws_gT=l[3], Ws_upT=l[4], Ws_d=l[5],
+                    y=yb, ws=ws) for li, l in enumerate(layers)], stream, reps=20)
+                moe[f"p{int(p * 100)}_b{B}"] = {"us": us, "gbs": nbytes / L / (us * 1e-6) / 1e9,
+                                                "active_experts": n_exp / L,
+                                                "kept_frac": kept_all / (n_exp * f)}
+        out["moe_128x768_top8_shared2048"] = {"results": moe,
+                                              "note": "us per MoE layer; 4 layers with distinct "
+                                                      "weights replayed round-robin (HBM-resident)"}
+        del layers
+
+    if "ffn70b" in which:
+        # Llama-3-70B-shaped SwiGLU FFN d=8192, ffn=28672 bf16, batch 1/4/8/16,
+        # per-batch union of magnitude masks, sparsity 0..0.9
+        d, f = 8192, 28672
+        n = 2
+        Wgu = []
+        Wdn = []
         for c in range(n):
-            def step(c=c, k=k):
-                sb.sfx_sparse_gemv(x, W1[c], flags=sb.SFX_FLAG_GELU, y=h, ws=ws)
-                select_gxo(k)
-                sb.sfx_sparse_gemv(h[0], W2[c], idx=idx[0], cnt=cnt, y=y[0], ws=ws)
-            steps.append(step)
-        us = graph_us(steps, stream)
-        nbytes = d * f * 2 + k * d * 2 + d * 2 + f * 4 * 3 + d * 2
-        # GLASS: the mask is fixed after prefill, so a decode step is up + down only
-        sb.sfx_mask_compact(None, sb.SFX_SEL_TOPK_GLASS, k=k, score_l=sl, score_g=sgl, lam=0.5, ws=ws)
-        gl = sb.sfx_mask_compact(None, sb.SFX_SEL_TOPK_GLASS, k=k, score_l=sl, score_g=sgl, lam=0.5,
-                                 ws=ws)
-        us_gl = graph_us([lambda c=c: (sb.sfx_sparse_gemv(x, W1[c], flags=sb.SFX_FLAG_GELU, y=h, ws=ws),
-                                       sb.sfx_sparse_gemv(h[0], W2[c], idx=gl["idx"][0],
-                                                          cnt=gl["cnt"], y=y[0], ws=ws))
-                          for c in range(n)], stream)
-        phi[f"keep{int(keep * 100)}"] = {"us_gxo": us, "us_glass_static_mask": us_gl,
-                                         "gbs_gxo": nbytes / (us * 1e-6) / 1e9}
-    out["phi2_gelu_ffn_fp16_topk"] = phi
-    del W1, W2
-
-    # MoE: 128 experts, d=2048, expert ffn=768, top-8, shared expert ffn=2048, bf16.
-    # Four layers with their own weights (1.2 GB each) are replayed round-robin,
-    # so a replay reads its active experts from HBM, not from the 126 MB L2.
-    E, d, f, fs, top, L = 128, 2048, 768, 2048, 8, 4
-    layers = []
-    xc = synth.calib_draws("moe", "x", 16, d, "bf16").to(dev)
-    zl = torch.zeros((16, E), dtype=torch.float32, device=dev)
-    ninf = torch.full((E,), -math.inf, dtype=torch.float32, device=dev)
-    for li in range(L):
-        WgT = synth.normal((E, f, d), synth.seed_of("moe", "WgT", li), 0.02, "bf16", dev)
-        WuT = synth.normal((E, f, d), synth.seed_of("moe", "WuT", li), 0.02, "bf16", dev)
-        Wd = synth.normal((E, f, d), synth.seed_of("moe", "Wd", li), 0.02, "bf16", dev)
-        SgT = synth.normal((fs, d), synth.seed_of("moe", "SgT", li), 0.02, "bf16", dev)
-        SuT = synth.normal((fs, d), synth.seed_of("moe", "SuT", li), 0.02, "bf16", dev)
-        Sd = synth.normal((fs, d), synth.seed_of("moe", "Sd", li), 0.02, "bf16", dev)
-        # per-expert gate activations of 16 calibration tokens routed to every expert
-        a_all = sb.sfx_moe_expert_sparse(xc, zl, WgT, WuT, Wd, ninf, E, want_a=True, ws=ws)["a"]
-        a_e = a_all.permute(1, 0, 2).contiguous()  # [E x 16 x ffn], experts in index order
-        te = {p: torch.tensor([sb.sfx_calibrate_thresholds(a_e[e], [p], ws=ws)[0]
-                               for e in range(E)], dtype=torch.float32, device=dev)
-              for p in (0.5, 0.8, 0.9)}
-        layers.append((WgT, WuT, Wd, SgT, SuT, Sd, te))
-        del a_all, a_e
-    moe = {}
-    for p in (0.5, 0.8, 0.9):
-        for B in (1, 4, 16):
-            xb = synth.eval_draw("moe", "x", B, d, "bf16").to(dev)
-            lgs = [synth.normal((B, E), synth.seed_of("moe", "logits", B, li), 1.0, "f32", dev)
-                   for li in range(L)]
+            Wg = synth.normal((d, f), synth.seed_of("l70", "Wg", c), 0.02, "bf16", dev)
+            Wu = synth.normal((d, f), synth.seed_of("l70", "Wu", c), 0.02, "bf16", dev)
+            Wgu.append(sb.sfx_pack_gate_up(Wg, Wu))
+            del Wg, Wu
+            Wdn.append(synth.normal((f, d), synth.seed_of("l70", "Wd", c), 0.02, "bf16", dev))
+        calib = synth.calib_draws("l70", "x", 64, d, "bf16").to(dev)
+        hc = torch.cat([sb.sfx_sparse_ffn_swiglu(calib[i:i + 16], Wgu[0], Wdn[0], want_h=True, ws=ws)["h"]
+                        for i in range(0, 64, 16)]).contiguous()
+        sweep = []
+        for B in (1, 4, 8, 16):
+            xb = synth.eval_draw("l70", "x", B, d, "bf16").to(dev)
             yb = torch.empty((B, d), dtype=torch.bfloat16, device=dev)
-            nbytes, n_exp, kept_all = 0, 0, 0
-            for li, (WgT, WuT, Wd, SgT, SuT, Sd, te) in enumerate(layers):
-                r = sb.sfx_moe_expert_sparse(xb, lgs[li], WgT, WuT, Wd, te[p], top, Ws_gT=SgT,
-                                             Ws_upT=SuT, Ws_d=Sd, y=yb, want_a=True, ws=ws)
-                sel = r["sel"].cpu().numpy()
-                a = r["a"]
-                experts = sorted({int(e) for e in sel.ravel()})
-                # bytes: dense gate rows of every active expert, kept up/down rows
-                # (union over the expert's tokens), shared expert, activations
-                kept = 0
-                for e in experts:
-                    mask = torch.zeros(f, dtype=torch.bool, device=dev)
-                    for t_ in range(B):
-                        for k_ in range(top):
-                            if sel[t_, k_] == e:
-                                mask |= a[t_, k_].abs() > te[p][e]
-                    kept += int(mask.sum())
-                nbytes += len(experts) * f * d * 2 + kept * 2 * d * 2 + 3 * d * fs * 2 + 2 * B * d * 2
-                n_exp += len(experts)
-                kept_all += kept
-            us = graph_us([lambda li=li, l=l: sb.sfx_moe_expert_sparse(
-                xb, lgs[li], l[0], l[1], l[2], l[6][p], top, Ws_gT=l[3], Ws_upT=l[4], Ws_d=l[5],
-                y=yb, ws=ws) for li, l in enumerate(layers)], stream, reps=20)
-            moe[f"p{int(p * 100)}_b{B}"] = {"us": us, "gbs": nbytes / L / (us * 1e-6) / 1e9,
-                                            "active_experts": n_exp / L,
-                                            "kept_frac": kept_all / (n_exp * f)}
-    out["moe_128x768_top8_shared2048"] = {"results": moe,
-                                          "note": "us per MoE layer; 4 layers with distinct "
-                                                  "weights replayed round-robin (HBM-resident)"}
-    del layers
-
-    # Llama-3-70B-shaped SwiGLU FFN d=8192, ffn=28672 bf16, batch 1/4/8/16,
-    # per-batch union of magnitude masks, sparsity 0..0.9
-    d, f = 8192, 28672
-    n = 2
-    Wgu = []
-    Wdn = []
-    for c in range(n):
-        Wg = synth.normal((d, f), synth.seed_of("l70", "Wg", c), 0.02, "bf16", dev)
-        Wu = synth.normal((d, f), synth.seed_of("l70", "Wu", c), 0.02, "bf16", dev)
-        Wgu.append(sb.sfx_pack_gate_up(Wg, Wu))
-        del Wg, Wu
-        Wdn.append(synth.normal((f, d), synth.seed_of("l70", "Wd", c), 0.02, "bf16", dev))
-    calib = synth.calib_draws("l70", "x", 64, d, "bf16").to(dev)
-    hc = torch.cat([sb.sfx_sparse_ffn_swiglu(calib[i:i + 16], Wgu[0], Wdn[0], want_h=True, ws=ws)["h"]
-                    for i in range(0, 64, 16)]).contiguous()
-    sweep = []
-    for B in (1, 4, 8, 16):
-        xb = synth.eval_draw("l70", "x", B, d, "bf16").to(dev)
-        yb = torch.empty((B, d), dtype=torch.bfloat16, device=dev)
-        hb = torch.empty((B, f), dtype=torch.float32, device=dev)
-        for p in [i / 10 for i in range(10)]:
-            t_in = sb.sfx_calibrate_thresholds(calib, [p], ws=ws)[0]
-            t_h = sb.sfx_calibrate_thresholds(hc, [p], ws=ws)[0]
-            r = sb.sfx_sparse_ffn_swiglu(xb, Wgu[0], Wdn[0], t_in, t_h, h=hb, y=yb,
-                                         want_bitmaps=True, ws=ws)
-            ux = int(np.unpackbits(r["bitmap_x"].view(torch.uint8).cpu().numpy().reshape(B, -1),
-                                   axis=1).any(0).sum())
-            uh = int(np.unpackbits(r["bitmap_h"].view(torch.uint8).cpu().numpy().reshape(B, -1),
-                                   axis=1).any(0).sum())
-            nbytes = ux * 2 * f * 2 + uh * d * 2 + B * (d * 2 * 2 + f * 4 * 2)
-            us = graph_us([lambda c=c: sb.sfx_sparse_ffn_swiglu(xb, Wgu[c], Wdn[c], t_in, t_h, h=hb,
-                                                                y=yb, ws=ws) for c in range(n)],
-                          stream, reps=3)
-            sweep.append({"batch": B, "sparsity": p, "us": us, "gbs": nbytes / (us * 1e-6) / 1e9,
-                          "union_frac_in": ux / d, "union_frac_h": uh / f})
-    out["llama3_70b_ffn_bf16"] = {"sweep": sweep, "dense_bytes": 3 * d * f * 2,
-                                  "note": "2 weight copies (2.8 GB) alternate between calls"}
+            hb = torch.empty((B, f), dtype=torch.float32, device=dev)
+            for p in [i / 10 for i in range(10)]:
+                t_in = sb.sfx_calibrate_thresholds(calib, [p], ws=ws)[0]
+                t_h = sb.sfx_calibrate_thresholds(hc, [p], ws=ws)[0]
+                r = sb.sfx_sparse_ffn_swiglu(xb, Wgu[0], Wdn[0], t_in, t_h, h=hb, y=yb,
+                                             want_bitmaps=True, ws=ws)
+                ux = int(np.unpackbits(r["bitmap_x"].view(torch.uint8).cpu().numpy().reshape(B, -1),
+                                       axis=1).any(0).sum())
+                uh = int(np.unpackbits(r["bitmap_h"].view(torch.uint8).cpu().numpy().reshape(B, -1),
+                                       axis=1).any(0).sum())
+                nbytes = ux * 2 * f * 2 + uh * d * 2 + B * (d * 2 * 2 + f * 4 * 2)
+                us = graph_us([lambda c=c: sb.sfx_sparse_ffn_swiglu(xb, Wgu[c], Wdn[c], t_in, t_h, h=hb,
+                                                                    y=yb, ws=ws) for c in range(n)],
+                              stream, reps=3)
+                sweep.append({"batch": B, "sparsity": p, "us": us, "gbs": nbytes / (us * 1e-6) / 1e9,
+                              "union_frac_in": ux / d, "union_frac_h": uh / f})
+        out["llama3_70b_ffn_bf16"] = {"sweep": sweep, "dense_bytes": 3 * d * f * 2,
+                                      "note": "2 weight copies (2.8 GB) alternate between calls"}
     return out
 
 
@@ -604,6 +613,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-other", action="store_true",
                     help="skip the other workloads (single GEMV, Phi-2, MoE, Llama-3-70B FFN)")
+    ap.add_argument("--other", default=",".join(OTHER_WORKLOADS),
+                    help="comma list of the other workloads to run: " + ", ".join(OTHER_WORKLOADS))
     args = ap.parse_args()
 
     rank, local_rank, world = env_rank()
@@ -753,7 +764,7 @@ def main():
 
     other = None
     if rank == 0 and not args.no_other:
-        other = bench_other_workloads(stream, dev)
+        other = bench_other_workloads(stream, dev, tuple(w for w in args.other.split(",") if w))
 
     e2e_val = replica_gbs(bytes_step, K, world, main_res["e2e_ms"])
     line = {

@@ -11,7 +11,7 @@
 // neuron ([ffn x d]), so a neuron's gate, up and down weights are three
 // contiguous 2d-byte rows.
 //
-// Launches per call (the second with programmatic dependent launch):
+// Launches per call (the second and third with programmatic dependent launch):
 //  1. moe_route_kernel (one CTA, one warp per token): softmax over E logits,
 //     top-k by probability (ties to the lower expert index), weights
 //     renormalised over the selection (or raw); the selected (token, slot)
@@ -34,7 +34,8 @@
 //              those rows; each warp adds its 256-column partial to the
 //              accumulator with 16-byte atomics (the combine order, hence the
 //              last bits of y, may vary between runs).
-//  3. moe_finalize_kernel: y = accumulator in the output dtype.
+//  3. moe_finalize_kernel (programmatic dependent of 2): y = accumulator in
+//     the output dtype.
 #include "sfx_common.cuh"
 #include "sfx_internal.h"
 
@@ -566,6 +567,7 @@ __global__ void __launch_bounds__(kMoeThreads, 2)
 // ---------------------------------------------------------------- 3. finalize
 
 __global__ void moe_finalize_kernel(const float* acc, long long n, void* y, int ydt) {
+  pdl_wait();  // the expert grid's accumulator
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (long long)gridDim.x * blockDim.x)
     store_as(y, i, ydt, acc[i]);
@@ -670,9 +672,21 @@ int run_moe(const void* x, int dt, const float* logits, int B, int d, int E, int
                      : launch_experts<__half>(B, x, d, ffn, ffn_s, top_k, max_active, W_gT,
                                                 W_upT, W_d, Ws_gT, Ws_upT, Ws_d, t_e, a_out, w, s);
   if (rc != SFX_OK) return rc;
+  // finalize as a programmatic dependent: its launch overlaps the expert grid's tail
   const long long n = (long long)B * d;
-  moe_finalize_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(w.acc, n, y, ydt);
-  return cudaGetLastError() == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((n + 255) / 256), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, moe_finalize_kernel, (const float*)w.acc, n, y, ydt) ==
+                 cudaSuccess
+             ? SFX_OK
+             : SFX_ERR_CUDA;
 }
 
 }  // namespace sfx
