@@ -8,7 +8,6 @@ package ``sparse_input_gemv_b200`` never imports it and shares no code with it
 both sides).
 
 Every function is pinned by ``tests/test_oracle_pins.py`` against values the
-source pages print, closed forms, invariants or brute force. One function is
-"parity unpinned" beyond its closed form: ``corrected_gxo_score``.
+source pages print, closed forms, invariants or brute force.
 """
 from .sfx_oracle import *  # noqa: F401,F403

@@ -37,6 +37,7 @@ import numpy as np
 __all__ = [
     "calibration_rank", "calibrate_threshold", "magnitude_mask", "compact",
     "union_mask", "topk_mask", "keep_count", "gxo_score", "corrected_gxo_score",
+    "corrected_gxo_score_f32",
     "glass_ranks", "glass_fuse", "glass_mask", "masked_gemv", "silu", "gelu_erf",
     "gelu_tanh", "ffn_swiglu", "ffn_swiglu_down", "ffn_gelu_topk_down",
     "moe_route", "moe_expert", "moe_layer", "round_to",
@@ -136,12 +137,36 @@ def corrected_gxo_score(g: np.ndarray, h: np.ndarray) -> np.ndarray:
     """Corrected GxO: g_j h_j + (1/2) |h_j| * ||g||_2  (fp64).
 
     [ATTR] "correction term": the first term is plain GxO, the second bounds
-    the inter-layer attribution error (Theorem 5.3) scaled by 1/2. Parity
-    unpinned beyond this closed form.
+    the inter-layer attribution error (Theorem 5.3) scaled by 1/2. Pinned by
+    closed forms; ``corrected_gxo_score_f32`` is the stored-precision twin the
+    GPU selection is compared with.
     """
     g = np.asarray(g, dtype=np.float64)
     h = np.asarray(h, dtype=np.float64)
     return g * h + 0.5 * np.abs(h) * math.sqrt(float(np.sum(g * g)))
+
+
+def corrected_gxo_score_f32(g: np.ndarray, h: np.ndarray) -> np.ndarray:
+    """Corrected GxO in the precision scores are stored and ranked in (float32).
+
+    [ATTR] "correction term": s_j = g_j h_j + (1/2) |h_j| ||g||_2, the norm
+    taken over all N1 neurons of the layer. Reading (the pages fix no
+    precision): as for plain GxO, each score is a float32 value, built from
+    correctly rounded float32 operations in a fixed order,
+      n  = fl32(sqrt_fp64(sum_k g_k^2))  (each square exact in fp64, the sum
+           correctly rounded: math.fsum; sqrt correctly rounded in fp64),
+      t1 = fl32(g_j * h_j),  t2 = fl32(|h_j| * (n / 2)),  s_j = fl32(t1 + t2),
+    so that a GPU taking the same steps ranks the same values. The sign is
+    kept: negative attributions rank lowest.
+    """
+    g32 = np.asarray(g, dtype=np.float32)
+    h32 = np.asarray(h, dtype=np.float32)
+    g64 = g32.astype(np.float64)
+    n = np.float32(math.sqrt(math.fsum((g64 * g64).tolist())))
+    half_n = np.float32(n * np.float32(0.5))  # exact: a power-of-two scaling
+    t1 = (g64 * h32.astype(np.float64)).astype(np.float32)
+    t2 = (np.abs(h32).astype(np.float64) * np.float64(half_n)).astype(np.float32)
+    return (t1.astype(np.float64) + t2.astype(np.float64)).astype(np.float32)
 
 
 def glass_ranks(score: np.ndarray) -> np.ndarray:

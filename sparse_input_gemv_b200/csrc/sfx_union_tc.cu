@@ -36,6 +36,7 @@
 #include "sfx_internal.h"
 
 #include <algorithm>
+#include <cstdlib>
 
 namespace sfx {
 
@@ -307,8 +308,11 @@ __global__ void __launch_bounds__(kTcThreads, 2) union_gemm_tc_kernel(const TcAr
       const uint32_t sa = sbase + s * kStageBytes;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {  // A: 64 rows x 16 groups of 16 bytes
+        // a warp takes 8 consecutive rows x 4 column groups: its 16-byte pieces
+        // land in four contiguous 128-byte runs of the stage (no bank conflicts;
+        // rows-fastest would put a row's 16 groups 128 bytes apart, 16-way)
         const int idx = tid + q * kProducers;
-        const int r = idx >> 4, g = idx & 15;
+        const int r = ((idx >> 7) << 3) | (idx & 7), g = (idx >> 3) & 15;
         const int row = c * kRowsPerStage + r;
         const bool valid = row < nrows && g * 8 < ncols;
         const TW* src = Wp + (valid ? (long long)list_row[row] * a.N + n0 + g * 8 : 0);
@@ -468,6 +472,8 @@ GemvPlan plan_union_tc(long long K, long long N) {
   const long long slots = 2LL * sm_count();
   long long S = std::max<long long>(1, slots / p.col_tiles);
   S = std::min<long long>(S, std::max<long long>(1, K / 256));
+  if (const char* e = std::getenv("SFX_TC_S"))  // tuning sweeps only
+    if (*e) S = std::max(1, std::atoi(e));
   long long slice = rup((K + S - 1) / S, kPackThreads);  // whole 256-row pack chunks
   if (slice > kMaxSlice) slice = kMaxSlice;
   p.S = (int)((K + slice - 1) / slice);

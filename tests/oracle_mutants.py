@@ -101,6 +101,22 @@ def _mutants(O):
         np.asarray(g, np.float64) * np.asarray(h, np.float64)
         + np.abs(np.asarray(h, np.float64)) * math.sqrt(float(np.sum(np.asarray(g, np.float64) ** 2)))))
 
+    def cgxo_f32(signed=True, l2=True, half=True):
+        def f(g, h):
+            g32 = np.asarray(g, np.float32).astype(np.float64)
+            h32 = np.asarray(h, np.float32).astype(np.float64)
+            n = math.sqrt(math.fsum((g32 * g32).tolist())) if l2 else float(np.sum(np.abs(g32)))
+            n = np.float64(np.float32(n)) * (0.5 if half else 1.0)
+            t1 = (g32 * h32).astype(np.float32).astype(np.float64)
+            if not signed:
+                t1 = np.abs(t1)
+            t2 = (np.abs(h32) * n).astype(np.float32).astype(np.float64)
+            return (t1 + t2).astype(np.float32)
+        return f
+    M["corrected_f32_ranks_abs_gxo"] = ("corrected_gxo_score_f32", cgxo_f32(signed=False))
+    M["corrected_f32_norm_is_l1"] = ("corrected_gxo_score_f32", cgxo_f32(l2=False))
+    M["corrected_f32_drops_half"] = ("corrected_gxo_score_f32", cgxo_f32(half=False))
+
     def round_bf16_truncates(y, dtype):
         if dtype != "bf16":
             return O.__dict__["_orig_round_to"](y, dtype)
@@ -117,6 +133,7 @@ MUTANT_NAMES = [
     "gemv_applies_union_mask", "silu_drops_factor_v", "gelu_is_tanh_form",
     "swiglu_silu_on_up", "route_not_renormalised", "expert_mask_on_raw_gate",
     "layer_drops_shared_expert", "gxo_not_rounded_to_fp32", "corrected_gxo_drops_half",
+    "corrected_f32_ranks_abs_gxo", "corrected_f32_norm_is_l1", "corrected_f32_drops_half",
     "bf16_rounding_truncates",
 ]
 

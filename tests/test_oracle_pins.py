@@ -197,6 +197,45 @@ def test_corrected_gxo_closed_form():
     assert O.corrected_gxo_score(g, h).tolist() == [3.0 + 2.5, -8.0 + 5.0]
 
 
+def test_corrected_gxo_f32_closed_form():
+    # ||g||_2 = 5 over both neurons: s = g h + |h| * 5 / 2, all exact in float32
+    g = np.array([3.0, 4.0], dtype=np.float32)
+    h = np.array([1.0, -2.0], dtype=np.float32)
+    s = O.corrected_gxo_score_f32(g, h)
+    assert s.dtype == np.float32
+    assert s.tolist() == [5.5, -3.0]
+
+
+def test_corrected_gxo_f32_norm_covers_every_neuron():
+    # the norm is the layer's (ATTR "correction term": sum over k = 1..N1),
+    # including a neuron whose own output is 0
+    g = np.array([0.0, 0.0, 12.0], dtype=np.float32)
+    h = np.array([1.0, -1.0, 0.0], dtype=np.float32)
+    assert O.corrected_gxo_score_f32(g, h).tolist() == [6.0, 6.0, 0.0]
+
+
+def test_corrected_gxo_f32_keeps_the_sign():
+    # GxO -4 vs 0.5: |GxO| ranks neuron 0 first; the corrected signed score
+    # -4 + 4 sqrt(2) / 2 = -1.17 < 0.5 + 0.5 sqrt(2) / 2 = 0.85 ranks neuron 1 first
+    g = np.array([1.0, 1.0], dtype=np.float32)
+    h = np.array([-4.0, 0.5], dtype=np.float32)
+    s = O.corrected_gxo_score_f32(g, h)
+    assert s[0] < 0 < s[1]
+    assert O.topk_mask(s, 1).tolist() == [False, True]
+    assert O.topk_mask(O.gxo_score(g, h), 1).tolist() == [True, False]
+
+
+def test_corrected_gxo_f32_within_rounding_of_the_fp64_definition():
+    rng = np.random.default_rng(11)
+    g = rng.standard_normal(4096).astype(np.float32)
+    h = rng.standard_normal(4096).astype(np.float32)
+    s32 = O.corrected_gxo_score_f32(g, h).astype(np.float64)
+    s64 = O.corrected_gxo_score(g, h)
+    n = math.sqrt(float(np.sum(g.astype(np.float64) ** 2)))
+    scale = np.abs(g.astype(np.float64) * h) + 0.5 * np.abs(h.astype(np.float64)) * n
+    assert np.all(np.abs(s32 - s64) <= 4 * 2.0 ** -24 * scale)
+
+
 # ---------------------------------------------------------------- GLASS
 
 def test_glass_ranks_direction():
