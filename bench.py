@@ -361,8 +361,8 @@ def bench_other_workloads(stream, dev, which=OTHER_WORKLOADS):
         import ctypes
         P = lambda tns: ctypes.c_void_p(tns.data_ptr())
 
-        def select_gxo(k):
-            lib.sfx_mask_compact(P(h), sb.SFX_F32, 1, f, sb.SFX_SEL_TOPK_GXO, 0.0, k, P(g), None, 0.5,
+        def select_gxo(k, sel=sb.SFX_SEL_TOPK_GXO):
+            lib.sfx_mask_compact(P(h), sb.SFX_F32, 1, f, sel, 0.0, k, P(g), None, 0.5,
                                  P(bitmap), P(idx), P(cnt), None, None, P(ws.buf), ws.buf.numel(),
                                  ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
         phi = {}
@@ -376,6 +376,15 @@ def bench_other_workloads(stream, dev, which=OTHER_WORKLOADS):
                     sb.sfx_sparse_gemv(h[0], W2[c], idx=idx[0], cnt=cnt, y=y[0], ws=ws)
                 steps.append(step)
             us = graph_us(steps, stream)
+            # the same step with the corrected GxO score (ATTR "correction term")
+            csteps = []
+            for c in range(n):
+                def cstep(c=c, k=k):
+                    sb.sfx_sparse_gemv(x, W1[c], flags=sb.SFX_FLAG_GELU, y=h, ws=ws)
+                    select_gxo(k, sb.SFX_SEL_TOPK_CGXO)
+                    sb.sfx_sparse_gemv(h[0], W2[c], idx=idx[0], cnt=cnt, y=y[0], ws=ws)
+                csteps.append(cstep)
+            us_c = graph_us(csteps, stream)
             nbytes = d * f * 2 + k * d * 2 + d * 2 + f * 4 * 3 + d * 2
             # GLASS: the mask is fixed after prefill, so a decode step is up + down only
             sb.sfx_mask_compact(None, sb.SFX_SEL_TOPK_GLASS, k=k, score_l=sl, score_g=sgl, lam=0.5, ws=ws)
@@ -385,7 +394,8 @@ def bench_other_workloads(stream, dev, which=OTHER_WORKLOADS):
                                            sb.sfx_sparse_gemv(h[0], W2[c], idx=gl["idx"][0],
                                                               cnt=gl["cnt"], y=y[0], ws=ws))
                               for c in range(n)], stream)
-            phi[f"keep{int(keep * 100)}"] = {"us_gxo": us, "us_glass_static_mask": us_gl,
+            phi[f"keep{int(keep * 100)}"] = {"us_gxo": us, "us_corrected_gxo": us_c,
+                                             "us_glass_static_mask": us_gl,
                                              "gbs_gxo": nbytes / (us * 1e-6) / 1e9}
         out["phi2_gelu_ffn_fp16_topk"] = phi
         del W1, W2

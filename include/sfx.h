@@ -60,7 +60,8 @@ typedef enum { SFX_F16 = 0, SFX_BF16 = 1, SFX_F32 = 2 } sfx_dtype;
 typedef enum {
   SFX_SEL_THRESHOLD = 0,   /* m_i = 1[|x_i| > t]                         [TEAL] */
   SFX_SEL_TOPK_GXO = 1,    /* top-k of s_i = |fl32(x_i * g_i)|            [ATTR] */
-  SFX_SEL_TOPK_GLASS = 2   /* top-k of (1-l) R^l_i + l R^g_i             [GLASS] */
+  SFX_SEL_TOPK_GLASS = 2,  /* top-k of (1-l) R^l_i + l R^g_i             [GLASS] */
+  SFX_SEL_TOPK_CGXO = 3    /* top-k of x_i g_i + |x_i| ||g||_2 / 2        [ATTR] */
 } sfx_select;
 
 typedef enum {
@@ -155,6 +156,11 @@ int sfx_calibrate_thresholds(const void* calib, int dt, long long S, long long K
  *               most important neuron ranked n (score descending, then index
  *               ascending); F = (1-lambda) R^l + lambda R^g in double; keep
  *               the k largest F, ties to the lower index. x is unused.
+ *  TOPK_CGXO:   corrected GxO ([ATTR] "correction term"): keep the k largest
+ *               signed s_bi = fl32(fl32(x_bi g_bi) + fl32(|x_bi| n_b / 2)) with
+ *               n_b = fl32(sqrt(sum_i g_bi^2)), the sum of squares in double over
+ *               all K neurons of the row; g = score_l (f32 [B x K]); ties to the
+ *               lower index.
  *
  *  x          (dev)  [B x K] of dtype dt (f16, bf16, f32); may be NULL for GLASS
  *  bitmap     (dev)  [B x ceil(K/32)] uint32, bit (i % 32) of word i/32 = m_bi;

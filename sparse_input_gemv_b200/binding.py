@@ -18,7 +18,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libsfx.so")
 
 SFX_F16, SFX_BF16, SFX_F32 = 0, 1, 2
-SFX_SEL_THRESHOLD, SFX_SEL_TOPK_GXO, SFX_SEL_TOPK_GLASS = 0, 1, 2
+SFX_SEL_THRESHOLD, SFX_SEL_TOPK_GXO, SFX_SEL_TOPK_GLASS, SFX_SEL_TOPK_CGXO = 0, 1, 2, 3
 SFX_OP_CALIBRATE, SFX_OP_MASK_COMPACT, SFX_OP_SPARSE_GEMV, SFX_OP_FFN_SWIGLU, SFX_OP_MOE = range(5)
 SFX_FLAG_GELU, SFX_FLAG_GELU_TANH, SFX_FLAG_UNION_MASK, SFX_FLAG_NO_RENORM, SFX_FLAG_CUDA_CORES = \
     0x1, 0x2, 0x4, 0x8, 0x10

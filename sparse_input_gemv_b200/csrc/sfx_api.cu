@@ -164,7 +164,7 @@ int sfx_mask_compact(const void* x, int dt, int B, int K, int sel, float t, int 
   if (!valid_dtype(dt)) return SFX_ERR_DTYPE;
   if (sel == SFX_SEL_THRESHOLD) {
     if (!x) return SFX_ERR_ARG;
-  } else if (sel == SFX_SEL_TOPK_GXO) {
+  } else if (sel == SFX_SEL_TOPK_GXO || sel == SFX_SEL_TOPK_CGXO) {
     if (!x || !score_l || k < 0 || k > K) return SFX_ERR_ARG;
     if (K > 32768) return SFX_ERR_UNSUPPORTED;
     if (union_idx) return SFX_ERR_UNSUPPORTED;

@@ -7,6 +7,9 @@
 //    "implementation"), selected exactly by an MSB-first radix select on the
 //    float bits (non-negative floats order like their bit patterns), equal
 //    scores resolved toward the lower index;
+//  * corrected GxO top-k: the same select on the signed score
+//    s_i = x_i g_i + |x_i| ||g||_2 / 2 (same page, "correction term"), mapped to
+//    an order-preserving unsigned key (sign bit flipped, negatives inverted);
 //  * GLASS:      ranks of two score vectors, F = (1-l) R^l + l R^g in double,
 //    top-k of F ("GLASS: Global-Local Aggregation for inference-time
 //    Sparsification", section 2.2). Ranks are computed by counting, which is
@@ -122,8 +125,9 @@ constexpr int kTopkBins = 2048;  // 2 bins per thread
 template <typename TX>
 __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __restrict__ x,
                                                                 const float* __restrict__ g,
-                                                                int K, int k, uint32_t* bitmap,
-                                                                int32_t* idx, int32_t* cnt) {
+                                                                int K, int k, int corrected,
+                                                                uint32_t* bitmap, int32_t* idx,
+                                                                int32_t* cnt) {
   extern __shared__ uint32_t keys[];  // [kpt][kMaskThreads], then the bitmap [ceil(K / 32)]
   __shared__ uint32_t hist[kTopkBins];
   __shared__ int s_w[kMaskWarps + 1];
@@ -134,6 +138,30 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
   const int kpt = (K + kMaskThreads - 1) / kMaskThreads;
   const TX* xb = x + (long long)b * K;
   const float* gb = g + (long long)b * K;
+  // corrected GxO: n / 2 with n = fl32(sqrt(sum g^2)), the squares exact in
+  // double and summed in double (a fixed order: per thread, then warp and
+  // block trees)
+  float half_n = 0.f;
+  if (corrected) {
+    __shared__ double s_d[kMaskWarps];
+    double ss = 0.0;
+    for (int i = tid; i < K; i += kMaskThreads) {
+      const double gv = (double)gb[i];
+      ss += gv * gv;
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    if ((tid & 31) == 0) s_d[tid >> 5] = ss;
+    __syncthreads();
+    if (tid < 32) {
+      double v = s_d[tid];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (tid == 0) s_d[0] = v;
+    }
+    __syncthreads();
+    half_n = __double2float_rn(sqrt(s_d[0])) * 0.5f;  // exact halving
+  }
   // coalesced reads, eight per thread in flight; element i belongs to thread
   // i / kpt, slot i % kpt
   for (int i0 = 0; i0 < K; i0 += 8 * kMaskThreads) {
@@ -149,7 +177,16 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
       const int i = i0 + u * kMaskThreads + tid;
       if (i < K) {
         const int t = i / kpt, j = i - t * kpt;
-        keys[j * kMaskThreads + t] = __float_as_uint(fabsf(__fmul_rn(xv[u], gv[u])));
+        uint32_t key;
+        if (corrected) {
+          // signed score -> unsigned key in the same order
+          const float sc = __fadd_rn(__fmul_rn(xv[u], gv[u]), __fmul_rn(fabsf(xv[u]), half_n));
+          const uint32_t bits = __float_as_uint(sc);
+          key = (bits & 0x80000000u) ? ~bits : (bits | 0x80000000u);
+        } else {
+          key = __float_as_uint(fabsf(__fmul_rn(xv[u], gv[u])));
+        }
+        keys[j * kMaskThreads + t] = key;
       }
     }
   }
@@ -295,8 +332,8 @@ static int launch_threshold(const void* x, int B, int K, float t, uint32_t* bitm
 }
 
 template <typename TX>
-static int launch_gxo(const void* x, const float* g, int B, int K, int k, uint32_t* bitmap,
-                      int32_t* idx, int32_t* cnt, cudaStream_t s) {
+static int launch_gxo(const void* x, const float* g, int B, int K, int k, int corrected,
+                      uint32_t* bitmap, int32_t* idx, int32_t* cnt, cudaStream_t s) {
   const int kpt = (K + kMaskThreads - 1) / kMaskThreads;
   const size_t smem = (size_t)kpt * kMaskThreads * 4 + (size_t)((K + 31) / 32) * 4;
   auto kern = topk_gxo_kernel<TX>;
@@ -305,7 +342,8 @@ static int launch_gxo(const void* x, const float* g, int B, int K, int k, uint32
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
           cudaSuccess)
     return SFX_ERR_CUDA;
-  kern<<<B, kMaskThreads, smem, s>>>(reinterpret_cast<const TX*>(x), g, K, k, bitmap, idx, cnt);
+  kern<<<B, kMaskThreads, smem, s>>>(reinterpret_cast<const TX*>(x), g, K, k, corrected, bitmap,
+                                     idx, cnt);
   return cudaGetLastError() == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
 }
 
@@ -321,10 +359,12 @@ int launch_mask_compact(const void* x, int dt, int B, int K, int sel, float t, i
     return launch_threshold<float>(x, B, K, t, bitmap, idx, cnt, uidx, ucnt, s);
   }
   int rc = SFX_OK;
-  if (sel == SFX_SEL_TOPK_GXO) {
-    if (dt == SFX_F16) rc = launch_gxo<__half>(x, score_l, B, K, k, bitmap, idx, cnt, s);
-    else if (dt == SFX_BF16) rc = launch_gxo<__nv_bfloat16>(x, score_l, B, K, k, bitmap, idx, cnt, s);
-    else rc = launch_gxo<float>(x, score_l, B, K, k, bitmap, idx, cnt, s);
+  if (sel == SFX_SEL_TOPK_GXO || sel == SFX_SEL_TOPK_CGXO) {
+    const int cor = sel == SFX_SEL_TOPK_CGXO;
+    if (dt == SFX_F16) rc = launch_gxo<__half>(x, score_l, B, K, k, cor, bitmap, idx, cnt, s);
+    else if (dt == SFX_BF16)
+      rc = launch_gxo<__nv_bfloat16>(x, score_l, B, K, k, cor, bitmap, idx, cnt, s);
+    else rc = launch_gxo<float>(x, score_l, B, K, k, cor, bitmap, idx, cnt, s);
   } else {
     // GLASS: ranks of both vectors, fused score, top-k flags, compaction
     const long long total = (long long)B * K;

@@ -103,6 +103,16 @@ def test_other_entry_points_reject_bad_arguments(lib):
     assert lib.sfx_mask_compact(VP(0x1000), sb.SFX_F32, 1, 16, sb.SFX_SEL_THRESHOLD, 0.0, 0,
                                 None, None, 0.5, None, None, None, None, None,
                                 VP(0x4000), 1 << 20, None) == -1
+    # corrected GxO: the same limits as GxO (k <= K, K <= 32768, no union list)
+    assert lib.sfx_mask_compact(VP(0x1000), sb.SFX_F32, 1, 16, sb.SFX_SEL_TOPK_CGXO, 0.0, 17,
+                                VP(0x2000), None, 0.5, None, None, VP(0x3000), None, None,
+                                VP(0x4000), 1 << 20, None) == -1
+    assert lib.sfx_mask_compact(VP(0x1000), sb.SFX_F32, 1, 40000, sb.SFX_SEL_TOPK_CGXO, 0.0, 4,
+                                VP(0x2000), None, 0.5, None, None, VP(0x3000), None, None,
+                                VP(0x4000), 1 << 20, None) == -7
+    assert lib.sfx_mask_compact(VP(0x1000), sb.SFX_F32, 1, 16, 4, 0.0, 4,
+                                VP(0x2000), None, 0.5, None, None, VP(0x3000), None, None,
+                                VP(0x4000), 1 << 20, None) == -1
     # FFN: misaligned down weights
     assert lib.sfx_sparse_ffn_swiglu(VP(0x1000), sb.SFX_BF16, 1, 64, 128, VP(0x2000), VP(0x3004),
                                      0.1, 0.1, VP(0x4000), sb.SFX_BF16, None, None, None, 0,

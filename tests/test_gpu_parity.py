@@ -120,6 +120,38 @@ def test_topk_gxo_bit_exact(K, keep):
     assert np.array_equal(out["bitmap"].cpu().numpy(), pack_bitmap(m[None]))
 
 
+@pytest.mark.parametrize("K,keep,xdt", [(10240, 0.3, "f32"), (10240, 0.5, "f32"), (10240, 0.7, "f32"),
+                                        (1000, 0.5, "bf16"), (37, 1.0, "f32"), (32768, 0.5, "f16"),
+                                        (3001, 0.0, "f32")])
+def test_topk_corrected_gxo_bit_exact(K, keep, xdt):
+    # ATTR "correction term": signed g h + |h| ||g|| / 2, ranked in float32
+    h = synth.normal((1, K), synth.seed_of("cgxo", K, "h"), 1.0, xdt)
+    g = synth.normal((1, K), synth.seed_of("cgxo", K, "g"), 1.0, "f32")
+    k = O.keep_count(keep, K)
+    out = sb.sfx_mask_compact(dev(h), sb.SFX_SEL_TOPK_CGXO, k=k, score_l=dev(g))
+    s = O.corrected_gxo_score_f32(g.numpy()[0], to64(h)[0].astype(np.float32))
+    m = O.topk_mask(s, k)
+    assert int(out["cnt"][0]) == k
+    assert np.array_equal(out["idx"][0, :k].cpu().numpy(), O.compact(m)[0])
+    assert np.array_equal(out["bitmap"].cpu().numpy(), pack_bitmap(m[None]))
+
+
+def test_topk_corrected_gxo_ties_and_batch():
+    # equal scores everywhere (ties to the lower index) and a second token with
+    # its own norm
+    K = 2048
+    h = torch.ones((2, K), dtype=torch.float32)
+    h[1] = torch.linspace(-3, 3, K)
+    g = torch.full((2, K), 0.5, dtype=torch.float32)
+    g[1, ::7] = -2.0
+    for k in (0, 1, 100, 2047, 2048):
+        out = sb.sfx_mask_compact(dev(h), sb.SFX_SEL_TOPK_CGXO, k=k, score_l=dev(g))
+        for b in range(2):
+            m = O.topk_mask(O.corrected_gxo_score_f32(g.numpy()[b], h.numpy()[b]), k)
+            assert int(out["cnt"][b]) == k
+            assert np.array_equal(out["idx"][b, :k].cpu().numpy(), O.compact(m)[0]), (k, b)
+
+
 def test_topk_gxo_ties_go_to_lower_index():
     K = 3000
     rng = np.random.default_rng(5)
