@@ -37,7 +37,7 @@ import numpy as np
 __all__ = [
     "calibration_rank", "calibrate_threshold", "magnitude_mask", "compact",
     "union_mask", "topk_mask", "keep_count", "gxo_score", "corrected_gxo_score",
-    "corrected_gxo_score_f32",
+    "corrected_gxo_score_f32", "ffn_static_mask",
     "glass_ranks", "glass_fuse", "glass_mask", "masked_gemv", "silu", "gelu_erf",
     "gelu_tanh", "ffn_swiglu", "ffn_swiglu_down", "ffn_gelu_topk_down",
     "moe_route", "moe_expert", "moe_layer", "round_to",
@@ -252,6 +252,29 @@ def ffn_swiglu(x, t_in, W_g, W_u, W_d, t_h):
     m_h = magnitude_mask(h, t_h)
     y = masked_gemv(h, m_h, W_d)
     return y, h, m_x, m_h
+
+
+def ffn_static_mask(x, W_a, W_d, keep, act="gelu", W_b=None):
+    """FFN whose intermediate neurons outside a fixed set are pruned on both sides.
+
+    [GLASS] "selection": with a neuron mask fixed for the prompt, the pruned
+    neurons' up-projection columns and down-projection rows are both skipped.
+    Written as the dense definition: h = act(x W_a) (GeLU, tanh GeLU) or
+    SiLU(x W_a) * (x W_b) (SwiGLU), then y = (h * m) W_d. x [B x d],
+    W_a / W_b [d x ffn], W_d [ffn x d], keep [ffn] bool. Returns (y, h).
+    """
+    x = np.atleast_2d(np.asarray(x, dtype=np.float64))
+    a = x @ np.asarray(W_a, dtype=np.float64)
+    if act == "gelu":
+        h = gelu_erf(a)
+    elif act == "gelu_tanh":
+        h = gelu_tanh(a)
+    elif act == "swiglu":
+        h = silu(a) * (x @ np.asarray(W_b, dtype=np.float64))
+    else:
+        raise ValueError(act)
+    m = np.broadcast_to(np.asarray(keep, dtype=bool), h.shape)
+    return masked_gemv(h, m, W_d), h
 
 
 def ffn_swiglu_down(h, t_h, W_d):

@@ -117,6 +117,11 @@ def _mutants(O):
     M["corrected_f32_norm_is_l1"] = ("corrected_gxo_score_f32", cgxo_f32(l2=False))
     M["corrected_f32_drops_half"] = ("corrected_gxo_score_f32", cgxo_f32(half=False))
 
+    def static_ignores_mask(x, W_a, W_d, keep, act="gelu", W_b=None):
+        return O.__dict__["_orig_ffn_static_mask"](x, W_a, W_d, np.ones_like(np.asarray(keep, bool)),
+                                                   act, W_b)
+    M["static_ffn_ignores_mask"] = ("ffn_static_mask", static_ignores_mask)
+
     def round_bf16_truncates(y, dtype):
         if dtype != "bf16":
             return O.__dict__["_orig_round_to"](y, dtype)
@@ -134,6 +139,7 @@ MUTANT_NAMES = [
     "swiglu_silu_on_up", "route_not_renormalised", "expert_mask_on_raw_gate",
     "layer_drops_shared_expert", "gxo_not_rounded_to_fp32", "corrected_gxo_drops_half",
     "corrected_f32_ranks_abs_gxo", "corrected_f32_norm_is_l1", "corrected_f32_drops_half",
+    "static_ffn_ignores_mask",
     "bf16_rounding_truncates",
 ]
 

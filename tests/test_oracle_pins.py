@@ -236,6 +236,26 @@ def test_corrected_gxo_f32_within_rounding_of_the_fp64_definition():
     assert np.all(np.abs(s32 - s64) <= 4 * 2.0 ** -24 * scale)
 
 
+def test_static_mask_ffn_limits_and_one_neuron():
+    rng = np.random.default_rng(21)
+    d, f = 6, 5
+    x = rng.standard_normal((2, d))
+    Wa, Wb, Wd = rng.standard_normal((d, f)), rng.standard_normal((d, f)), rng.standard_normal((f, d))
+    # all kept: the dense GeLU FFN; none kept: zero
+    y_all, h = O.ffn_static_mask(x, Wa, Wd, np.ones(f, bool))
+    phi = np.array([[0.5 * (1 + math.erf(v / math.sqrt(2))) for v in r] for r in x @ Wa])
+    assert np.allclose(y_all, ((x @ Wa) * phi) @ Wd, rtol=1e-12, atol=1e-12)
+    assert np.all(O.ffn_static_mask(x, Wa, Wd, np.zeros(f, bool))[0] == 0.0)
+    # one kept neuron j: y = h_j * W_d[j, :], with SwiGLU h_j = SiLU(x.Wa_j) (x.Wb_j)
+    j = 3
+    keep = np.zeros(f, bool)
+    keep[j] = True
+    y1, _ = O.ffn_static_mask(x, Wa, Wd, keep, act="swiglu", W_b=Wb)
+    a, u = x @ Wa[:, j], x @ Wb[:, j]
+    hj = a / (1 + np.exp(-a)) * u
+    assert np.allclose(y1, hj[:, None] * Wd[j][None, :], rtol=1e-12, atol=1e-12)
+
+
 # ---------------------------------------------------------------- GLASS
 
 def test_glass_ranks_direction():
