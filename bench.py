@@ -352,6 +352,7 @@ def bench_other_workloads(stream, dev, which=OTHER_WORKLOADS):
         g = synth.normal((1, f), synth.seed_of("phi2", "g"), 1.0, "f32", dev)
         sl = synth.abs_normal((1, f), synth.seed_of("phi2", "local"), device=dev)
         sgl = synth.abs_normal((1, f), synth.seed_of("phi2", "global"), device=dev)
+        W1T = [w.t().contiguous() for w in W1]  # one row per neuron, for the static set
         h = torch.empty((1, f), dtype=torch.float32, device=dev)
         y = torch.empty((1, d), dtype=torch.float16, device=dev)
         bitmap = torch.zeros((1, (f + 31) // 32), dtype=torch.int32, device=dev)
@@ -394,11 +395,19 @@ def bench_other_workloads(stream, dev, which=OTHER_WORKLOADS):
                                            sb.sfx_sparse_gemv(h[0], W2[c], idx=gl["idx"][0],
                                                               cnt=gl["cnt"], y=y[0], ws=ws))
                               for c in range(n)], stream)
+            # GLASS set on both projections: up rows and down rows of the kept neurons only
+            us_both = graph_us([lambda c=c: sb.sfx_static_ffn(x, W1T[c], W2[c], gl["idx"][0],
+                                                              gl["cnt"], y=y, ws=ws)
+                                for c in range(n)], stream)
+            bytes_both = 2 * k * d * 2 + 2 * d * 2
             phi[f"keep{int(keep * 100)}"] = {"us_gxo": us, "us_corrected_gxo": us_c,
                                              "us_glass_static_mask": us_gl,
+                                             "us_glass_both_projections": us_both,
+                                             "gbs_glass_both_projections":
+                                                 bytes_both / (us_both * 1e-6) / 1e9,
                                              "gbs_gxo": nbytes / (us * 1e-6) / 1e9}
         out["phi2_gelu_ffn_fp16_topk"] = phi
-        del W1, W2
+        del W1, W2, W1T
 
     if "moe" in which:
         # MoE: 128 experts, d=2048, expert ffn=768, top-8, shared expert ffn=2048, bf16.

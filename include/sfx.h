@@ -94,7 +94,8 @@ typedef enum {
   SFX_OP_MASK_COMPACT = 1,
   SFX_OP_SPARSE_GEMV = 2,
   SFX_OP_FFN_SWIGLU = 3,
-  SFX_OP_MOE = 4
+  SFX_OP_MOE = 4,
+  SFX_OP_STATIC_FFN = 5
 } sfx_op;
 
 /* Bytes of workspace an operation needs (>= 256: the status header).
@@ -104,6 +105,7 @@ typedef enum {
  *  FFN_SWIGLU:    a = B, b = d,     c = ffn,          d = unused
  *  MOE:           a = B, b = d,     c = E,            d = ffn (expert), e = top_k,
  *                 f = ffn_shared
+ *  STATIC_FFN:    a = B, b = d
  * Returns 0 for an unknown op or invalid sizes. */
 size_t sfx_workspace_bytes(int op, long long a, long long b, long long c, long long d,
                            long long e, long long f);
@@ -304,6 +306,35 @@ int sfx_moe_expert_sparse(const void* x, int dt, const float* logits, int B, int
                           const void* Ws_upT, const void* Ws_d, int ffn_shared, void* y, int ydt,
                           float* a_out, int32_t* sel_out, int flags,
                           void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * a9. FFN with a static neuron mask on both projections          [GLASS]
+ *
+ * "GLASS: Global-Local Aggregation for inference-time Sparsification",
+ * "selection": with the kept neuron set S fixed for the prompt (for example
+ * the SFX_SEL_TOPK_GLASS list of sfx_mask_compact), the pruned neurons' up
+ * columns are skipped as well as their down rows. For every token t:
+ *   GeLU (W_bT == NULL):  h_j = GeLU(W_aT[j, :] . x_t)   (SFX_FLAG_GELU_TANH:
+ *                         the tanh form, else the erf form)
+ *   SwiGLU (W_bT given):  h_j = SiLU(W_aT[j, :] . x_t) (W_bT[j, :] . x_t)
+ *   y_t = sum_{j in S} h_j W_d[j, :]
+ * reading only the rows j in S of every matrix. Neurons are combined in an
+ * fp32 accumulator with atomics, so the last bits of y may differ between runs.
+ *
+ *  x       (dev) [B x d] dtype dt (bf16 or f16), 16-byte aligned
+ *  W_aT, W_bT (optional), W_d (dev) [ffn x d] dtype dt, one row per neuron
+ *  idx     (dev) [>= *cnt] int32 distinct kept neurons in [0, ffn) (any order;
+ *          an entry outside sets SFX_DEV_BAD_INDEX in the workspace status and
+ *          adds 0)
+ *  cnt     (dev) [1] int32 number of kept neurons (clamped to [0, ffn])
+ *  y       (dev) [B x d] dtype ydt
+ *  ws      (dev) sfx_workspace_bytes(SFX_OP_STATIC_FFN, B, d)
+ * Limits: 1 <= B <= 16, d % 8 == 0, B * d <= 98304, ffn >= 1; violations
+ * return SFX_ERR_ARG / SFX_ERR_DTYPE / SFX_ERR_ALIGN before any launch.
+ * ---------------------------------------------------------------------- */
+int sfx_static_ffn(const void* x, int dt, int B, int d, int ffn, const void* W_aT,
+                   const void* W_bT, const void* W_d, const int32_t* idx, const int32_t* cnt,
+                   int flags, void* y, int ydt, void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }

@@ -19,7 +19,8 @@ LIB_PATH = os.path.join(_PKG, "libsfx.so")
 
 SFX_F16, SFX_BF16, SFX_F32 = 0, 1, 2
 SFX_SEL_THRESHOLD, SFX_SEL_TOPK_GXO, SFX_SEL_TOPK_GLASS, SFX_SEL_TOPK_CGXO = 0, 1, 2, 3
-SFX_OP_CALIBRATE, SFX_OP_MASK_COMPACT, SFX_OP_SPARSE_GEMV, SFX_OP_FFN_SWIGLU, SFX_OP_MOE = range(5)
+SFX_OP_CALIBRATE, SFX_OP_MASK_COMPACT, SFX_OP_SPARSE_GEMV, SFX_OP_FFN_SWIGLU, SFX_OP_MOE, \
+    SFX_OP_STATIC_FFN = range(6)
 SFX_FLAG_GELU, SFX_FLAG_GELU_TANH, SFX_FLAG_UNION_MASK, SFX_FLAG_NO_RENORM, SFX_FLAG_CUDA_CORES = \
     0x1, 0x2, 0x4, 0x8, 0x10
 SFX_FLAG_SWIGLU = 0x20
@@ -50,6 +51,8 @@ _SIGS = {
     "sfx_pack_gate_up": (_I, [_VP, _VP, _I, _I, _I, _VP, _VP]),
     "sfx_moe_expert_sparse": (_I, [_VP, _I, _VP, _I, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP,
                                    _VP, _I, _VP, _I, _VP, _VP, _I, _VP, _SZ, _VP]),
+    "sfx_static_ffn": (_I, [_VP, _I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _I, _VP, _I, _VP, _SZ,
+                            _VP]),
 }
 EXPORTED = tuple(_SIGS)
 
@@ -317,6 +320,28 @@ def sfx_moe_expert_sparse(x, logits, W_gT, W_upT, W_d, t_e, top_k, Ws_gT=None, W
     if want_a:
         out["a"], out["sel"] = a, sel
     return out
+
+
+def sfx_static_ffn(x, W_aT, W_d, idx, cnt, W_bT=None, flags=0, out_dtype=None, y=None,
+                   ws: Workspace | None = None, stream=None):
+    """FFN with a static neuron set on both projections; returns y [B x d].
+
+    W_aT (and W_bT for SwiGLU), W_d: [ffn x d] one row per neuron; idx: int32
+    kept neurons, cnt: int32 [1] device count; flags: SFX_FLAG_GELU_TANH for
+    the tanh GeLU (erf GeLU otherwise; W_bT selects SwiGLU).
+    """
+    squeeze = x.dim() == 1
+    x2 = x[None] if squeeze else x
+    _need_cuda(x2, W_aT, W_bT, W_d, idx, cnt)
+    B, d = x2.shape
+    ffn = W_aT.shape[0]
+    if y is None:
+        y = torch.empty((B, d), dtype=out_dtype or x2.dtype, device=x2.device)
+    ws, buf = _ws(ws, sfx_workspace_bytes(SFX_OP_STATIC_FFN, B, d), x2.device)
+    _check("sfx_static_ffn", load().sfx_static_ffn(
+        _ptr(x2), _DT[x2.dtype], B, d, ffn, _ptr(W_aT), _ptr(W_bT), _ptr(W_d), _ptr(idx), _ptr(cnt),
+        int(flags), _ptr(y), _DT[y.dtype], _ptr(buf), buf.numel(), _stream(stream)))
+    return y[0] if squeeze and y.dim() == 2 else y
 
 
 def sfx_device_sm_count() -> int:

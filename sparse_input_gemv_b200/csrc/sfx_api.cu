@@ -99,6 +99,9 @@ size_t sfx_workspace_bytes(int op, long long a, long long b, long long c, long l
     case SFX_OP_MOE:
       if (a < 1 || b < 8 || c < 1 || d < 8 || e < 1) return 0;
       return kWsHeader + moe_workspace_bytes((int)a, (int)b, (int)c, (int)d, (int)e, (int)f);
+    case SFX_OP_STATIC_FFN:
+      if (a < 1 || b < 8) return 0;
+      return kWsHeader + static_ffn_workspace_bytes((int)a, (int)b);
   }
   return 0;
 }
@@ -301,6 +304,23 @@ int sfx_moe_expert_sparse(const void* x, int dt, const float* logits, int B, int
                  shared ? ffn_shared : 0, y, ydt, a_out, sel_out, flags,
                  reinterpret_cast<unsigned char*>(ws) + kWsHeader, need - kWsHeader,
                  as_stream(stream));
+}
+
+int sfx_static_ffn(const void* x, int dt, int B, int d, int ffn, const void* W_aT,
+                   const void* W_bT, const void* W_d, const int32_t* idx, const int32_t* cnt,
+                   int flags, void* y, int ydt, void* ws, size_t ws_bytes, void* stream) {
+  if (!x || !W_aT || !W_d || !idx || !cnt || !y) return SFX_ERR_ARG;
+  if (B < 1 || B > 16 || d < 8 || ffn < 1 || (long long)B * d > 98304) return SFX_ERR_ARG;
+  if (!(dt == SFX_F16 || dt == SFX_BF16) || !valid_dtype(ydt)) return SFX_ERR_DTYPE;
+  if (d % 8 != 0 || !aligned16(x) || !aligned16(W_aT) || !aligned16(W_d) ||
+      (W_bT && !aligned16(W_bT)))
+    return SFX_ERR_ALIGN;
+  const size_t need = sfx_workspace_bytes(SFX_OP_STATIC_FFN, B, d, 0, 0, 0, 0);
+  if (!ws || ws_bytes < need) return SFX_ERR_WORKSPACE;
+  const int act = (flags & SFX_FLAG_GELU_TANH) ? EPI_GELU_TANH : EPI_GELU;
+  return run_static_ffn(x, dt, B, d, ffn, W_aT, W_bT, W_d, idx, cnt, act, y, ydt,
+                        reinterpret_cast<unsigned char*>(ws) + kWsHeader,
+                        reinterpret_cast<unsigned*>(ws), as_stream(stream));
 }
 
 }  // extern "C"

@@ -85,6 +85,12 @@ int run_moe(const void* x, int dt, const float* logits, int B, int d, int E, int
             int ydt, float* a_out, int32_t* sel_out, int flags, unsigned char* ws_body,
             size_t body_bytes, cudaStream_t stream);
 
+// FFN with a static neuron mask (sfx_static_ffn.cu)
+size_t static_ffn_workspace_bytes(int B, int d);
+int run_static_ffn(const void* x, int dt, int B, int d, int ffn, const void* WaT, const void* WbT,
+                   const void* Wd, const int32_t* idx, const int32_t* cnt, int act, void* y,
+                   int ydt, unsigned char* ws_body, unsigned* status, cudaStream_t stream);
+
 // gate/up interleave (sfx_api.cu)
 int launch_pack_gate_up(const void* W_g, const void* W_u, int dt, int d, int ffn, void* W_gu,
                         cudaStream_t stream);

@@ -449,7 +449,8 @@ static int launch_experts(int B, const void* x, int d, int ffn, int ffn_s, int t
   auto kern = moe_expert_kernel<TW>;
   const size_t smem = (size_t)B * (d + kXPad) * sizeof(TW);  // x of an item's tokens (<= B)
   static size_t configured = 0;  // one opt-in per kernel instantiation
-  if (smem > 48 * 1024 && smem > configured) {
+  // opt in whenever the size grows: dynamic plus ~17 KB static may pass 48 KB
+  if (smem > configured) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
         cudaSuccess)
       return SFX_ERR_CUDA;

@@ -1,0 +1,189 @@
+// FFN with a static neuron mask on both projections, on sm_100a.
+//
+// "GLASS: Global-Local Aggregation for inference-time Sparsification",
+// "selection": the set S of kept intermediate neurons is fixed for the prompt,
+// so the pruned neurons' up-projection columns are skipped as well as their
+// down-projection rows. Every matrix is stored one row per intermediate neuron
+// ([ffn x d]), so a kept neuron's weights are contiguous 2d-byte rows:
+//   GeLU:    h_j = GeLU(W_aT[j, :] . x_t)                   (erf or tanh form)
+//   SwiGLU:  h_j = SiLU(W_aT[j, :] . x_t) (W_bT[j, :] . x_t)
+//   y_t = sum_{j in S} h_j W_d[j, :]
+//
+// Launches: the fp32 accumulator is zeroed (cudaMemsetAsync), then
+// static_ffn_kernel (persistent CTAs, programmatic dependent launch): each CTA
+// takes chunks of S whose size it derives from the device-side count so that
+// the chunks spread over all resident CTAs; a chunk's rows of every matrix are
+// bulk-prefetched to L2 at once (they are known before any arithmetic), the dot
+// products run as tensor-core tiles, and the down projection adds 16-byte
+// float4 atomics into the accumulator (the combine order, hence the last bits
+// of y, may vary between runs); then static_ffn_finalize_kernel writes y.
+#include "sfx_common.cuh"
+#include "sfx_internal.h"
+#include "sfx_rowdot.cuh"
+
+namespace sfx {
+
+constexpr int kSfChunkMax = 64;  // kept neurons per work item, at most
+constexpr int kSfChunkMin = 16;  // one tensor-core row tile
+
+template <typename TW>
+__global__ void __launch_bounds__(kRowThreads, 2)
+    static_ffn_kernel(const TW* __restrict__ x, int B, int d, int ffn, const TW* __restrict__ WaT,
+                      const TW* __restrict__ WbT, const TW* __restrict__ Wd,
+                      const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt_p, int act,
+                      float* acc, unsigned* status) {
+  extern __shared__ __align__(16) unsigned char s_xraw[];  // [B][d + kXPad] staged x
+  __shared__ float s_part[kRowThreads / 32][16][kRowTok];
+  __shared__ float s_a[kSfChunkMax][kRowTok];
+  __shared__ float s_v[kSfChunkMax][kRowTok];
+  __shared__ int s_list[kSfChunkMax];
+  __shared__ int s_bad[kSfChunkMax];
+  __shared__ int s_tok[kRowTok];
+
+  const int tid = threadIdx.x;
+  pdl_wait();  // x, the list and the zeroed accumulator come from earlier work on the stream
+  const int cnt = min(max(*cnt_p, 0), ffn);
+  // chunk size from the count: about one item per resident CTA, 16..64 neurons
+  int ch = (cnt + (int)gridDim.x - 1) / (int)gridDim.x;
+  ch = ch < kSfChunkMin ? kSfChunkMin : (ch > kSfChunkMax ? kSfChunkMax : ch);
+  const int n_items = (cnt + ch - 1) / ch;
+  if ((int)blockIdx.x >= n_items) return;
+  const long long row_bytes = (long long)d * sizeof(TW);
+  const int nmat = WbT ? 3 : 2;
+
+  // every row of an item is known up front: bulk-prefetch them all to L2
+  auto prefetch_item = [&](int it) {
+    const int j0 = it * ch, nj = min(ch, cnt - j0);
+    for (int k = tid; k < nmat * nj; k += kRowThreads) {
+      const int m = k / nj;
+      const int r = idx[j0 + (k - m * nj)];
+      if (r < 0 || r >= ffn) continue;  // reported when the item runs
+      const TW* base = m == 0 ? WaT : (m == 1 ? Wd : WbT);
+      prefetch_l2_bulk(base + (long long)r * d, (uint32_t)row_bytes);
+    }
+  };
+  prefetch_item(blockIdx.x);
+
+  const int xstride = d + kXPad;
+  TW* xs = reinterpret_cast<TW*>(s_xraw);
+  for (int i = tid; i < B * (d / 8); i += kRowThreads) {
+    const int b = i / (d / 8), c = i - b * (d / 8);
+    *reinterpret_cast<uint4*>(xs + (long long)b * xstride + c * 8) =
+        __ldg(reinterpret_cast<const uint4*>(x + (long long)b * d) + c);
+  }
+  if (tid < B) s_tok[tid] = tid;
+
+  for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+    const int j0 = it * ch, nj = min(ch, cnt - j0);
+    __syncthreads();  // staged x ready; the previous item is done with the arrays
+    if (tid < nj) {
+      int r = idx[j0 + tid];
+      const int bad = r < 0 || r >= ffn;
+      if (bad) {
+        raise_status(status, SFX_DEV_BAD_INDEX);
+        r = 0;  // read a valid row, contribute nothing
+      }
+      s_list[tid] = r;
+      s_bad[tid] = bad;
+    }
+    __syncthreads();
+    if (it + (int)gridDim.x < n_items) prefetch_item(it + gridDim.x);
+    int n_tiles, ksplit;
+    auto row_of = [&](int r) { return (long long)s_list[r]; };
+    mma_rows(WaT, row_of, nj, d, xs, xstride, B, s_part, &n_tiles, &ksplit);
+    __syncthreads();
+    if (WbT) {
+      for (int i = tid; i < nj * B; i += kRowThreads) {
+        const int r = i / B, t = i - r * B;
+        s_a[r][t] = sum_parts(s_part, n_tiles, ksplit, r, t);
+      }
+      __syncthreads();
+      mma_rows(WbT, row_of, nj, d, xs, xstride, B, s_part, &n_tiles, &ksplit);
+      __syncthreads();
+    }
+    for (int i = tid; i < nj * B; i += kRowThreads) {
+      const int r = i / B, t = i - r * B;
+      const float s = sum_parts(s_part, n_tiles, ksplit, r, t);
+      float v;
+      if (WbT) v = silu_f(s_a[r][t]) * s;
+      else v = act == EPI_GELU_TANH ? gelu_tanh_f(s) : gelu_erf_f(s);
+      s_v[r][t] = s_bad[r] ? 0.f : v;
+    }
+    __syncthreads();
+    down_all(Wd, s_list, nj, s_v, B, s_tok, d, acc);
+  }
+}
+
+__global__ void static_ffn_finalize_kernel(const float* acc, long long n, void* y, int ydt) {
+  pdl_wait();  // the accumulator of the previous grid
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x)
+    store_as(y, i, ydt, acc[i]);
+}
+
+size_t static_ffn_workspace_bytes(int B, int d) { return (size_t)B * d * 4; }
+
+template <typename TW>
+static int launch_static(const void* x, int B, int d, int ffn, const void* WaT, const void* WbT,
+                         const void* Wd, const int32_t* idx, const int32_t* cnt, int act, float* acc,
+                         unsigned* status, cudaStream_t s) {
+  auto kern = static_ffn_kernel<TW>;
+  const size_t smem = (size_t)B * (d + kXPad) * sizeof(TW);
+  static size_t configured = 0;
+  // opt in whenever the size grows: dynamic plus ~17 KB static may pass 48 KB
+  if (smem > configured) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+        cudaSuccess)
+      return SFX_ERR_CUDA;
+    configured = smem;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRowThreads, smem) !=
+          cudaSuccess ||
+      per_sm < 1)
+    return SFX_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(sm_count() * per_sm), 1, 1);
+  cfg.blockDim = dim3(kRowThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, reinterpret_cast<const TW*>(x), B, d, ffn,
+                            reinterpret_cast<const TW*>(WaT), reinterpret_cast<const TW*>(WbT),
+                            reinterpret_cast<const TW*>(Wd), idx, cnt, act, acc, status) ==
+                 cudaSuccess
+             ? SFX_OK
+             : SFX_ERR_CUDA;
+}
+
+int run_static_ffn(const void* x, int dt, int B, int d, int ffn, const void* WaT, const void* WbT,
+                   const void* Wd, const int32_t* idx, const int32_t* cnt, int act, void* y,
+                   int ydt, unsigned char* body, unsigned* status, cudaStream_t s) {
+  float* acc = reinterpret_cast<float*>(body);
+  const long long n = (long long)B * d;
+  if (cudaMemsetAsync(acc, 0, (size_t)n * 4, s) != cudaSuccess) return SFX_ERR_CUDA;
+  const int rc = dt == SFX_BF16 ? launch_static<__nv_bfloat16>(x, B, d, ffn, WaT, WbT, Wd, idx,
+                                                               cnt, act, acc, status, s)
+                                : launch_static<__half>(x, B, d, ffn, WaT, WbT, Wd, idx, cnt, act,
+                                                        acc, status, s);
+  if (rc != SFX_OK) return rc;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((n + 255) / 256), 1, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, static_ffn_finalize_kernel, (const float*)acc, n, y, ydt) ==
+                 cudaSuccess
+             ? SFX_OK
+             : SFX_ERR_CUDA;
+}
+
+}  // namespace sfx

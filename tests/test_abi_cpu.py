@@ -127,6 +127,16 @@ def test_other_entry_points_reject_bad_arguments(lib):
                                      VP(0x3000), VP(0x4000), VP(0x5000), VP(0x6000), None, None,
                                      None, 0, VP(0x7000), sb.SFX_BF16, None, None, 0, VP(0x8000),
                                      1 << 30, None) == -1
+    # static-mask FFN: too many tokens, misaligned weights, fp32 weights
+    assert lib.sfx_static_ffn(VP(0x1000), sb.SFX_BF16, 17, 64, 32, VP(0x2000), None, VP(0x3000),
+                              VP(0x4000), VP(0x5000), 0, VP(0x6000), sb.SFX_BF16, VP(0x7000),
+                              1 << 20, None) == -1
+    assert lib.sfx_static_ffn(VP(0x1000), sb.SFX_BF16, 1, 64, 32, VP(0x2008), None, VP(0x3000),
+                              VP(0x4000), VP(0x5000), 0, VP(0x6000), sb.SFX_BF16, VP(0x7000),
+                              1 << 20, None) == -3
+    assert lib.sfx_static_ffn(VP(0x1000), sb.SFX_F32, 1, 64, 32, VP(0x2000), None, VP(0x3000),
+                              VP(0x4000), VP(0x5000), 0, VP(0x6000), sb.SFX_BF16, VP(0x7000),
+                              1 << 20, None) == -2
     # MoE: the shared expert's three matrices come together or not at all
     assert lib.sfx_moe_expert_sparse(VP(0x1000), sb.SFX_BF16, VP(0x2000), 1, 64, 4, 64, 2,
                                      VP(0x3000), VP(0x4000), VP(0x5000), VP(0x6000), VP(0x9000),

@@ -110,7 +110,7 @@ def test_moe_top1_of_1():
     run_case("moe-one", 4, 1, 128, 32, 1, 0, 0.5)
 
 
-@pytest.mark.parametrize("B,p", [(1, 0.5), (4, 0.8)])
+@pytest.mark.parametrize("B,p", [(1, 0.5), (4, 0.8), (8, 0.5)])
 def test_moe_128_experts_full_size(B, p):
     # 128 experts, d = 2048, expert ffn = 768 SwiGLU, top-8, shared ffn = 2048
     run_case("moe-config", B, 128, 2048, 768, 8, 2048, p)
