@@ -105,7 +105,7 @@ typedef enum {
  *  FFN_SWIGLU:    a = B, b = d,     c = ffn,          d = unused
  *  MOE:           a = B, b = d,     c = E,            d = ffn (expert), e = top_k,
  *                 f = ffn_shared
- *  STATIC_FFN:    a = B, b = d
+ *  STATIC_FFN:    a = B, b = d,     c = ffn
  * Returns 0 for an unknown op or invalid sizes. */
 size_t sfx_workspace_bytes(int op, long long a, long long b, long long c, long long d,
                            long long e, long long f);
@@ -318,8 +318,10 @@ int sfx_moe_expert_sparse(const void* x, int dt, const float* logits, int B, int
  *                         the tanh form, else the erf form)
  *   SwiGLU (W_bT given):  h_j = SiLU(W_aT[j, :] . x_t) (W_bT[j, :] . x_t)
  *   y_t = sum_{j in S} h_j W_d[j, :]
- * reading only the rows j in S of every matrix. Neurons are combined in an
- * fp32 accumulator with atomics, so the last bits of y may differ between runs.
+ * reading only the rows j in S of every matrix. For B > 1 neurons are combined
+ * in an fp32 accumulator with atomics, so the last bits of y may differ
+ * between runs; B = 1 runs the kept up rows, then the deterministic
+ * index-list GEMV over the kept down rows.
  *
  *  x       (dev) [B x d] dtype dt (bf16 or f16), 16-byte aligned
  *  W_aT, W_bT (optional), W_d (dev) [ffn x d] dtype dt, one row per neuron
@@ -328,7 +330,7 @@ int sfx_moe_expert_sparse(const void* x, int dt, const float* logits, int B, int
  *          adds 0)
  *  cnt     (dev) [1] int32 number of kept neurons (clamped to [0, ffn])
  *  y       (dev) [B x d] dtype ydt
- *  ws      (dev) sfx_workspace_bytes(SFX_OP_STATIC_FFN, B, d)
+ *  ws      (dev) sfx_workspace_bytes(SFX_OP_STATIC_FFN, B, d, ffn)
  * Limits: 1 <= B <= 16, d % 8 == 0, B * d <= 98304, ffn >= 1; violations
  * return SFX_ERR_ARG / SFX_ERR_DTYPE / SFX_ERR_ALIGN before any launch.
  * ---------------------------------------------------------------------- */

@@ -337,7 +337,7 @@ def sfx_static_ffn(x, W_aT, W_d, idx, cnt, W_bT=None, flags=0, out_dtype=None, y
     ffn = W_aT.shape[0]
     if y is None:
         y = torch.empty((B, d), dtype=out_dtype or x2.dtype, device=x2.device)
-    ws, buf = _ws(ws, sfx_workspace_bytes(SFX_OP_STATIC_FFN, B, d), x2.device)
+    ws, buf = _ws(ws, sfx_workspace_bytes(SFX_OP_STATIC_FFN, B, d, ffn), x2.device)
     _check("sfx_static_ffn", load().sfx_static_ffn(
         _ptr(x2), _DT[x2.dtype], B, d, ffn, _ptr(W_aT), _ptr(W_bT), _ptr(W_d), _ptr(idx), _ptr(cnt),
         int(flags), _ptr(y), _DT[y.dtype], _ptr(buf), buf.numel(), _stream(stream)))

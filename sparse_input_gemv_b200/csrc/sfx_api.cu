@@ -100,8 +100,8 @@ size_t sfx_workspace_bytes(int op, long long a, long long b, long long c, long l
       if (a < 1 || b < 8 || c < 1 || d < 8 || e < 1) return 0;
       return kWsHeader + moe_workspace_bytes((int)a, (int)b, (int)c, (int)d, (int)e, (int)f);
     case SFX_OP_STATIC_FFN:
-      if (a < 1 || b < 8) return 0;
-      return kWsHeader + static_ffn_workspace_bytes((int)a, (int)b);
+      if (a < 1 || b < 8 || c < 1) return 0;
+      return kWsHeader + static_ffn_workspace_bytes((int)a, (int)b, (int)c);
   }
   return 0;
 }
@@ -315,7 +315,7 @@ int sfx_static_ffn(const void* x, int dt, int B, int d, int ffn, const void* W_a
   if (d % 8 != 0 || !aligned16(x) || !aligned16(W_aT) || !aligned16(W_d) ||
       (W_bT && !aligned16(W_bT)))
     return SFX_ERR_ALIGN;
-  const size_t need = sfx_workspace_bytes(SFX_OP_STATIC_FFN, B, d, 0, 0, 0, 0);
+  const size_t need = sfx_workspace_bytes(SFX_OP_STATIC_FFN, B, d, ffn, 0, 0, 0);
   if (!ws || ws_bytes < need) return SFX_ERR_WORKSPACE;
   const int act = (flags & SFX_FLAG_GELU_TANH) ? EPI_GELU_TANH : EPI_GELU;
   return run_static_ffn(x, dt, B, d, ffn, W_aT, W_bT, W_d, idx, cnt, act, y, ydt,

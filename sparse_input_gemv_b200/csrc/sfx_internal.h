@@ -86,7 +86,7 @@ int run_moe(const void* x, int dt, const float* logits, int B, int d, int E, int
             size_t body_bytes, cudaStream_t stream);
 
 // FFN with a static neuron mask (sfx_static_ffn.cu)
-size_t static_ffn_workspace_bytes(int B, int d);
+size_t static_ffn_workspace_bytes(int B, int d, int ffn);
 int run_static_ffn(const void* x, int dt, int B, int d, int ffn, const void* WaT, const void* WbT,
                    const void* Wd, const int32_t* idx, const int32_t* cnt, int act, void* y,
                    int ydt, unsigned char* ws_body, unsigned* status, cudaStream_t stream);

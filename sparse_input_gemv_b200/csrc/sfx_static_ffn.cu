@@ -9,7 +9,10 @@
 //   SwiGLU:  h_j = SiLU(W_aT[j, :] . x_t) (W_bT[j, :] . x_t)
 //   y_t = sum_{j in S} h_j W_d[j, :]
 //
-// Launches: the fp32 accumulator is zeroed (cudaMemsetAsync), then
+// Batch 1 (decode) takes two launches: static_up_rows_kernel streams the kept up
+// rows (one warp per row, a whole row's loads in flight) into h, then the
+// index-list GEMV reads the kept down rows. Larger batches take three:
+// the fp32 accumulator is zeroed (cudaMemsetAsync), then
 // static_ffn_kernel (persistent CTAs, programmatic dependent launch): each CTA
 // takes chunks of S whose size it derives from the device-side count so that
 // the chunks spread over all resident CTAs; a chunk's rows of every matrix are
@@ -114,6 +117,82 @@ __global__ void __launch_bounds__(kRowThreads, 2)
   }
 }
 
+// Batch 1: h[S[k]] = act(W_aT[S[k], :] . x) for every kept neuron, one warp per
+// row with the whole row's 16-byte loads in flight (x read through L1). The
+// down projection then runs as the index-list GEMV over the kept rows of W_d.
+template <typename TW, bool SWI>
+__global__ void __launch_bounds__(256, 4) static_up_rows_kernel(const TW* __restrict__ x, int d,
+                                                                int ffn, const TW* __restrict__ WaT,
+                                                                const TW* __restrict__ WbT,
+                                                                const int32_t* __restrict__ idx,
+                                                                const int32_t* __restrict__ cnt_p,
+                                                                int act, float* h,
+                                                                unsigned* status) {
+  // 16-byte loads per lane in flight per row (4 KB of one row, or 2 KB of each
+  // of the two SwiGLU rows, per warp); 64 registers keep 32 warps per SM
+  constexpr int kLoads = SWI ? 4 : 8;
+  pdl_wait();  // x and the list may come from the previous grid
+  const int lane = threadIdx.x & 31;
+  const int gw = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int nw = (int)((gridDim.x * blockDim.x) >> 5);
+  const int cnt = min(max(*cnt_p, 0), ffn);
+  // start every row this warp will read towards L2 (one bulk prefetch per row,
+  // spread over the lanes), so the rows stream while the first ones are summed
+  const uint32_t row_bytes = (uint32_t)((long long)d * sizeof(TW));
+  for (int k = gw + lane * nw; k < cnt; k += 32 * nw) {
+    const int r = idx[k];
+    if (r >= 0 && r < ffn) {
+      prefetch_l2_bulk(WaT + (long long)r * d, row_bytes);
+      if (WbT) prefetch_l2_bulk(WbT + (long long)r * d, row_bytes);
+    }
+  }
+  for (int k = gw; k < cnt; k += nw) {
+    const int r = idx[k];
+    if (r < 0 || r >= ffn) {
+      if (lane == 0) raise_status(status, SFX_DEV_BAD_INDEX);
+      continue;  // the down GEMV skips it too
+    }
+    float sa = 0.f, sb = 0.f;
+    const TW* pa = WaT + (long long)r * d;
+    const TW* pb = SWI ? WbT + (long long)r * d : nullptr;
+    for (int c0 = lane * 8; c0 < d; c0 += 256 * kLoads) {
+      uint4 qa[kLoads], qb[kLoads];
+#pragma unroll
+      for (int u = 0; u < kLoads; ++u) {
+        const int c = c0 + u * 256;
+        if (c < d) {
+          qa[u] = __ldcs(reinterpret_cast<const uint4*>(pa + c));
+          if (SWI) qb[u] = __ldcs(reinterpret_cast<const uint4*>(pb + c));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kLoads; ++u) {
+        const int c = c0 + u * 256;
+        if (c < d) {
+          float xv[8], wa[8];
+          unpack8(__ldg(reinterpret_cast<const uint4*>(x + c)), xv, TW());
+          unpack8(qa[u], wa, TW());
+#pragma unroll
+          for (int e = 0; e < 8; ++e) sa = fmaf(wa[e], xv[e], sa);
+          if (SWI) {
+            float wb[8];
+            unpack8(qb[u], wb, TW());
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sb = fmaf(wb[e], xv[e], sb);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) {
+      sa += __shfl_xor_sync(0xffffffffu, sa, o);
+      sb += __shfl_xor_sync(0xffffffffu, sb, o);
+    }
+    if (lane == 0)
+      h[r] = SWI ? silu_f(sa) * sb : (act == EPI_GELU_TANH ? gelu_tanh_f(sa) : gelu_erf_f(sa));
+  }
+}
+
 __global__ void static_ffn_finalize_kernel(const float* acc, long long n, void* y, int ydt) {
   pdl_wait();  // the accumulator of the previous grid
   for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -121,7 +200,14 @@ __global__ void static_ffn_finalize_kernel(const float* acc, long long n, void* 
     store_as(y, i, ydt, acc[i]);
 }
 
-size_t static_ffn_workspace_bytes(int B, int d) { return (size_t)B * d * 4; }
+// batch > 1: the fp32 accumulator [B x d]; batch 1: h [ffn] f32, then the down
+// GEMV's split-K partials
+static size_t al256s(size_t v) { return (v + 255) / 256 * 256; }
+size_t static_ffn_workspace_bytes(int B, int d, int ffn) {
+  const size_t fused = (size_t)B * d * 4;
+  const size_t one = al256s((size_t)ffn * 4) + gemv_workspace_bytes(ffn, d, 1);
+  return B == 1 ? (fused > one ? fused : one) : fused;
+}
 
 template <typename TW>
 static int launch_static(const void* x, int B, int d, int ffn, const void* WaT, const void* WbT,
@@ -163,6 +249,47 @@ static int launch_static(const void* x, int B, int d, int ffn, const void* WaT, 
 int run_static_ffn(const void* x, int dt, int B, int d, int ffn, const void* WaT, const void* WbT,
                    const void* Wd, const int32_t* idx, const int32_t* cnt, int act, void* y,
                    int ydt, unsigned char* body, unsigned* status, cudaStream_t s) {
+  if (B == 1) {
+    // kept up rows streamed one warp per row, then the index-list GEMV for the down rows
+    float* h = reinterpret_cast<float*>(body);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(sm_count() * 4), 1, 1);  // four resident CTAs per SM
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
+    if (dt == SFX_BF16) {
+      using T = __nv_bfloat16;
+      e = cudaLaunchKernelEx(&cfg, WbT ? static_up_rows_kernel<T, true> : static_up_rows_kernel<T, false>,
+                             reinterpret_cast<const T*>(x), d, ffn, reinterpret_cast<const T*>(WaT),
+                             reinterpret_cast<const T*>(WbT), idx, cnt, act, h, status);
+    } else {
+      using T = __half;
+      e = cudaLaunchKernelEx(&cfg, WbT ? static_up_rows_kernel<T, true> : static_up_rows_kernel<T, false>,
+                             reinterpret_cast<const T*>(x), d, ffn, reinterpret_cast<const T*>(WaT),
+                             reinterpret_cast<const T*>(WbT), idx, cnt, act, h, status);
+    }
+    if (e != cudaSuccess) return SFX_ERR_CUDA;
+    GemvArgs g = {};
+    g.x = h;
+    g.W = Wd;
+    g.y = y;
+    g.idx = idx;
+    g.cnt = cnt;
+    g.status = status;
+    g.counters = reinterpret_cast<int32_t*>(reinterpret_cast<unsigned char*>(status) + kWsStatusBytes);
+    g.partials = reinterpret_cast<float*>(body + al256s((size_t)ffn * 4));
+    g.K = ffn;
+    g.N = d;
+    g.B = 1;
+    g.ydt = ydt;
+    g.epi = EPI_NONE;
+    return launch_sparse_gemv(dt, SFX_F32, plan_gemv(ffn, d, 1, true), g, s, true);
+  }
   float* acc = reinterpret_cast<float*>(body);
   const long long n = (long long)B * d;
   if (cudaMemsetAsync(acc, 0, (size_t)n * 4, s) != cudaSuccess) return SFX_ERR_CUDA;
