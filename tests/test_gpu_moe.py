@@ -106,6 +106,11 @@ def test_moe_without_shared_expert_and_raw_weights():
     run_case("moe-noshared", 5, 12, 256, 64, 3, 0, 0.5, flags=sb.SFX_FLAG_NO_RENORM)
 
 
+def test_moe_most_experts_and_tokens():
+    # the largest expert count (1024) and batch (16) the entry point takes
+    run_case("moe-wide", 16, 1024, 128, 32, 4, 64, 0.5)
+
+
 def test_moe_top1_of_1():
     run_case("moe-one", 4, 1, 128, 32, 1, 0, 0.5)
 

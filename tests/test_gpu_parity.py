@@ -391,3 +391,49 @@ def test_union_tensor_core_epilogues():
 @pytest.mark.parametrize("B", [4, 16])
 def test_ffn_swiglu_batched_tensor_cores(B):
     ffn_case(B, 1024, 3584, 0.5, seed=f"ffn-b{B}")
+
+
+def _cols64(W, j0, j1):
+    return W[:, j0:j1].float().cpu().numpy().astype(np.float64)
+
+
+def _oracle_h_chunked(x64, m_x, Wg, Wu, chunk=2048):
+    """The oracle's h = SiLU(g) * u over all neurons, column block by column block
+    (the same fp64 products as O.ffn_swiglu without holding all weights in fp64)."""
+    xm = np.where(m_x, x64, 0.0)
+    ffn = Wg.shape[1]
+    h = np.empty((x64.shape[0], ffn))
+    for j0 in range(0, ffn, chunk):
+        j1 = min(ffn, j0 + chunk)
+        g = O.masked_gemv(xm, np.ones_like(m_x), _cols64(Wg, j0, j1))
+        u = O.masked_gemv(xm, np.ones_like(m_x), _cols64(Wu, j0, j1))
+        h[:, j0:j1] = O.silu(g) * u
+    return h
+
+
+@pytest.mark.parametrize("B", [1, 16])
+def test_ffn_swiglu_llama3_70b_full_size_sampled(B):
+    # the full 1.4 GB layer in the launch configuration the bench times; the
+    # oracle checks the input mask bit for bit, h on every neuron and y on a
+    # sample of output columns
+    d, ffn, p, seed = 8192, 28672, 0.5, "llama3-70b-ffn"
+    calib_x = synth.calib_draws(seed, "x", 64, d, "bf16")
+    t_in = O.calibrate_threshold(to64(calib_x), p)
+    Wg = weights(d, ffn, f"{seed}-g", "bf16", "cuda")
+    Wu = weights(d, ffn, f"{seed}-u", "bf16", "cuda")
+    Wd = weights(ffn, d, f"{seed}-d", "bf16", "cuda")
+    Wgu = sb.sfx_pack_gate_up(Wg, Wu)
+    hc = _oracle_h_chunked(to64(calib_x[:16]), np.ones((16, d), bool), Wg, Wu)
+    t_h = float(np.float32(O.calibrate_threshold(hc, p)))
+    x = synth.eval_draw(seed, "x", B, d, "bf16")
+    out = sb.sfx_sparse_ffn_swiglu(dev(x), Wgu, Wd, t_in, t_h, want_h=True, want_bitmaps=True)
+    x64 = to64(x)
+    m_x = O.magnitude_mask(x64, t_in)
+    assert np.array_equal(out["bitmap_x"].cpu().numpy(), pack_bitmap(m_x))
+    h = _oracle_h_chunked(x64, m_x, Wg, Wu)
+    assert_close(to64(out["h"]), O.round_to(h, "f32"), "h (70B)")
+    m_h = O.magnitude_mask(h, t_h)
+    cols = np.sort(np.random.default_rng(17).choice(d, size=256, replace=False))
+    Wd_cols = Wd[:, torch.from_numpy(cols).cuda()].float().cpu().numpy().astype(np.float64)
+    want = O.masked_gemv(h, m_h, Wd_cols)
+    assert_close(to64(out["y"])[:, cols], O.round_to(want, "bf16"), "y sampled columns (70B)")
