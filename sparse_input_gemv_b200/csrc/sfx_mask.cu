@@ -112,23 +112,22 @@ __device__ __forceinline__ int block_excl_scan(int v, int* s_w, int* total) {
   return r;
 }
 
-// Exact top-k of s_i = |fl32(x_i * g_i)| for one token per CTA. Thread t owns
-// the contiguous elements [t kpt, (t + 1) kpt); its j-th key sits in shared
-// memory at j * kMaskThreads + t (conflict-free passes). Three radix passes
-// over the key bits (11, 11 and 10 bits, most significant first; wide digits
-// keep the histogram atomics spread even though the scores share their
-// leading bits) find the k-th largest key T and how many keys equal to T are
-// kept; two block scans then give every thread its ties' ranks and its output
-// position, so the list comes out ascending with ties resolved toward the
-// lower index.
+// Exact top-k of s_i = |fl32(x_i * g_i)| (or the corrected GxO score) for one
+// token per CTA. Thread t owns the contiguous elements [t kpt, (t + 1) kpt),
+// kpt <= KPT, and keeps their keys in registers. Three radix passes over the
+// key bits (11, 11 and 10 bits, most significant first; wide digits keep the
+// histogram atomics spread even though the scores share their leading bits)
+// find the k-th largest key T and how many keys equal to T are kept; two block
+// scans then give every thread its ties' ranks and its output position, so the
+// list comes out ascending with ties resolved toward the lower index.
 constexpr int kTopkBins = 2048;  // 2 bins per thread
-template <typename TX>
+template <typename TX, int KPT>
 __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __restrict__ x,
                                                                 const float* __restrict__ g,
                                                                 int K, int k, int corrected,
                                                                 uint32_t* bitmap, int32_t* idx,
                                                                 int32_t* cnt) {
-  extern __shared__ uint32_t keys[];  // [kpt][kMaskThreads], then the bitmap [ceil(K / 32)]
+  extern __shared__ uint32_t s_bits[];  // the bitmap [ceil(K / 32)]
   __shared__ uint32_t hist[kTopkBins];
   __shared__ int s_w[kMaskWarps + 1];
   __shared__ uint32_t s_prefix;
@@ -138,6 +137,15 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
   const int kpt = (K + kMaskThreads - 1) / kMaskThreads;
   const TX* xb = x + (long long)b * K;
   const float* gb = g + (long long)b * K;
+  const int e0 = tid * kpt;
+  const int nt = K - e0 < 0 ? 0 : (K - e0 < kpt ? K - e0 : kpt);  // this thread's elements
+  // this thread's inputs (a contiguous run: its lines are shared through L1)
+  float xv[KPT], gv[KPT];
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    xv[j] = j < nt ? to_f32(xb[e0 + j]) : 0.f;
+    gv[j] = j < nt ? gb[e0 + j] : 0.f;
+  }
   // corrected GxO: n / 2 with n = fl32(sqrt(sum g^2)), the squares exact in
   // double and summed in double (a fixed order: per thread, then warp and
   // block trees)
@@ -145,10 +153,8 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
   if (corrected) {
     __shared__ double s_d[kMaskWarps];
     double ss = 0.0;
-    for (int i = tid; i < K; i += kMaskThreads) {
-      const double gv = (double)gb[i];
-      ss += gv * gv;
-    }
+#pragma unroll
+    for (int j = 0; j < KPT; ++j) ss += (double)gv[j] * (double)gv[j];
 #pragma unroll
     for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     if ((tid & 31) == 0) s_d[tid >> 5] = ss;
@@ -162,38 +168,19 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
     __syncthreads();
     half_n = __double2float_rn(sqrt(s_d[0])) * 0.5f;  // exact halving
   }
-  // coalesced reads, eight per thread in flight; element i belongs to thread
-  // i / kpt, slot i % kpt
-  for (int i0 = 0; i0 < K; i0 += 8 * kMaskThreads) {
-    float xv[8], gv[8];
+  uint32_t key[KPT];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kMaskThreads + tid;
-      xv[u] = i < K ? to_f32(xb[i]) : 0.f;
-      gv[u] = i < K ? gb[i] : 0.f;
-    }
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      const int i = i0 + u * kMaskThreads + tid;
-      if (i < K) {
-        const int t = i / kpt, j = i - t * kpt;
-        uint32_t key;
-        if (corrected) {
-          // signed score -> unsigned key in the same order
-          const float sc = __fadd_rn(__fmul_rn(xv[u], gv[u]), __fmul_rn(fabsf(xv[u]), half_n));
-          const uint32_t bits = __float_as_uint(sc);
-          key = (bits & 0x80000000u) ? ~bits : (bits | 0x80000000u);
-        } else {
-          key = __float_as_uint(fabsf(__fmul_rn(xv[u], gv[u])));
-        }
-        keys[j * kMaskThreads + t] = key;
-      }
+  for (int j = 0; j < KPT; ++j) {
+    if (corrected) {
+      // signed score -> unsigned key in the same order
+      const float sc = __fadd_rn(__fmul_rn(xv[j], gv[j]), __fmul_rn(fabsf(xv[j]), half_n));
+      const uint32_t bits = __float_as_uint(sc);
+      key[j] = (bits & 0x80000000u) ? ~bits : (bits | 0x80000000u);
+    } else {
+      key[j] = __float_as_uint(fabsf(__fmul_rn(xv[j], gv[j])));
     }
   }
-  const int e0 = tid * kpt;
-  const int nt = K - e0 < 0 ? 0 : (K - e0 < kpt ? K - e0 : kpt);  // this thread's elements
   const int words = (K + 31) >> 5;
-  uint32_t* s_bits = keys + (size_t)kpt * kMaskThreads;
   for (int w = tid; w < words; w += kMaskThreads) s_bits[w] = 0u;
 
   uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k;
@@ -208,11 +195,10 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
     for (int ps = 0; ps < 3; ++ps) {
       const int shift = kShift[ps];
       const uint32_t dmask = (1u << kBits[ps]) - 1u;
-      __syncthreads();  // keys and zeroed bins (or the previous selection) visible
-      for (int j = 0; j < nt; ++j) {
-        const uint32_t key = keys[j * kMaskThreads + tid];
-        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1u);
-      }
+      __syncthreads();  // zeroed bins (or the previous selection) visible
+#pragma unroll
+      for (int j = 0; j < KPT; ++j)
+        if (j < nt && (key[j] & pmask) == prefix) atomicAdd(&hist[(key[j] >> shift) & dmask], 1u);
       __syncthreads();
       // keys in bins above this thread's two: total minus the inclusive prefix
       const uint32_t h0 = hist[2 * tid], h1 = hist[2 * tid + 1];
@@ -236,16 +222,14 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
       remaining = s_remaining;
       pmask |= dmask << shift;
     }
-  } else {
-    __syncthreads();
   }
   const uint32_t T = prefix;  // k-th largest key; `remaining` of the keys equal to T are kept
   // ties before this thread, then this thread's kept count and output position
   int n_gt = 0, n_eq = 0;
-  for (int j = 0; j < nt; ++j) {
-    const uint32_t key = keys[j * kMaskThreads + tid];
-    n_gt += (k > 0 && key > T);
-    n_eq += (k > 0 && key == T);
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    n_gt += (j < nt && k > 0 && key[j] > T);
+    n_eq += (j < nt && k > 0 && key[j] == T);
   }
   int tot;
   const int eq_before = block_excl_scan(n_eq, s_w, &tot);
@@ -256,25 +240,27 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
   int pos = pos0, eq_seen = 0;
   uint32_t word = 0;  // bits of the current bitmap word gathered by this thread
   int word_id = e0 >> 5;
-  for (int j = 0; j < nt; ++j) {
-    const int i = e0 + j;
-    const uint32_t key = keys[j * kMaskThreads + tid];
-    bool keep = false;
-    if (k > 0) {
-      if (key > T) {
-        keep = true;
-      } else if (key == T) {
-        keep = eq_seen < eq_keep;
-        ++eq_seen;
+#pragma unroll
+  for (int j = 0; j < KPT; ++j) {
+    if (j < nt) {
+      const int i = e0 + j;
+      bool keep = false;
+      if (k > 0) {
+        if (key[j] > T) {
+          keep = true;
+        } else if (key[j] == T) {
+          keep = eq_seen < eq_keep;
+          ++eq_seen;
+        }
       }
+      if (keep && out) out[pos++] = i;
+      if ((i >> 5) != word_id) {  // flush a finished word (shared with neighbours: OR)
+        if (word) atomicOr(&s_bits[word_id], word);
+        word = 0;
+        word_id = i >> 5;
+      }
+      if (keep) word |= 1u << (i & 31);
     }
-    if (keep && out) out[pos++] = i;
-    if ((i >> 5) != word_id) {  // flush a finished word (shared with neighbours: OR)
-      if (word) atomicOr(&s_bits[word_id], word);
-      word = 0;
-      word_id = i >> 5;
-    }
-    if (keep) word |= 1u << (i & 31);
   }
   if (word) atomicOr(&s_bits[word_id], word);
   __syncthreads();
@@ -331,20 +317,24 @@ static int launch_threshold(const void* x, int B, int K, float t, uint32_t* bitm
   return cudaGetLastError() == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
 }
 
+template <typename TX, int KPT>
+static int launch_gxo_k(const void* x, const float* g, int B, int K, int k, int corrected,
+                        uint32_t* bitmap, int32_t* idx, int32_t* cnt, cudaStream_t s) {
+  const size_t smem = (size_t)((K + 31) / 32) * 4;  // the bitmap (<= 4 KB)
+  topk_gxo_kernel<TX, KPT><<<B, kMaskThreads, smem, s>>>(reinterpret_cast<const TX*>(x), g, K, k,
+                                                          corrected, bitmap, idx, cnt);
+  return cudaGetLastError() == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
+}
+
+// keys per thread in registers: K <= 1024 KPT (K <= 32768)
 template <typename TX>
 static int launch_gxo(const void* x, const float* g, int B, int K, int k, int corrected,
                       uint32_t* bitmap, int32_t* idx, int32_t* cnt, cudaStream_t s) {
   const int kpt = (K + kMaskThreads - 1) / kMaskThreads;
-  const size_t smem = (size_t)kpt * kMaskThreads * 4 + (size_t)((K + 31) / 32) * 4;
-  auto kern = topk_gxo_kernel<TX>;
-  // dynamic + ~8 KB static (the 2048-bin histogram) may pass the 48 KB default
-  if (smem + sizeof(uint32_t) * kTopkBins + 1024 > 48 * 1024 &&
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-          cudaSuccess)
-    return SFX_ERR_CUDA;
-  kern<<<B, kMaskThreads, smem, s>>>(reinterpret_cast<const TX*>(x), g, K, k, corrected, bitmap,
-                                     idx, cnt);
-  return cudaGetLastError() == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
+  if (kpt <= 4) return launch_gxo_k<TX, 4>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
+  if (kpt <= 8) return launch_gxo_k<TX, 8>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
+  if (kpt <= 16) return launch_gxo_k<TX, 16>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
+  return launch_gxo_k<TX, 32>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
 }
 
 int launch_mask_compact(const void* x, int dt, int B, int K, int sel, float t, int k,
