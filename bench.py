@@ -507,6 +507,35 @@ def bench_other_workloads(stream, dev, which=OTHER_WORKLOADS):
                               stream, reps=3)
                 sweep.append({"batch": B, "sparsity": p, "us": us, "gbs": nbytes / (us * 1e-6) / 1e9,
                               "union_frac_in": ux / d, "union_frac_h": uh / f})
+        # the same layer on correlated tokens (shared per-neuron scales; masks of
+        # different tokens overlap with pairwise Jaccard ~0.56 at p = 0.5)
+        ccal = synth.correlated_draws("l70c", "x", 64, d, "bf16", draw=0).to(dev)
+        chc = torch.cat([sb.sfx_sparse_ffn_swiglu(ccal[i:i + 16], Wgu[0], Wdn[0], want_h=True,
+                                                  ws=ws)["h"] for i in range(0, 64, 16)]).contiguous()
+        csweep = []
+        for B in (4, 8, 16):
+            xb = synth.correlated_draws("l70c", "x", B, d, "bf16").to(dev)
+            yb = torch.empty((B, d), dtype=torch.bfloat16, device=dev)
+            hb = torch.empty((B, f), dtype=torch.float32, device=dev)
+            for p in (0.5, 0.7, 0.9):
+                t_in = sb.sfx_calibrate_thresholds(ccal, [p], ws=ws)[0]
+                t_h = sb.sfx_calibrate_thresholds(chc, [p], ws=ws)[0]
+                r = sb.sfx_sparse_ffn_swiglu(xb, Wgu[0], Wdn[0], t_in, t_h, h=hb, y=yb,
+                                             want_bitmaps=True, ws=ws)
+                ux = int(np.unpackbits(r["bitmap_x"].view(torch.uint8).cpu().numpy().reshape(B, -1),
+                                       axis=1).any(0).sum())
+                uh = int(np.unpackbits(r["bitmap_h"].view(torch.uint8).cpu().numpy().reshape(B, -1),
+                                       axis=1).any(0).sum())
+                nbytes = ux * 2 * f * 2 + uh * d * 2 + B * (d * 2 * 2 + f * 4 * 2)
+                us = graph_us([lambda c=c: sb.sfx_sparse_ffn_swiglu(xb, Wgu[c], Wdn[c], t_in, t_h, h=hb,
+                                                                    y=yb, ws=ws) for c in range(n)],
+                              stream, reps=3)
+                csweep.append({"batch": B, "sparsity": p, "us": us, "gbs": nbytes / (us * 1e-6) / 1e9,
+                               "union_frac_in": ux / d, "union_frac_h": uh / f})
+        out["llama3_70b_ffn_bf16_correlated_tokens"] = {
+            "sweep": csweep,
+            "note": "x_bi = exp(1.5 n_i) z_bi (shared per-neuron scales); pairwise mask Jaccard "
+                    "~0.56 at p = 0.5"}
         out["llama3_70b_ffn_bf16"] = {"sweep": sweep, "dense_bytes": 3 * d * f * 2,
                                       "note": "2 weight copies (2.8 GB) alternate between calls"}
     return out
