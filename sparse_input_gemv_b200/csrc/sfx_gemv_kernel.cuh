@@ -14,7 +14,8 @@
 //   2. streams the active rows' segments W[i, n0:n0+NT] with 128-bit loads
 //      that bypass L1 and carry an L2 evict-first policy: each warp owns one
 //      256-column chunk of the tile (32 lanes x 8 bf16/fp16) and keeps four
-//      rows in flight, so an SM holds ~64 KB of weight reads in flight,
+//      rows in flight (eight in the 4-slot kernel, which runs one CTA per SM),
+//      so an SM holds ~64 KB of weight reads in flight,
 //      enough to cover HBM latency; products accumulate in fp32 registers;
 //   3. reduces the warps of each chunk in shared memory, then across K
 //      splits: every CTA writes its fp32 partial tile and the last CTA to
@@ -37,7 +38,10 @@ namespace sfx {
 // 512 threads (two CTAs per SM) up to 4 batch slots; 256 threads with the
 // register room for 8 x BMAX accumulators above that.
 __host__ __device__ constexpr int gemv_threads(int bmax) { return bmax >= 8 ? 256 : 512; }
-constexpr int kRowsInFlight = 4;  // independent row loads per warp
+// independent row loads per warp: 4 at batch 1 (two CTAs per SM), 8 for the
+// 4-slot kernel (one CTA per SM, with the registers to spare), so that an SM
+// keeps ~64 KB of weight reads in flight either way
+__host__ __device__ constexpr int rows_in_flight(int bmax) { return bmax == 4 ? 8 : 4; }
 
 __device__ __forceinline__ float apply_epi(int epi, float v) {
   if (epi == EPI_GELU) return gelu_erf_f(v);
@@ -192,16 +196,17 @@ __global__ void __launch_bounds__(gemv_threads(BMAX), (BMAX == 1) ? 2 : 1)
     for (int j = 0; j < 8; ++j) acc[b][j] = 0.f;
 
   if (col_ok) {
-    // rows wrow, wrow + WPC, wrow + 2 WPC, ... ; kRowsInFlight of them per step
-    for (int r0 = wrow; r0 < nrows; r0 += WPC * kRowsInFlight) {
-      uint4 q[kRowsInFlight];
+    // rows wrow, wrow + WPC, wrow + 2 WPC, ... ; kRows of them per step
+    constexpr int kRows = rows_in_flight(BMAX);
+    for (int r0 = wrow; r0 < nrows; r0 += WPC * kRows) {
+      uint4 q[kRows];
 #pragma unroll
-      for (int u = 0; u < kRowsInFlight; ++u) {
+      for (int u = 0; u < kRows; ++u) {
         const int r = r0 + u * WPC;
         if (r < nrows) q[u] = ldg_stream(Wc + (long long)list_row[r] * a.N, pol);
       }
 #pragma unroll
-      for (int u = 0; u < kRowsInFlight; ++u) {
+      for (int u = 0; u < kRows; ++u) {
         const int r = r0 + u * WPC;
         if (r < nrows) {
           float w[8];
