@@ -24,6 +24,7 @@ int sm_count() {
 
 static int bmax_for(int B) {
   if (B <= 1) return 1;
+  if (B <= 2) return 2;
   if (B <= 4) return 4;
   if (B <= 8) return 8;
   return 16;
@@ -41,8 +42,8 @@ static constexpr size_t kListBudget = 48 * 1024;
 GemvPlan plan_gemv(long long K, long long N, int B, bool idx_mode) {
   GemvPlan p;
   p.BMAX = bmax_for(B);
-  // resident CTAs: two per SM at batch 1 (64 registers per thread), one above
-  const int slots = sm_count() * (p.BMAX == 1 ? 2 : 1);
+  // resident CTAs: two per SM up to 2 batch slots (64 registers per thread), one above
+  const int slots = sm_count() * (p.BMAX <= 2 ? 2 : 1);
   // Column tile: the first of 256, 512, 1024, 2048 columns whose tiles times
   // K splits fill at least 90% of the resident slots in one wave; otherwise
   // the best filling one. (Measured on B200 for the Llama-3-8B shapes:

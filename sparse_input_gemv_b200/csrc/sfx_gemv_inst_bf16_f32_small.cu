@@ -6,10 +6,12 @@ namespace sfx {
 
 int gemv_bf16_f32_small(const GemvPlan& p, const GemvArgs& a, cudaStream_t s, bool pdl) {
   if (p.NT == 256 && p.BMAX == 1) return launch_t<__nv_bfloat16, float, 256, 1>(p, a, s, pdl);
+  if (p.NT == 256 && p.BMAX == 2) return launch_t<__nv_bfloat16, float, 256, 2>(p, a, s, pdl);
   if (p.NT == 256 && p.BMAX == 4) return launch_t<__nv_bfloat16, float, 256, 4>(p, a, s, pdl);
   if (p.NT == 256 && p.BMAX == 8) return launch_t<__nv_bfloat16, float, 256, 8>(p, a, s, pdl);
   if (p.NT == 256 && p.BMAX == 16) return launch_t<__nv_bfloat16, float, 256, 16>(p, a, s, pdl);
   if (p.NT == 512 && p.BMAX == 1) return launch_t<__nv_bfloat16, float, 512, 1>(p, a, s, pdl);
+  if (p.NT == 512 && p.BMAX == 2) return launch_t<__nv_bfloat16, float, 512, 2>(p, a, s, pdl);
   if (p.NT == 512 && p.BMAX == 4) return launch_t<__nv_bfloat16, float, 512, 4>(p, a, s, pdl);
   if (p.NT == 512 && p.BMAX == 8) return launch_t<__nv_bfloat16, float, 512, 8>(p, a, s, pdl);
   if (p.NT == 512 && p.BMAX == 16) return launch_t<__nv_bfloat16, float, 512, 16>(p, a, s, pdl);

@@ -38,9 +38,9 @@ namespace sfx {
 // 512 threads (two CTAs per SM) up to 4 batch slots; 256 threads with the
 // register room for 8 x BMAX accumulators above that.
 __host__ __device__ constexpr int gemv_threads(int bmax) { return bmax >= 8 ? 256 : 512; }
-// independent row loads per warp: 4 at batch 1 (two CTAs per SM), 8 for the
-// 4-slot kernel (one CTA per SM, with the registers to spare), so that an SM
-// keeps ~64 KB of weight reads in flight either way
+// independent row loads per warp: 4 for the 1- and 2-slot kernels (two CTAs
+// per SM), 8 for the 4-slot kernel (one CTA per SM, with the registers to
+// spare), so that an SM keeps ~64 KB of weight reads in flight either way
 __host__ __device__ constexpr int rows_in_flight(int bmax) { return bmax == 4 ? 8 : 4; }
 
 __device__ __forceinline__ float apply_epi(int epi, float v) {
@@ -59,7 +59,7 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p, uint64_t pol) {
 }
 
 template <typename TW, typename TX, int NT, int BMAX>
-__global__ void __launch_bounds__(gemv_threads(BMAX), (BMAX == 1) ? 2 : 1)
+__global__ void __launch_bounds__(gemv_threads(BMAX), (BMAX <= 2) ? 2 : 1)
     sparse_gemv_kernel(const GemvArgs a) {
   constexpr int kThreads = gemv_threads(BMAX);
   constexpr int kWarps = kThreads / 32;
