@@ -230,6 +230,7 @@ struct MoeItems {
 struct MoeItem {
   bool shared;
   int p, e, j0, nj;
+  int q0, ne;  // routed items: first grouped pair and number of tokens
 };
 
 // Decodes item `it`; false for a routed item past the active experts (all
@@ -241,13 +242,21 @@ __device__ __forceinline__ bool decode_item(int it, const MoeItems& I, int ffn, 
   if (m.shared) {
     m.p = -1;
     m.e = 0;
+    m.q0 = m.ne = 0;  // the shared expert takes every token
     m.j0 = it * I.ch_s;
     m.nj = ffn_s - m.j0 < I.ch_s ? ffn_s - m.j0 : I.ch_s;
   } else {
     const int k = it - I.n_shared;
     m.p = k / I.n_chunks;
-    if (m.p >= *w.n_active) return false;
-    m.e = w.active[m.p];
+    // p < max_active, so the expert and token offsets are in bounds: load them
+    // together with the count (one round trip instead of three)
+    const int na = *w.n_active;
+    const int e = w.active[m.p];
+    const int q0 = w.tok_off[m.p], q1 = w.tok_off[m.p + 1];
+    if (m.p >= na) return false;
+    m.e = e;
+    m.q0 = q0;
+    m.ne = q1 - q0;
     m.j0 = (k - m.p * I.n_chunks) * I.ch;
     m.nj = ffn - m.j0 < I.ch ? ffn - m.j0 : I.ch;
   }
@@ -325,8 +334,8 @@ __global__ void __launch_bounds__(kMoeThreads, 2)
         s_w[tid] = 1.f;
       }
     } else {
-      const int q0 = w.tok_off[cur.p];
-      ne = w.tok_off[cur.p + 1] - q0;
+      const int q0 = cur.q0;
+      ne = cur.ne;
       te = t_e[cur.e];
       if (tid < ne) {
         s_tok[tid] = w.tok[q0 + tid];
