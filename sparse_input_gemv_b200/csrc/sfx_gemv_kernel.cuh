@@ -6,8 +6,8 @@
 // and only the needed weights are loaded; "Activation sparsity (LLM)"
 // glossary: a zero input skips one weight row).
 //
-// Grid = (column tiles of NT columns) x (K splits), 512 threads, two CTAs per
-// SM for batch 1. Each CTA
+// Grid = (column tiles of NT columns) x (K splits), 512 threads; kernels with
+// 1 or 2 batch slots run two CTAs per SM, the 4-slot kernel one. Each CTA
 //   1. builds the active list of its K-slice in shared memory: |x| > t per
 //      token, warp ballots + popc + a block prefix give ascending positions
 //      (or it reads its share of a caller-provided list);
