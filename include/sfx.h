@@ -191,6 +191,11 @@ int sfx_mask_compact(const void* x, int dt, int B, int K, int sel, float t, int 
  *    mask, unless SFX_FLAG_UNION_MASK makes every token use the union.
  *  - idx != NULL (B must be 1): the active rows are idx[0 .. *cnt-1]
  *    (device count), e.g. from sfx_mask_compact's top-k modes.
+ * Kernels: B <= 2, or an idx list: CUDA cores (fp32 FMAs). B >= 3 with a
+ * threshold: the union rows are fetched once into registers and multiplied on
+ * the tensor cores (mma.sync, fp32 accumulation; fp32 x enters as two 16-bit
+ * halves, hi + lo); SFX_FLAG_CUDA_CORES keeps such a batch on CUDA cores.
+ * Either way the K-split sums are added in a fixed order (same bits per call).
  * Epilogue: SFX_FLAG_GELU / SFX_FLAG_GELU_TANH apply GeLU to y;
  * SFX_FLAG_SWIGLU treats columns (2j, 2j+1) as (gate_j, up_j) and writes
  * h_j = SiLU(gate_j) * up_j to y as fp32 [B x N/2] (ydt must be SFX_F32) --

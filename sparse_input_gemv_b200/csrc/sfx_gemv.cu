@@ -100,8 +100,13 @@ size_t gemv_workspace_bytes(long long K, long long N, int B) {
   GemvPlan q = plan_gemv(K, N, B, true);
   const long long S = std::max(p.S, q.S);
   const size_t cuda_cores = (size_t)(S > 1 ? S : 0) * B * N * 4;
-  const size_t tc = B >= kTcMinBatch ? union_tc_workspace_bytes(K, N, B) : 0;
+  const size_t tc = B >= union_min_batch() ? union_tc_workspace_bytes(K, N, B) : 0;
   return std::max(cuda_cores, tc);
+}
+
+int union_min_batch() {
+  const int v = env_int("SFX_UNION_MIN_B", 0);  // tuning sweeps only
+  return v >= 2 ? v : (union_uses_mma() ? kMmaMinBatch : kTcMinBatch);
 }
 
 // Per-(weight, activation, tile) instantiations live in sfx_gemv_inst_*.cu so
@@ -120,7 +125,7 @@ SFX_DECL(gemv_f16_f32_small) SFX_DECL(gemv_f16_f32_large)
 int launch_sparse_gemv(int wdt, int xdt, const GemvPlan& p, GemvArgs a, cudaStream_t s, bool) {
   const bool pdl = true;
   // a batch of 4..16 tokens in threshold mode: the union tile on tensor cores
-  if (a.B >= kTcMinBatch && a.idx == nullptr && !a.no_tc)
+  if (a.B >= union_min_batch() && a.idx == nullptr && !a.no_tc)
     return launch_union_tc(wdt, xdt, plan_union_tc(a.K, a.N), a, s);
   if (p.col_tiles > kCounterSlots) return SFX_ERR_UNSUPPORTED;
   a.S = p.S;

@@ -50,6 +50,8 @@ struct GemvPlan {
   int list_cap = 0;
   int col_tiles = 0;
   size_t smem = 0;
+  int kind = 0;      // 0 CUDA-core GEMV, 1 union on tcgen05, 2 union on mma.sync
+  int chunks = 0;    // kind 2: 64-column chunks per CTA
 };
 
 int sm_count();
@@ -58,9 +60,18 @@ size_t gemv_workspace_bytes(long long K, long long N, int B);  // excludes the h
 int launch_sparse_gemv(int wdt, int xdt, const GemvPlan& plan, GemvArgs a, cudaStream_t stream,
                        bool pdl);
 
-// batch-union GEMM on tcgen05 (sfx_union_tc.cu), used for B >= kTcMinBatch
-constexpr int kTcMinBatch = 5;  // measured: CUDA cores win up to 4 tokens
+// batch-union GEMM (sfx_union_tc.cu), used for B >= union_min_batch()
+// Smallest batch that takes the union path (measured on B200: the CUDA-core
+// kernel wins at 2 tokens; the mma.sync union kernel from 3 or 4 tokens on,
+// the tcgen05 one from 5)
+constexpr int kMmaMinBatch = 3;
+constexpr int kTcMinBatch = 5;
+int union_min_batch();          // by union kernel, unless overridden for a sweep
 GemvPlan plan_union_tc(long long K, long long N);
+// The union product runs on mma.sync with register-direct weight loads
+// (union_gemm_mma_kernel) instead of tcgen05 (union_gemm_tc_kernel).
+constexpr bool kUnionMmaDefault = true;
+bool union_uses_mma();
 size_t union_tc_workspace_bytes(long long K, long long N, int B);
 int launch_union_tc(int wdt, int xdt, const GemvPlan& plan, const GemvArgs& a, cudaStream_t stream);
 

@@ -1,42 +1,48 @@
-// Batch-union skinny GEMM on the 5th-generation tensor cores (tcgen05).
+// Batch-union skinny GEMM on the tensor cores.
 //
 // For a batch of B <= 16 tokens with per-token magnitude masks ("TEAL:
 // Training-Free Activation Sparsity in Large Language Models", slide 8),
 // y[b, n] = sum_i (x[b, i] m[b, i]) W[i, n]. The rows any token keeps (the
 // union) are fetched once and multiplied as a dense tile: with B tokens the
-// product has B FLOPs per weight byte, more than CUDA cores sustain at HBM
-// speed once B grows, so it runs as tcgen05.mma:
+// product has B FLOPs per weight byte, more than CUDA cores issue at HBM speed
+// once B grows.
 //
-//   D[m, b] (TMEM, fp32)  +=  A[m, k] * B[k, b]
-//   A = W[union rows, n0 : n0+128]   (M = 128 output columns, MN-major)
-//   B = x[b, union rows] * m[b, row] (N = 16 padded tokens, K-major)
-//
-// Two kernels:
-//  1. union_pack_kernel, one CTA per K-split: compacts the split's union rows
-//     (warp ballots, ascending) into a row list in the workspace, and writes
-//     the B operand for them -- already in the canonical K-major no-swizzle
-//     layout of 16-row K-steps (8 x 8 core matrices, SBO = 128 B between token
-//     groups, LBO = 256 B between row halves), bf16/f16, plus a "lo" copy
-//     holding x - hi when x is fp32 (two MMAs per K-step keep ~16 bits).
-//     Rows past the list are zero, padded to whole 64-row stages.
-//  2. union_gemm_tc_kernel, grid (128-column tiles) x (K-splits), warp
-//     specialised: 8 producer warps copy A (64 rows x 256 B per stage, 16-byte
-//     cp.async straight into the canonical MN-major layout: SBO = 128 B
-//     between column groups, LBO = 2 KB between row halves; L2 evict-first)
-//     and B (the packed tiles) into a 4-stage ring and signal each stage's
-//     "full" mbarrier with cp.async.mbarrier.arrive.noinc; one MMA warp waits
-//     on it, issues the stage's four K-steps as tcgen05.mma into a TMEM
+//  1. union_count_kernel and union_pack_kernel, one CTA per 256-row chunk of
+//     K: compact each K-split's union rows (warp ballots, ascending) into a row
+//     list in the workspace and write the x operand for them as 16 x 16
+//     bf16/f16 tiles per 16-row K-step (x * m per token, zero rows past the
+//     list up to whole 64-row stages), plus a "lo" copy holding x - hi when x
+//     is fp32 (two MMAs per K-step keep ~16 bits). The tile layout is the
+//     register order of an mma.sync A fragment for kernel 2a, or the
+//     canonical K-major no-swizzle layout of tcgen05 (8 x 8 core matrices,
+//     SBO = 128 B between token groups, LBO = 256 B between row halves) for 2b.
+//  2a. union_gemm_mma_kernel (the default; section 3 below): every warp loads
+//     its weight rows straight into registers, transposes them with movmatrix
+//     into B fragments and runs m16n8k16 MMAs; no shared-memory staging.
+//  2b. union_gemm_tc_kernel (SFX_UNION_KERNEL=tc), tcgen05.mma with
+//     D[m, b] (TMEM, fp32) += A[m, k] * B[k, b], A = W[union rows, n0 : n0+128]
+//     (M = 128 output columns, MN-major), B = the packed x tiles (N = 16).
+//     Grid (128-column tiles) x (K-splits), warp specialised: 8 producer warps
+//     copy A (64 rows x 256 B per stage, 16-byte cp.async straight into the
+//     canonical MN-major layout: SBO = 128 B between column groups, LBO = 2 KB
+//     between row halves; L2 evict-first) and B into a 4-stage ring and signal
+//     each stage's "full" mbarrier with cp.async.mbarrier.arrive.noinc; one
+//     MMA warp waits on it, issues the stage's four K-steps into a TMEM
 //     accumulator and commits them to the stage's "empty" mbarrier, on which
-//     the producers wait before refilling. No CTA-wide barrier in the loop.
-//     Epilogue: tcgen05.ld (warps 0-3 own TMEM lanes 32w..32w+31), then the
-//     deterministic split-K reduction shared with the CUDA-core kernel.
-// Every mbarrier wait is bounded; on timeout the kernel raises
-// SFX_DEV_TIMEOUT, drains its copies, frees its TMEM and returns.
+//     the producers wait before refilling. Epilogue: tcgen05.ld (warps 0-3 own
+//     TMEM lanes 32w..32w+31), then the deterministic split-K reduction.
+//     Every mbarrier wait is bounded; on timeout the kernel raises
+//     SFX_DEV_TIMEOUT, drains its copies, frees its TMEM and returns.
+// Measured on B200 at 16 tokens, 2a streams 4.3-5.4 TB/s and 2b 2.3-3.5
+// TB/s: 2b is limited by its producers' cp.async gather of 256-byte row pieces
+// into shared memory, not by the MMAs.
 #include "sfx_common.cuh"
 #include "sfx_internal.h"
+#include "sfx_rowdot.cuh"
 
 #include <algorithm>
 #include <cstdlib>
+#include <cstring>
 
 namespace sfx {
 
@@ -64,6 +70,8 @@ struct TcArgs {
   int32_t* chunk_counts;  // [ceil(K / 256)] union rows per 256-row chunk
   uint16_t* pack;     // [S x slice/16 x (hi, lo) x 256] B tiles per split
   int split_b;        // 1 if x is fp32 (hi + lo tiles)
+  int frag;           // 1: x tiles in mma.sync A-fragment order (union_gemm_mma_kernel)
+  int chunks;         // union_gemm_mma_kernel: 64-column chunks per CTA (1, 2, 4 or 8)
 };
 
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid,
@@ -136,6 +144,18 @@ template <> __device__ __forceinline__ float from_bits16<__half>(uint16_t b) {
 // offset (in elements) of (token b, row kk) inside one 16 x 16 K-major B tile
 __device__ __forceinline__ int btile_off(int b, int kk) {
   return ((b & 7) * 16 + (b >> 3) * 128 + (kk & 7) * 2 + (kk >> 3) * 256) / 2;
+}
+
+// offset (in elements) of (token b, row kk) inside one 16 x 16 tile stored in
+// the register order of an m16n8k16 A fragment (A[m = token][k = row]): lane
+// 4g + q holds A[g][2q, 2q+1], A[g+8][2q, 2q+1], A[g][2q+8, 2q+9],
+// A[g+8][2q+8, 2q+9] as 16 contiguous bytes
+__device__ __forceinline__ int frag_off(int b, int kk) {
+  return (((b & 7) << 2) | ((kk & 7) >> 1)) * 8 + (kk & 1) + ((b >> 3) << 1) + ((kk >> 3) << 2);
+}
+
+__device__ __forceinline__ int xtile_off(bool frag, int b, int kk) {
+  return frag ? frag_off(b, kk) : btile_off(b, kk);
 }
 
 }  // namespace
@@ -230,8 +250,9 @@ __global__ void __launch_bounds__(kPackThreads) union_pack_kernel(const TcArgs t
     for (int b = 0; b < kTcN; ++b) {
       const float v = ((bits >> b) & 1u) ? xv[b] : 0.f;
       const uint16_t hi = to_bits16<TW>(v);
-      tl[btile_off(b, kk)] = hi;
-      if (t.split_b) tl[256 + btile_off(b, kk)] = to_bits16<TW>(v - from_bits16<TW>(hi));
+      const int off = xtile_off(t.frag, b, kk);
+      tl[off] = hi;
+      if (t.split_b) tl[256 + off] = to_bits16<TW>(v - from_bits16<TW>(hi));
     }
   }
   if (chunk == last) {
@@ -241,8 +262,9 @@ __global__ void __launch_bounds__(kPackThreads) union_pack_kernel(const TcArgs t
     for (int e = n * kTcN + tid; e < padded * kTcN; e += kPackThreads) {
       const int pos = e / kTcN, b = e % kTcN;
       uint16_t* tl = pack + (long long)(pos / kTcK) * tile_elems;
-      tl[btile_off(b, pos % kTcK)] = 0;
-      if (t.split_b) tl[256 + btile_off(b, pos % kTcK)] = 0;
+      const int off = xtile_off(t.frag, b, pos % kTcK);
+      tl[off] = 0;
+      if (t.split_b) tl[256 + off] = 0;
     }
   }
   pdl_launch_dependents();
@@ -457,29 +479,286 @@ __global__ void __launch_bounds__(kTcThreads, 2) union_gemm_tc_kernel(const TcAr
   if (tid == 0) a.counters[tile] = 0;
 }
 
+
+// ---------------------------------------------------------------- 3. mma.sync GEMM
+
+// The same union product with the weights loaded straight into registers:
+// y[b, n0 + c] = sum over union rows r of x'[b, r] W[r, n0 + c], per warp a
+// 64-column chunk and 16 union rows (a K-block) at a time. A CTA of 8 warps
+// covers C = 1, 2, 4 or 8 chunks; the 8 / C warps of a chunk take its K-blocks
+// in turn and are summed in a fixed order through shared memory (narrow
+// matrices get more column tiles instead of more K splits). Lane 4p + c loads 16 bytes of row p (and of row p + 8) at columns
+// 8c .. 8c + 7 and 32 + 8c .. 32 + 8c + 7 of the slice (64 contiguous bytes per
+// row and load). Each 32-bit register j of such a load is one element pair of
+// an 8 x 8 matrix M[p][2c + e] = W[row p][col 8c + 2j + e]; movmatrix.trans
+// hands lane 4g + q the pair M[2q][g], M[2q + 1][g]: rows 2q, 2q + 1 at one
+// column, which is the B fragment of m16n8k16 (k = union row, n = column).
+// The A fragment (m = token, k = union row) is one 16-byte load from the
+// packed tiles. Lane 4g + q ends with tokens g and g + 8 at the 8 consecutive
+// columns 8q .. 8q + 7 of each 32-column half. No shared-memory staging of
+// weights and no CTA barrier inside the loop: every warp streams on its own,
+// kMmaDepth K-blocks (4 KB) in flight.
+constexpr int kMmaWarps = 8;
+constexpr int kMmaThreads = kMmaWarps * 32;
+constexpr int kMmaWarpCols = 64;
+constexpr int kMmaDepth = 2;
+// token row stride of the reduction buffer: 2 (mod 32) words, so that the
+// float2 stores of a half-warp (tokens g = 0..3, column groups q = 0..3) hit
+// 16 distinct bank pairs
+constexpr int kRedStride = kMmaWarpCols + 2;
+constexpr size_t kRedBytes = (size_t)kMmaWarps * 16 * kRedStride * 4;
+
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t v) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(v));
+  return d;
+}
+
+__device__ __forceinline__ uint4 ld_frag(const uint16_t* p) {
+  return __ldg(reinterpret_cast<const uint4*>(p));
+}
+
+// 16-byte weight load: skip L1, L2 evict-first (weights are read once)
+__device__ __forceinline__ uint4 ld_weight16(const void* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
+__device__ __forceinline__ float epi_f(int epi, float v) {
+  if (epi == EPI_GELU) return gelu_erf_f(v);
+  if (epi == EPI_GELU_TANH) return gelu_tanh_f(v);
+  return v;
+}
+
+template <typename TW, bool SPLIT>
+__global__ void __launch_bounds__(kMmaThreads, 2) union_gemm_mma_kernel(const TcArgs t) {
+  const GemvArgs& a = t.g;
+  // [row list] during the loop, then [8 warps][16 tokens][kRedStride] fp32 sums
+  extern __shared__ __align__(16) unsigned char smem[];
+  int32_t* list_row = reinterpret_cast<int32_t*>(smem);
+  float* red = reinterpret_cast<float*>(smem);
+  __shared__ int s_last;
+
+  const int C = t.chunks, WPC = kMmaWarps / C;  // 64-column chunks, warps per chunk
+  const int NT = kMmaWarpCols * C;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int chunk = warp % C, wrow = warp / C;
+  const int tile = blockIdx.x, split = blockIdx.y;
+  const long long n0 = (long long)tile * NT;
+  const long long N = a.N;
+  const int p = lane >> 2, c = lane & 3;  // load role: row p (and p + 8), column group c
+  const int g = lane >> 2, q = lane & 3;  // fragment role
+
+  pdl_wait();  // the pack kernel's rows, counts and x tiles
+  const int nrows = min(max(t.counts[split], 0), a.slice);
+  for (int r = tid; r < nrows; r += kMmaThreads) list_row[r] = t.rows[(long long)split * a.slice + r];
+  __syncthreads();
+
+  const int tile_elems = 256 * (SPLIT ? 2 : 1);
+  const uint16_t* pack = t.pack + (long long)split * (a.slice / kTcK) * tile_elems;
+  const long long nw = n0 + chunk * kMmaWarpCols;  // first column of this warp
+  // the two 16-byte column groups of this lane (N is a multiple of 8)
+  const bool col0 = nw + 8 * c < N, col1 = nw + 32 + 8 * c < N;
+  const TW* Wb = reinterpret_cast<const TW*>(a.W) + nw + 8 * c;
+  const uint64_t pol = l2_evict_first_policy();
+  const int nblk = (nrows + kTcK - 1) / kTcK;
+
+  float acc[2][4][4];
+#pragma unroll
+  for (int m = 0; m < 2; ++m)
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[m][j][e] = 0.f;
+
+  // the WPC warps of a chunk take groups of kMmaDepth K-blocks in turn
+  const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+  for (int kb0 = wrow * kMmaDepth; kb0 < nblk; kb0 += WPC * kMmaDepth) {
+    uint4 w[kMmaDepth][2][2];  // [K-block][row half][column half]
+    uint4 xa[kMmaDepth], xl[kMmaDepth];
+#pragma unroll
+    for (int u = 0; u < kMmaDepth; ++u) {
+      const int kb = kb0 + u;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = kb * kTcK + h * 8 + p;
+        const bool rv = kb < nblk && r < nrows;
+        const TW* src = Wb + (rv ? (long long)list_row[r] * N : 0);
+        w[u][h][0] = (rv && col0) ? ld_weight16(src, pol) : z;
+        w[u][h][1] = (rv && col1) ? ld_weight16(src + 32, pol) : z;
+      }
+      if (kb < nblk) {
+        xa[u] = ld_frag(pack + (long long)kb * tile_elems + lane * 8);
+        if (SPLIT) xl[u] = ld_frag(pack + (long long)kb * tile_elems + 256 + lane * 8);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kMmaDepth; ++u) {
+      if (kb0 + u >= nblk) break;
+#pragma unroll
+      for (int m = 0; m < 2; ++m) {
+        const uint32_t r0[4] = {w[u][0][m].x, w[u][0][m].y, w[u][0][m].z, w[u][0][m].w};
+        const uint32_t r1[4] = {w[u][1][m].x, w[u][1][m].y, w[u][1][m].z, w[u][1][m].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t b0 = movmatrix_trans(r0[j]);
+          const uint32_t b1 = movmatrix_trans(r1[j]);
+          mma_16816(acc[m][j], xa[u].x, xa[u].y, xa[u].z, xa[u].w, b0, b1, TW());
+          if (SPLIT) mma_16816(acc[m][j], xl[u].x, xl[u].y, xl[u].z, xl[u].w, b0, b1, TW());
+        }
+      }
+    }
+  }
+  pdl_launch_dependents();
+
+  // lane (g, q): acc[m][j][e] = token g, acc[m][j][2 + e] = token g + 8, at
+  // chunk column 32m + 8q + 2j + e. Through shared memory: red[warp][token][col]
+  __syncthreads();  // every warp is done with the row list
+  {
+    float* rw = red + warp * (16 * kRedStride);
+#pragma unroll
+    for (int hi = 0; hi < 2; ++hi)
+#pragma unroll
+      for (int m = 0; m < 2; ++m)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<float2*>(rw + (g + 8 * hi) * kRedStride + 32 * m + 8 * q + 2 * j) =
+              make_float2(acc[m][j][2 * hi], acc[m][j][2 * hi + 1]);
+  }
+  __syncthreads();
+
+  // (chunk, token, column pair): the chunk's WPC warps summed in order, then
+  // the epilogue (S == 1) or this split's partial tile
+  const bool swiglu = a.epi == EPI_SWIGLU;
+  const int ncols = (int)min((long long)NT, N - n0);
+  const int items = C * a.B * (kMmaWarpCols / 2);
+  for (int e = tid; e < items; e += kMmaThreads) {
+    const int ch = e / (a.B * (kMmaWarpCols / 2));
+    const int rem = e - ch * (a.B * (kMmaWarpCols / 2));
+    const int b = rem / (kMmaWarpCols / 2), cp = rem - b * (kMmaWarpCols / 2);
+    const int col = ch * kMmaWarpCols + 2 * cp;  // within the tile
+    if (col >= ncols) continue;
+    float s0 = 0.f, s1 = 0.f;
+    for (int w = 0; w < WPC; ++w) {
+      const float2 v =
+          *reinterpret_cast<const float2*>(red + ((w * C + ch) * 16 + b) * kRedStride + 2 * cp);
+      s0 += v.x;
+      s1 += v.y;
+    }
+    const long long n = n0 + col;
+    if (a.S == 1) {
+      if (swiglu) {
+        reinterpret_cast<float*>(a.y)[(long long)b * (N / 2) + n / 2] = silu_f(s0) * s1;
+      } else {
+        store_as(a.y, (long long)b * N + n, a.ydt, epi_f(a.epi, s0));
+        store_as(a.y, (long long)b * N + n + 1, a.ydt, epi_f(a.epi, s1));
+      }
+    } else {
+      *reinterpret_cast<float2*>(a.partials + ((long long)split * a.B + b) * N + n) =
+          make_float2(s0, s1);
+    }
+  }
+  if (a.S == 1) return;
+
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(&a.counters[tile], 1) == a.S - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // the last CTA of the tile sums the S partials in split order, column pairs
+  // so that the SwiGLU epilogue sees (gate, up) together
+  const long long vs = (long long)a.B * N;
+  for (int e = tid; e < a.B * (NT / 2); e += kMmaThreads) {
+    const int b = e / (NT / 2), c2 = 2 * (e % (NT / 2));
+    if (c2 >= ncols) continue;
+    const float* pb = a.partials + (long long)b * N + n0 + c2;
+    float s0 = 0.f, s1 = 0.f;
+    for (int s = 0; s < a.S; ++s) {
+      const float2 v = __ldcg(reinterpret_cast<const float2*>(pb + s * vs));
+      s0 += v.x;
+      s1 += v.y;
+    }
+    if (swiglu) {
+      reinterpret_cast<float*>(a.y)[(long long)b * (N / 2) + (n0 + c2) / 2] = silu_f(s0) * s1;
+    } else {
+      store_as(a.y, (long long)b * N + n0 + c2, a.ydt, epi_f(a.epi, s0));
+      store_as(a.y, (long long)b * N + n0 + c2 + 1, a.ydt, epi_f(a.epi, s1));
+    }
+  }
+  if (tid == 0) a.counters[tile] = 0;
+}
+
 // ------------------------------------------------------------------ host
 
 static long long rup(long long v, long long m) { return (v + m - 1) / m * m; }
-static constexpr long long kMaxSlice = 6144;  // 24 KB row list in shared memory
+static constexpr long long kMaxSlice = 6144;       // tcgen05: 24 KB row list in shared memory
+static constexpr long long kMmaMaxSlice = 16384;   // mma.sync: 64 KB row list
 
-GemvPlan plan_union_tc(long long K, long long N) {
-  GemvPlan p;
-  p.NT = kTcM;
-  p.BMAX = kTcN;
-  p.col_tiles = (int)((N + kTcM - 1) / kTcM);
-  // one wave of resident CTAs (two per SM); K splits only to fill it (at
-  // least 256 rows each) or to keep a split's list within kMaxSlice rows
+bool union_uses_mma() {
+  const char* e = std::getenv("SFX_UNION_KERNEL");  // "tc" or "mma"
+  if (e && *e) return std::strcmp(e, "mma") == 0;
+  return kUnionMmaDefault;
+}
+
+// Splits of K for `tiles` column tiles: one wave of resident CTAs (two per
+// SM), K splits only to fill it (at least 256 rows each) or to keep a split's
+// list within kMaxSlice rows.
+static void plan_splits(GemvPlan& p, long long K, long long max_slice) {
   const long long slots = 2LL * sm_count();
   long long S = std::max<long long>(1, slots / p.col_tiles);
   S = std::min<long long>(S, std::max<long long>(1, K / 256));
   if (const char* e = std::getenv("SFX_TC_S"))  // tuning sweeps only
     if (*e) S = std::max(1, std::atoi(e));
   long long slice = rup((K + S - 1) / S, kPackThreads);  // whole 256-row pack chunks
-  if (slice > kMaxSlice) slice = kMaxSlice;
+  if (slice > max_slice) slice = max_slice;
   p.S = (int)((K + slice - 1) / slice);
   p.slice = (int)slice;
   p.list_cap = (int)slice;
-  p.smem = (size_t)kStages * kStageBytes + (size_t)slice * 4;
+}
+
+GemvPlan plan_union_tc(long long K, long long N) {
+  GemvPlan p;
+  p.BMAX = kTcN;
+  if (!union_uses_mma()) {
+    p.kind = 1;
+    p.NT = kTcM;
+    p.col_tiles = (int)((N + kTcM - 1) / kTcM);
+    plan_splits(p, K, kMaxSlice);
+    p.smem = (size_t)kStages * kStageBytes + (size_t)p.slice * 4;
+    return p;
+  }
+  // mma.sync: the CTA tile (1, 2, 4 or 8 chunks of 64 columns) that needs the
+  // fewest K splits, 2 chunks among equals, else the narrowest. Measured on
+  // B200 at 16 tokens: the serial sum of many split partials by the last CTA
+  // of a tile costs more than narrow tiles do (the K-blocks of a chunk are
+  // shared by its warps and summed through shared memory).
+  p.kind = 2;
+  int C = 8;
+  const char* e = std::getenv("SFX_MMA_CHUNKS");  // tuning sweeps only
+  if (e && *e) {
+    C = std::atoi(e);
+    if (C != 1 && C != 2 && C != 4) C = 8;
+  } else {
+    int best_S = 1 << 30;
+    for (int cand = 1; cand <= 8; cand *= 2) {
+      GemvPlan q;
+      q.col_tiles = (int)((N + 64LL * cand - 1) / (64LL * cand));
+      plan_splits(q, K, kMmaMaxSlice);
+      if (q.S < best_S || (q.S == best_S && cand == 2)) {
+        best_S = q.S;
+        C = cand;
+      }
+    }
+  }
+  p.chunks = C;
+  p.NT = 64 * C;
+  p.col_tiles = (int)((N + p.NT - 1) / p.NT);
+  plan_splits(p, K, kMmaMaxSlice);
+  p.smem = std::max((size_t)p.slice * 4, kRedBytes);
   return p;
 }
 
@@ -516,6 +795,19 @@ static int configure_tc_kernel() {
   return rc;
 }
 
+template <typename TW>
+static int configure_mma_kernel() {
+  const int bytes = (int)std::max((size_t)kMmaMaxSlice * 4, kRedBytes);
+  static int rc =
+      (cudaFuncSetAttribute(union_gemm_mma_kernel<TW, false>,
+                            cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess &&
+       cudaFuncSetAttribute(union_gemm_mma_kernel<TW, true>,
+                            cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess)
+          ? SFX_OK
+          : SFX_ERR_CUDA;
+  return rc;
+}
+
 template <typename TW, typename TX>
 static int launch_tc(const GemvPlan& p, TcArgs t, cudaStream_t s) {
   cudaLaunchAttribute attr[1];
@@ -530,11 +822,17 @@ static int launch_tc(const GemvPlan& p, TcArgs t, cudaStream_t s) {
   if (cudaLaunchKernelEx(&cfg, union_count_kernel<TX>, t) != cudaSuccess) return SFX_ERR_CUDA;
   if (cudaLaunchKernelEx(&cfg, union_pack_kernel<TW, TX>, t) != cudaSuccess) return SFX_ERR_CUDA;
 
+  cfg.gridDim = dim3((unsigned)p.col_tiles, (unsigned)p.S, 1);
+  cfg.dynamicSmemBytes = p.smem;
+  if (t.frag) {  // p.smem = the row list (up to 64 KB) or the reduction buffer
+    cfg.blockDim = dim3(kMmaThreads, 1, 1);
+    auto kern = t.split_b ? union_gemm_mma_kernel<TW, true> : union_gemm_mma_kernel<TW, false>;
+    if (configure_mma_kernel<TW>() != SFX_OK) return SFX_ERR_CUDA;
+    return cudaLaunchKernelEx(&cfg, kern, t) == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
+  }
   auto kern = union_gemm_tc_kernel<TW>;
   if (configure_tc_kernel<TW>() != SFX_OK) return SFX_ERR_CUDA;
-  cfg.gridDim = dim3((unsigned)p.col_tiles, (unsigned)p.S, 1);
   cfg.blockDim = dim3(kTcThreads, 1, 1);
-  cfg.dynamicSmemBytes = p.smem;
   return cudaLaunchKernelEx(&cfg, kern, t) == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
 }
 
@@ -555,6 +853,8 @@ int launch_union_tc(int wdt, int xdt, const GemvPlan& p, const GemvArgs& a, cuda
   t.chunk_counts = reinterpret_cast<int32_t*>(aux + lay.chunk_counts);
   t.pack = reinterpret_cast<uint16_t*>(aux + lay.pack);
   t.split_b = xdt == SFX_F32 ? 1 : 0;
+  t.frag = p.kind == 2 ? 1 : 0;
+  t.chunks = p.chunks;
   if (wdt == SFX_BF16) {
     if (xdt == SFX_BF16) return launch_tc<__nv_bfloat16, __nv_bfloat16>(p, t, s);
     if (xdt == SFX_F32) return launch_tc<__nv_bfloat16, float>(p, t, s);

@@ -353,6 +353,12 @@ def test_workspace_shared_across_operations():
 
 
 # ---------------------------------------------------------------- batch union on tensor cores
+# (the tcgen05 kernel; the default mma.sync kernel has its own test file)
+
+@pytest.fixture
+def tc_union(monkeypatch):
+    monkeypatch.setenv("SFX_UNION_KERNEL", "tc")
+
 
 @pytest.mark.parametrize("B,K,N,p,wdt,xdt,out", [
     (4, 4096, 2048, 0.5, "bf16", "bf16", "bf16"),
@@ -361,11 +367,11 @@ def test_workspace_shared_across_operations():
     (5, 33, 136, 0.0, "bf16", "bf16", "f32"),       # tiny, dense
     (16, 8192, 1024, 0.9, "bf16", "bf16", "bf16"),  # sparse union (1 - 0.9^16 = 81% rows)
 ])
-def test_union_tensor_core_matches_oracle(B, K, N, p, wdt, xdt, out):
+def test_union_tensor_core_matches_oracle(B, K, N, p, wdt, xdt, out, tc_union):
     gemv_case(B, K, N, p, wdt, xdt=xdt, seed="tc", out=out)
 
 
-def test_union_tensor_core_equals_cuda_core_path():
+def test_union_tensor_core_equals_cuda_core_path(tc_union):
     B, K, N = 16, 4096, 3072
     x = synth.eval_draw("tc-vs-cc", "x", B, K, "bf16")
     W = dev(weights(K, N, "tc-vs-cc", "bf16"))
@@ -376,7 +382,7 @@ def test_union_tensor_core_equals_cuda_core_path():
     assert_close(to64(y_tc), to64(y_cc), "tensor cores vs CUDA cores")
 
 
-def test_union_tensor_core_epilogues():
+def test_union_tensor_core_epilogues(tc_union):
     gemv_case(4, 2560, 1024, 0.4, "f16", out="f32", flags=sb.SFX_FLAG_GELU, seed="tc-gelu")
     B, K, N = 6, 1024, 512
     x = synth.eval_draw("tc-umask", "x", B, K, "bf16")
@@ -389,7 +395,7 @@ def test_union_tensor_core_epilogues():
 
 
 @pytest.mark.parametrize("B", [4, 16])
-def test_ffn_swiglu_batched_tensor_cores(B):
+def test_ffn_swiglu_batched_tensor_cores(B, tc_union):
     ffn_case(B, 1024, 3584, 0.5, seed=f"ffn-b{B}")
 
 
