@@ -289,6 +289,34 @@ class Stack:
         return self.L * ((NQKV + D + 2 * FFN) * D * 2 + FFN * D * 2)
 
 
+def dense_library_us_per_layer(stack, stream, reps=5):
+    """Dense reference: the same layers through torch.matmul (cuBLAS) and torch
+    elementwise ops (SiLU(g) * u in bf16), all rows read, µs per layer. A library
+    yardstick only; it is not on the measured path."""
+    L = stack.L
+    dev = stack.Wqkv[0].device
+    yq = torch.empty((1, NQKV), dtype=torch.bfloat16, device=dev)
+    yo = torch.empty((1, D), dtype=torch.bfloat16, device=dev)
+    gu = torch.empty((1, 2 * FFN), dtype=torch.bfloat16, device=dev)
+    yf = torch.empty((1, D), dtype=torch.bfloat16, device=dev)
+
+    def layers():
+        for l in range(L):
+            torch.mm(stack.xq[l:l + 1], stack.Wqkv[l], out=yq)
+            torch.mm(stack.xo[l:l + 1], stack.Wo[l], out=yo)
+            torch.mm(stack.xf[l:l + 1], stack.Wgu[l], out=gu)
+            h = torch.nn.functional.silu(gu[:, 0::2]) * gu[:, 1::2]
+            torch.mm(h, stack.Wd[l], out=yf)
+
+    layers()
+    torch.cuda.synchronize()
+    g = capture(layers, stream)
+    g.replay()
+    ms = time_graph(g, reps, stream)
+    del g
+    return ms * 1e3 / (reps * L)
+
+
 def capture(fn, stream):
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=stream):
@@ -536,8 +564,24 @@ def bench_other_workloads(stream, dev, which=OTHER_WORKLOADS):
             "sweep": csweep,
             "note": "x_bi = exp(1.5 n_i) z_bi (shared per-neuron scales); pairwise mask Jaccard "
                     "~0.56 at p = 0.5"}
+        # dense library reference: torch.matmul (cuBLAS) for both projections and
+        # torch ops for SiLU(g) * u, every row read
+        lib = []
+        for B in (1, 4, 8, 16):
+            xb = synth.eval_draw("l70", "x", B, d, "bf16").to(dev)
+            gu = torch.empty((B, 2 * f), dtype=torch.bfloat16, device=dev)
+            yb = torch.empty((B, d), dtype=torch.bfloat16, device=dev)
+
+            def dense(c, xb=xb, gu=gu, yb=yb):
+                torch.mm(xb, Wgu[c], out=gu)
+                torch.mm(torch.nn.functional.silu(gu[:, 0::2]) * gu[:, 1::2], Wdn[c], out=yb)
+
+            us = graph_us([lambda c=c: dense(c) for c in range(n)], stream, reps=3)
+            lib.append({"batch": B, "us": us, "gbs": 3 * d * f * 2 / (us * 1e-6) / 1e9})
         out["llama3_70b_ffn_bf16"] = {"sweep": sweep, "dense_bytes": 3 * d * f * 2,
-                                      "note": "2 weight copies (2.8 GB) alternate between calls"}
+                                      "dense_library": lib,
+                                      "note": "2 weight copies (2.8 GB) alternate between calls; "
+                                              "dense_library = torch.matmul (cuBLAS) reference"}
     return out
 
 
@@ -764,6 +808,7 @@ def main():
         kernels[name] = {"us": avg_us, "bytes": kb, "gbs": kb / (avg_us * 1e-6) / 1e9}
         del g
     ffn_us = kernels["ffn_gate_up"]["us"] + kernels["ffn_down"]["us"]
+    dense_lib_us = dense_library_us_per_layer(stack, stream)
 
     peaks = {}
     try:
@@ -827,6 +872,8 @@ def main():
         "us_per_layer": us_layer, "us_per_layer_ffn": ffn_us,
         "dense_us_per_layer": dense_us,
         "speedup_vs_dense": (dense_us / us_layer) if dense_us else None,
+        "dense_library_us_per_layer": dense_lib_us,
+        "speedup_vs_dense_library": dense_lib_us / us_layer,
         "thresholds": main_res["t"],
         "kernels": kernels, "roofline": roofline, "sweep": sweep,
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": main_res["h2d"],

@@ -497,11 +497,13 @@ __global__ void __launch_bounds__(kTcThreads, 2) union_gemm_tc_kernel(const TcAr
 // packed tiles. Lane 4g + q ends with tokens g and g + 8 at the 8 consecutive
 // columns 8q .. 8q + 7 of each 32-column half. No shared-memory staging of
 // weights and no CTA barrier inside the loop: every warp streams on its own,
-// kMmaDepth K-blocks (4 KB) in flight.
+// with 16-bit x through a rolling pipeline of kMmaPipe K-blocks (two, 4 KB,
+// in flight while one is multiplied), with fp32 x in groups of kMmaDepth.
 constexpr int kMmaWarps = 8;
 constexpr int kMmaThreads = kMmaWarps * 32;
 constexpr int kMmaWarpCols = 64;
-constexpr int kMmaDepth = 2;
+constexpr int kMmaDepth = 2;  // fp32 x: K-blocks loaded per group
+constexpr int kMmaPipe = 3;   // 16-bit x: register slots of the rolling pipeline
 // token row stride of the reduction buffer: 2 (mod 32) words, so that the
 // float2 stores of a half-warp (tokens g = 0..3, column groups q = 0..3) hit
 // 16 distinct bank pairs
@@ -574,41 +576,67 @@ __global__ void __launch_bounds__(kMmaThreads, 2) union_gemm_mma_kernel(const Tc
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[m][j][e] = 0.f;
 
-  // the WPC warps of a chunk take groups of kMmaDepth K-blocks in turn
   const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-  for (int kb0 = wrow * kMmaDepth; kb0 < nblk; kb0 += WPC * kMmaDepth) {
-    uint4 w[kMmaDepth][2][2];  // [K-block][row half][column half]
-    uint4 xa[kMmaDepth], xl[kMmaDepth];
+  // one K-block: the weight pieces of its 16 rows and the x fragment(s)
+  auto load = [&](int kb, bool kv, uint4 (&ws)[2][2], uint4& xas, uint4& xls) {
 #pragma unroll
-    for (int u = 0; u < kMmaDepth; ++u) {
-      const int kb = kb0 + u;
+    for (int h = 0; h < 2; ++h) {
+      const int r = kb * kTcK + h * 8 + p;
+      const bool rv = kv && r < nrows;
+      const TW* src = Wb + (rv ? (long long)list_row[r] * N : 0);
+      ws[h][0] = (rv && col0) ? ld_weight16(src, pol) : z;
+      ws[h][1] = (rv && col1) ? ld_weight16(src + 32, pol) : z;
+    }
+    xas = kv ? ld_frag(pack + (long long)kb * tile_elems + lane * 8) : z;
+    if (SPLIT) xls = kv ? ld_frag(pack + (long long)kb * tile_elems + 256 + lane * 8) : z;
+  };
+  auto compute = [&](const uint4 (&ws)[2][2], const uint4& xas, const uint4& xls) {
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int r = kb * kTcK + h * 8 + p;
-        const bool rv = kb < nblk && r < nrows;
-        const TW* src = Wb + (rv ? (long long)list_row[r] * N : 0);
-        w[u][h][0] = (rv && col0) ? ld_weight16(src, pol) : z;
-        w[u][h][1] = (rv && col1) ? ld_weight16(src + 32, pol) : z;
-      }
-      if (kb < nblk) {
-        xa[u] = ld_frag(pack + (long long)kb * tile_elems + lane * 8);
-        if (SPLIT) xl[u] = ld_frag(pack + (long long)kb * tile_elems + 256 + lane * 8);
+    for (int m = 0; m < 2; ++m) {
+      const uint32_t r0[4] = {ws[0][m].x, ws[0][m].y, ws[0][m].z, ws[0][m].w};
+      const uint32_t r1[4] = {ws[1][m].x, ws[1][m].y, ws[1][m].z, ws[1][m].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t b0 = movmatrix_trans(r0[j]);
+        const uint32_t b1 = movmatrix_trans(r1[j]);
+        mma_16816(acc[m][j], xas.x, xas.y, xas.z, xas.w, b0, b1, TW());
+        if (SPLIT) mma_16816(acc[m][j], xls.x, xls.y, xls.z, xls.w, b0, b1, TW());
       }
     }
+  };
+  if constexpr (!SPLIT) {
+    // this warp's K-blocks wrow, wrow + WPC, ... through a rolling pipeline of
+    // kMmaPipe register slots: kMmaPipe - 1 K-blocks stay in flight while one
+    // is multiplied
+    const int nmine = nblk > wrow ? (nblk - wrow + WPC - 1) / WPC : 0;
+    uint4 w[kMmaPipe][2][2];
+    uint4 xa[kMmaPipe], xl[kMmaPipe];
 #pragma unroll
-    for (int u = 0; u < kMmaDepth; ++u) {
-      if (kb0 + u >= nblk) break;
+    for (int u = 0; u < kMmaPipe - 1; ++u) load(wrow + u * WPC, u < nmine, w[u], xa[u], xl[u]);
+    for (int i0 = 0; i0 < nmine; i0 += kMmaPipe) {
 #pragma unroll
-      for (int m = 0; m < 2; ++m) {
-        const uint32_t r0[4] = {w[u][0][m].x, w[u][0][m].y, w[u][0][m].z, w[u][0][m].w};
-        const uint32_t r1[4] = {w[u][1][m].x, w[u][1][m].y, w[u][1][m].z, w[u][1][m].w};
+      for (int u = 0; u < kMmaPipe; ++u) {
+        const int i = i0 + u;
+        if (i >= nmine) break;
+        constexpr int kAhead = kMmaPipe - 1;
+        const int ls = (u + kAhead) % kMmaPipe;
+        load(wrow + (i + kAhead) * WPC, i + kAhead < nmine, w[ls], xa[ls], xl[ls]);
+        compute(w[u], xa[u], xl[u]);
+      }
+    }
+  } else {
+    // fp32 x (hi + lo fragments, two MMAs per tile): the WPC warps of a chunk
+    // take groups of kMmaDepth K-blocks in turn, loaded together, then
+    // multiplied (a rolling pipeline costs this variant more than it saves)
+    for (int kb0 = wrow * kMmaDepth; kb0 < nblk; kb0 += WPC * kMmaDepth) {
+      uint4 w[kMmaDepth][2][2];
+      uint4 xa[kMmaDepth], xl[kMmaDepth];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint32_t b0 = movmatrix_trans(r0[j]);
-          const uint32_t b1 = movmatrix_trans(r1[j]);
-          mma_16816(acc[m][j], xa[u].x, xa[u].y, xa[u].z, xa[u].w, b0, b1, TW());
-          if (SPLIT) mma_16816(acc[m][j], xl[u].x, xl[u].y, xl[u].z, xl[u].w, b0, b1, TW());
-        }
+      for (int u = 0; u < kMmaDepth; ++u) load(kb0 + u, kb0 + u < nblk, w[u], xa[u], xl[u]);
+#pragma unroll
+      for (int u = 0; u < kMmaDepth; ++u) {
+        if (kb0 + u >= nblk) break;
+        compute(w[u], xa[u], xl[u]);
       }
     }
   }
