@@ -125,6 +125,20 @@ int sfx_check_device_status(void* ws, unsigned int* bits_out, void* stream);
 int sfx_device_sm_count(void);
 const char* sfx_build_info(void);
 
+/* The launch plan sfx_sparse_gemv takes for a B x K input and a [K x N]
+ * matrix (host only: no GPU work, no allocation; the plan depends on the
+ * device's SM count, 148 when no device is visible). flags as for
+ * sfx_sparse_gemv (SFX_FLAG_CUDA_CORES changes the plan); idx_mode != 0 for
+ * a caller index list (B must be 1). out (host int[6]):
+ *   out[0] kernel: 0 CUDA-core GEMV, 1 batch union on tcgen05, 2 batch union
+ *          on mma.sync
+ *   out[1] columns per CTA tile      out[2] K splits     out[3] column tiles
+ *   out[4] 64-column chunks per CTA (kernel 2, else 0)
+ *   out[5] rows of K per split (threshold mode; kernel 0 with a caller list:
+ *          the list capacity of a split)
+ * Returns SFX_OK or SFX_ERR_ARG. */
+int sfx_gemv_plan(int B, long long K, long long N, int flags, int idx_mode, int* out);
+
 /* ------------------------------------------------------------------------
  * a1. Threshold calibration                                 [TEAL] slide 8
  *

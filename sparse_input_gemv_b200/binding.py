@@ -39,6 +39,7 @@ _SIGS = {
     "sfx_check_device_status": (_I, [_VP, _VP, _VP]),
     "sfx_device_sm_count": (_I, []),
     "sfx_build_info": (ctypes.c_char_p, []),
+    "sfx_gemv_plan": (_I, [_I, _LL, _LL, _I, _I, _VP]),
     "sfx_calibrate_thresholds": (_I, [_VP, _I, _LL, _LL, _VP, _I, _VP, _VP, _SZ, _VP]),
     "sfx_mask_compact": (_I, [_VP, _I, _I, _I, _I, _F, _I, _VP, _VP, _D, _VP, _VP, _VP, _VP, _VP,
                               _VP, _SZ, _VP]),
@@ -346,3 +347,16 @@ def sfx_static_ffn(x, W_aT, W_d, idx, cnt, W_bT=None, flags=0, out_dtype=None, y
 
 def sfx_device_sm_count() -> int:
     return int(load().sfx_device_sm_count())
+
+
+GEMV_KERNELS = ("cuda_cores", "union_tcgen05", "union_mma")
+
+
+def sfx_gemv_plan(B, K, N, flags=0, idx_mode=False) -> dict:
+    """The launch plan sfx_sparse_gemv takes for these sizes (host only)."""
+    out = (ctypes.c_int * 6)()
+    _check("sfx_gemv_plan", load().sfx_gemv_plan(int(B), int(K), int(N), int(flags),
+                                                  1 if idx_mode else 0,
+                                                  ctypes.cast(out, ctypes.c_void_p)))
+    return {"kernel": GEMV_KERNELS[out[0]], "NT": out[1], "S": out[2], "col_tiles": out[3],
+            "chunks": out[4], "slice": out[5]}

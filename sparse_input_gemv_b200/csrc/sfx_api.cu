@@ -81,6 +81,18 @@ int sfx_device_sm_count(void) { return sm_count(); }
 
 const char* sfx_build_info(void) { return "sfx 0.1 sm_100a"; }
 
+int sfx_gemv_plan(int B, long long K, long long N, int flags, int idx_mode, int* out) {
+  if (!out || B < 1 || B > 16 || K < 1 || N < 8 || (idx_mode && B != 1)) return SFX_ERR_ARG;
+  const GemvPlan p = gemv_launch_plan(K, N, B, idx_mode != 0, (flags & SFX_FLAG_CUDA_CORES) != 0);
+  out[0] = p.kind;
+  out[1] = p.NT;
+  out[2] = p.S;
+  out[3] = p.col_tiles;
+  out[4] = p.kind == 2 ? p.chunks : 0;
+  out[5] = (p.kind == 0 && idx_mode) ? p.list_cap : p.slice;
+  return SFX_OK;
+}
+
 size_t sfx_workspace_bytes(int op, long long a, long long b, long long c, long long d,
                            long long e, long long f) {
   switch (op) {
