@@ -83,7 +83,10 @@ const char* sfx_build_info(void) { return "sfx 0.1 sm_100a"; }
 
 int sfx_gemv_plan(int B, long long K, long long N, int flags, int idx_mode, int* out) {
   if (!out || B < 1 || B > 16 || K < 1 || N < 8 || (idx_mode && B != 1)) return SFX_ERR_ARG;
-  const GemvPlan p = gemv_launch_plan(K, N, B, idx_mode != 0, (flags & SFX_FLAG_CUDA_CORES) != 0);
+  // the choice launch_sparse_gemv makes: the batch union for union_min_batch()
+  // tokens or more in threshold mode unless SFX_FLAG_CUDA_CORES, else CUDA cores
+  const bool uni = B >= union_min_batch() && !idx_mode && !(flags & SFX_FLAG_CUDA_CORES);
+  const GemvPlan p = uni ? plan_union_tc(K, N) : plan_gemv(K, N, B, idx_mode != 0);
   out[0] = p.kind;
   out[1] = p.NT;
   out[2] = p.S;

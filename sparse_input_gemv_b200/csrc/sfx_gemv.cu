@@ -122,19 +122,10 @@ SFX_DECL(gemv_f16_f32_small) SFX_DECL(gemv_f16_f32_large)
 // (griddepcontrol.wait) before it reads any input or workspace, so it is
 // correct after any predecessor, and its CTAs get scheduled while the
 // previous kernel finishes its tail.
-bool gemv_uses_union(int B, bool idx_mode, bool cuda_cores) {
-  return B >= union_min_batch() && !idx_mode && !cuda_cores;
-}
-
-GemvPlan gemv_launch_plan(long long K, long long N, int B, bool idx_mode, bool cuda_cores) {
-  return gemv_uses_union(B, idx_mode, cuda_cores) ? plan_union_tc(K, N)
-                                                  : plan_gemv(K, N, B, idx_mode);
-}
-
 int launch_sparse_gemv(int wdt, int xdt, const GemvPlan& p, GemvArgs a, cudaStream_t s, bool) {
   const bool pdl = true;
-  // a batch of 3..16 tokens in threshold mode: the union tile on tensor cores
-  if (gemv_uses_union(a.B, a.idx != nullptr, a.no_tc != 0))
+  // a batch of 4..16 tokens in threshold mode: the union tile on tensor cores
+  if (a.B >= union_min_batch() && a.idx == nullptr && !a.no_tc)
     return launch_union_tc(wdt, xdt, plan_union_tc(a.K, a.N), a, s);
   if (p.col_tiles > kCounterSlots) return SFX_ERR_UNSUPPORTED;
   a.S = p.S;

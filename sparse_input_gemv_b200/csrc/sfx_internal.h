@@ -59,9 +59,6 @@ GemvPlan plan_gemv(long long K, long long N, int B, bool idx_mode);
 size_t gemv_workspace_bytes(long long K, long long N, int B);  // excludes the header
 int launch_sparse_gemv(int wdt, int xdt, const GemvPlan& plan, GemvArgs a, cudaStream_t stream,
                        bool pdl);
-// Which kernel family and plan launch_sparse_gemv takes for these sizes.
-bool gemv_uses_union(int B, bool idx_mode, bool cuda_cores);
-GemvPlan gemv_launch_plan(long long K, long long N, int B, bool idx_mode, bool cuda_cores);
 
 // batch-union GEMM (sfx_union_tc.cu), used for B >= union_min_batch()
 // Smallest batch that takes the union path (measured on B200: the CUDA-core
