@@ -128,12 +128,22 @@ KERNEL_SOURCES = ("sparse_input_gemv_b200/csrc/sfx_gemv_kernel.cuh",
 PROFILE_SUMMARIES = {"ffn_gate_up": "profiles/sparse_gemv_gate_up_llama3_8b.md"}
 
 
+def _code_only(src: str) -> str:
+    """C/C++/CUDA source without comments and blank lines (string literals are
+    kept; the sources hold no comment markers inside strings)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def kernel_source_hash() -> str:
+    """Hash of the GEMV sources' code: a comment edit keeps it, a code edit changes it."""
     import hashlib
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -124,7 +124,8 @@ SFX_DECL(gemv_f16_f32_small) SFX_DECL(gemv_f16_f32_large)
 // previous kernel finishes its tail.
 int launch_sparse_gemv(int wdt, int xdt, const GemvPlan& p, GemvArgs a, cudaStream_t s, bool) {
   const bool pdl = true;
-  // a batch of 4..16 tokens in threshold mode: the union tile on tensor cores
+  // a batch of union_min_batch() .. 16 tokens in threshold mode: the union
+  // tile on the tensor cores
   if (a.B >= union_min_batch() && a.idx == nullptr && !a.no_tc)
     return launch_union_tc(wdt, xdt, plan_union_tc(a.K, a.N), a, s);
   if (p.col_tiles > kCounterSlots) return SFX_ERR_UNSUPPORTED;
