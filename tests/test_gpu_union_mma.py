@@ -75,6 +75,19 @@ def test_union_mma_matches_oracle(B, K, N, p, wdt, xdt, out):
     case(B, K, N, p, wdt, xdt, out)
 
 
+@pytest.mark.parametrize("chunks", [1, 2, 4, 8])
+@pytest.mark.parametrize("B,K,N,p,wdt,xdt,out,flags", [
+    (16, 4096, 1000, 0.5, "bf16", "bf16", "f32", 0),           # N % 64 != 0
+    (5, 3000, 2056, 0.3, "f16", "f32", "f16", 0),              # fp32 x, ragged K
+    (9, 2048, 4096, 0.4, "bf16", "bf16", "f32", sb.SFX_FLAG_SWIGLU),
+])
+def test_union_mma_every_tile_width(chunks, B, K, N, p, wdt, xdt, out, flags, monkeypatch):
+    # 8 / chunks warps share each 64-column chunk and are summed in shared memory
+    monkeypatch.setenv("SFX_MMA_CHUNKS", str(chunks))
+    assert sb.sfx_gemv_plan(B, K, N, flags)["chunks"] == chunks
+    case(B, K, N, p, wdt, xdt, out, flags=flags, seed=f"mma-c{chunks}")
+
+
 def test_union_mma_epilogues():
     case(4, 2560, 1024, 0.4, "f16", "f16", "f32", flags=sb.SFX_FLAG_GELU, seed="mma-gelu")
     case(16, 4096, 28672, 0.5, "bf16", "bf16", "f32", flags=sb.SFX_FLAG_SWIGLU, seed="mma-gu")
