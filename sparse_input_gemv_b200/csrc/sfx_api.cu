@@ -4,6 +4,8 @@
 #include "sfx_common.cuh"
 #include "sfx_internal.h"
 
+#include <mutex>
+
 #include <cmath>
 #include <vector>
 
@@ -59,6 +61,17 @@ int launch_pack_gate_up(const void* W_g, const void* W_u, int, int d, int ffn, v
       reinterpret_cast<uint16_t*>(W_gu));
   return cudaGetLastError() == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
 }
+int ensure_dynamic_smem(const void* kern, size_t bytes, size_t* configured) {
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (bytes <= *configured) return SFX_OK;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) !=
+      cudaSuccess)
+    return SFX_ERR_CUDA;
+  *configured = bytes;
+  return SFX_OK;
+}
+
 }  // namespace sfx
 
 extern "C" {

@@ -157,8 +157,8 @@ static int calibrate_t(const T* data, long long n, const long long* ranks, int P
   if (cudaMemcpyAsync(rank, ranks, sizeof(long long) * P, cudaMemcpyHostToDevice, s) != cudaSuccess)
     return SFX_ERR_CUDA;
   auto k1 = calib_hist1_kernel<T>;
-  if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, 32768 * 4) !=
-      cudaSuccess)
+  static size_t k1_configured = 0;
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(k1), 32768 * 4, &k1_configured) != SFX_OK)
     return SFX_ERR_CUDA;
   const int grid = sm_count();
   k1<<<grid, kCalibThreads, 32768 * 4, s>>>(data, n, f32 ? 16 : 0, hist1);
@@ -167,9 +167,9 @@ static int calibrate_t(const T* data, long long n, const long long* ranks, int P
     for (int shift = 8; shift >= 0; shift -= 8) {
       if (cudaMemsetAsync(histp, 0, (size_t)P * 256 * 4, s) != cudaSuccess) return SFX_ERR_CUDA;
       const size_t smem_p = ((size_t)P * 256 + P) * 4;
-      if (smem_p > 48 * 1024 &&
-          cudaFuncSetAttribute(calib_histp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem_p) != cudaSuccess)
+      static size_t histp_configured = 48 * 1024;  // the default limit
+      if (ensure_dynamic_smem(reinterpret_cast<const void*>(calib_histp_kernel), smem_p,
+                              &histp_configured) != SFX_OK)
         return SFX_ERR_CUDA;
       calib_histp_kernel<<<grid, kCalibThreads, smem_p, s>>>(reinterpret_cast<const float*>(data), n,
                                                         shift, P, prefix, histp);

@@ -55,6 +55,12 @@ struct GemvPlan {
 };
 
 int sm_count();
+
+// Raises the kernel's dynamic shared-memory limit to at least `bytes` (never
+// lowers it). *configured remembers the limit set so far; calls from several
+// host threads are serialised, so the remembered limit is never above the one
+// in force. Returns SFX_OK or SFX_ERR_CUDA.
+int ensure_dynamic_smem(const void* kern, size_t bytes, size_t* configured);
 GemvPlan plan_gemv(long long K, long long N, int B, bool idx_mode);
 size_t gemv_workspace_bytes(long long K, long long N, int B);  // excludes the header
 int launch_sparse_gemv(int wdt, int xdt, const GemvPlan& plan, GemvArgs a, cudaStream_t stream,

@@ -459,12 +459,8 @@ static int launch_experts(int B, const void* x, int d, int ffn, int ffn_s, int t
   const size_t smem = (size_t)B * (d + kXPad) * sizeof(TW);  // x of an item's tokens (<= B)
   static size_t configured = 0;  // one opt-in per kernel instantiation
   // opt in whenever the size grows: dynamic plus ~17 KB static may pass 48 KB
-  if (smem > configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return SFX_ERR_CUDA;
-    configured = smem;
-  }
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem, &configured) != SFX_OK)
+    return SFX_ERR_CUDA;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kMoeThreads, smem) !=
           cudaSuccess ||
@@ -503,12 +499,9 @@ int run_moe(const void* x, int dt, const float* logits, int B, int d, int E, int
   const size_t route_smem = (size_t)B * E * 4 + (size_t)B * top_k * 8;
   if (route_smem > 48 * 1024) {
     static size_t route_configured = 0;
-    if (route_smem > route_configured) {
-      if (cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)route_smem) != cudaSuccess)
-        return SFX_ERR_CUDA;
-      route_configured = route_smem;
-    }
+    if (ensure_dynamic_smem(reinterpret_cast<const void*>(moe_route_kernel), route_smem,
+                            &route_configured) != SFX_OK)
+      return SFX_ERR_CUDA;
   }
   const int route_threads = 32 * (B > 4 ? B : 4);
   moe_route_kernel<<<1, route_threads, route_smem, s>>>(logits, B, E, top_k, renorm, d, w,

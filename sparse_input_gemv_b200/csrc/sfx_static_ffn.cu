@@ -217,12 +217,8 @@ static int launch_static(const void* x, int B, int d, int ffn, const void* WaT, 
   const size_t smem = (size_t)B * (d + kXPad) * sizeof(TW);
   static size_t configured = 0;
   // opt in whenever the size grows: dynamic plus ~17 KB static may pass 48 KB
-  if (smem > configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-        cudaSuccess)
-      return SFX_ERR_CUDA;
-    configured = smem;
-  }
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), smem, &configured) != SFX_OK)
+    return SFX_ERR_CUDA;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kRowThreads, smem) !=
           cudaSuccess ||
