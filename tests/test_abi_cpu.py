@@ -36,6 +36,33 @@ def test_header_declares_the_five_calls():
         assert fn in names
 
 
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    # the boundary needs no C++ or CUDA types: a C99 program compiles against the
+    # header and links against the library with the system C compiler
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_sfx.c"
+    src.write_text(
+        '#include "sfx.h"\n'
+        "int main(void) {\n"
+        "  int plan[6];\n"
+        "  if (sfx_gemv_plan(1, 4096, 4096, 0, 0, plan) != SFX_OK) return 1;\n"
+        "  return sfx_workspace_bytes(SFX_OP_SPARSE_GEMV, 1, 4096, 4096, SFX_BF16, 0, 0) >= 256 ? 0 : 2;\n"
+        "}\n")
+    exe = tmp_path / "use_sfx"
+    lib_dir = os.path.dirname(sb.LIB_PATH)
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe),
+                        "-L", lib_dir, "-lsfx", f"-Wl,-rpath,{lib_dir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert run.returncode == 0, (run.returncode, run.stderr)
+
+
 def test_library_exports_every_declared_symbol(lib):
     names = header_functions()
     assert len(names) >= 12
