@@ -39,7 +39,7 @@ __all__ = [
     "union_mask", "topk_mask", "keep_count", "gxo_score", "corrected_gxo_score",
     "corrected_gxo_score_f32", "ffn_static_mask",
     "glass_ranks", "glass_fuse", "glass_mask", "masked_gemv", "silu", "gelu_erf",
-    "gelu_tanh", "ffn_swiglu", "ffn_swiglu_down", "ffn_gelu_topk_down",
+    "gelu_tanh", "ffn_swiglu", "ffn_gelu_topk_down",
     "moe_route", "moe_expert", "moe_layer", "round_to",
 ]
 
@@ -275,13 +275,6 @@ def ffn_static_mask(x, W_a, W_d, keep, act="gelu", W_b=None):
         raise ValueError(act)
     m = np.broadcast_to(np.asarray(keep, dtype=bool), h.shape)
     return masked_gemv(h, m, W_d), h
-
-
-def ffn_swiglu_down(h, t_h, W_d):
-    """Down stage alone on a given h (used to check a stage on the GPU's own h)."""
-    h = np.atleast_2d(np.asarray(h, dtype=np.float64))
-    m_h = magnitude_mask(h, t_h)
-    return masked_gemv(h, m_h, W_d), m_h
 
 
 def ffn_gelu_topk_down(h, g, W2, k):
