@@ -139,6 +139,30 @@ const char* sfx_build_info(void);
  * Returns SFX_OK or SFX_ERR_ARG. */
 int sfx_gemv_plan(int B, long long K, long long N, int flags, int idx_mode, int* out);
 
+/* Plan overrides for tuning sweeps and tests (host only, process-wide).
+ * The library reads no environment variable: a launch plan is the planner's
+ * choice unless a caller overrides one of these knobs. Value 0 restores the
+ * planner's choice for that knob. Overrides apply to calls planned after
+ * this one returns; setting them while other host threads launch is a race
+ * on which plan those launches take (each launch still sees valid values).
+ *  SFX_PLAN_UNION_KERNEL  batch-union kernel: 1 tcgen05, 2 mma.sync
+ *  SFX_PLAN_UNION_MIN_B   smallest batch on the union path (2..16)
+ *  SFX_PLAN_GEMV_NT       CUDA-core GEMV column tile: 256, 512, 1024, 2048
+ *  SFX_PLAN_GEMV_S        CUDA-core GEMV K splits (>= 1; the list capacity
+ *                         may still raise it)
+ *  SFX_PLAN_UNION_S       batch-union K splits (>= 1, same caveat)
+ *  SFX_PLAN_MMA_CHUNKS    mma.sync union tile in 64-column chunks: 1, 2, 4, 8
+ * Returns SFX_OK, or SFX_ERR_ARG for an unknown key or a value out of range. */
+typedef enum {
+  SFX_PLAN_UNION_KERNEL = 0,
+  SFX_PLAN_UNION_MIN_B = 1,
+  SFX_PLAN_GEMV_NT = 2,
+  SFX_PLAN_GEMV_S = 3,
+  SFX_PLAN_UNION_S = 4,
+  SFX_PLAN_MMA_CHUNKS = 5
+} sfx_plan_key;
+int sfx_set_plan_override(int key, int value);
+
 /* ------------------------------------------------------------------------
  * a1. Threshold calibration                                 [TEAL] slide 8
  *
@@ -250,8 +274,11 @@ int sfx_sparse_gemv(const void* x, int xdt, int B, int K, const void* W, int wdt
  *    `stream`, then launches. All calls share the one array and it keeps the
  *    last call's contents, so calls that overlap on the GPU (other streams,
  *    other host threads) race with each other; issue them one after another.
- *  - Out-of-range list indices are skipped as in sfx_sparse_gemv, but their
- *    status bit is not reported.
+ *  - The device status word lives in the array too and no call reads it
+ *    back: an out-of-range list index (skipped, as in sfx_sparse_gemv) and a
+ *    bounded wait that gave up (SFX_DEV_TIMEOUT: y is then left partly
+ *    unwritten) both go unreported, and the next call clears the word.
+ *    Callers that need those checks use sfx_sparse_gemv with a workspace.
  * ---------------------------------------------------------------------- */
 int sfx_sparse_gemv_noalloc(const void* x, int xdt, int B, int K, const void* W, int wdt, int N,
                             float t, const int32_t* idx, const int32_t* cnt,

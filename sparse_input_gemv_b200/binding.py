@@ -40,6 +40,7 @@ _SIGS = {
     "sfx_device_sm_count": (_I, []),
     "sfx_build_info": (ctypes.c_char_p, []),
     "sfx_gemv_plan": (_I, [_I, _LL, _LL, _I, _I, _VP]),
+    "sfx_set_plan_override": (_I, [_I, _I]),
     "sfx_calibrate_thresholds": (_I, [_VP, _I, _LL, _LL, _VP, _I, _VP, _VP, _SZ, _VP]),
     "sfx_mask_compact": (_I, [_VP, _I, _I, _I, _I, _F, _I, _VP, _VP, _D, _VP, _VP, _VP, _VP, _VP,
                               _VP, _SZ, _VP]),
@@ -238,7 +239,9 @@ def sfx_sparse_gemv_noalloc(x, W, t=-math.inf, idx=None, cnt=None, out_dtype=Non
     x2 = x[None] if squeeze else x
     _need_cuda(x2, W, idx, cnt)
     B, K = x2.shape
-    N = W.shape[1]
+    K2, N = W.shape
+    if K2 != K:
+        raise ValueError("x and W disagree on K")
     out_dtype = torch.float32 if flags & SFX_FLAG_SWIGLU else (out_dtype or W.dtype)
     if y is None:
         y = torch.empty((B, N // 2 if flags & SFX_FLAG_SWIGLU else N), dtype=out_dtype,
@@ -350,6 +353,34 @@ def sfx_device_sm_count() -> int:
 
 
 GEMV_KERNELS = ("cuda_cores", "union_tcgen05", "union_mma")
+
+SFX_PLAN_UNION_KERNEL, SFX_PLAN_UNION_MIN_B, SFX_PLAN_GEMV_NT, SFX_PLAN_GEMV_S, SFX_PLAN_UNION_S, \
+    SFX_PLAN_MMA_CHUNKS = range(6)
+UNION_TCGEN05, UNION_MMA = 1, 2
+
+
+def sfx_set_plan_override(key: int, value: int):
+    """Override one launch-plan knob (0 = the planner's choice); tuning and tests only."""
+    _check("sfx_set_plan_override", load().sfx_set_plan_override(int(key), int(value)))
+
+
+class plan_overrides:
+    """Context manager: set plan overrides {key: value} and restore the planner on exit."""
+
+    def __init__(self, **kv):
+        names = {"union_kernel": SFX_PLAN_UNION_KERNEL, "union_min_b": SFX_PLAN_UNION_MIN_B,
+                 "gemv_nt": SFX_PLAN_GEMV_NT, "gemv_s": SFX_PLAN_GEMV_S,
+                 "union_s": SFX_PLAN_UNION_S, "mma_chunks": SFX_PLAN_MMA_CHUNKS}
+        self.kv = {names[k]: v for k, v in kv.items()}
+
+    def __enter__(self):
+        for k, v in self.kv.items():
+            sfx_set_plan_override(k, v)
+        return self
+
+    def __exit__(self, *exc):
+        for k in self.kv:
+            sfx_set_plan_override(k, 0)
 
 
 def sfx_gemv_plan(B, K, N, flags=0, idx_mode=False) -> dict:

@@ -4,9 +4,9 @@
 #include "sfx_common.cuh"
 #include "sfx_internal.h"
 
-#include <mutex>
-
+#include <atomic>
 #include <cmath>
+#include <mutex>
 #include <vector>
 
 using namespace sfx;
@@ -54,6 +54,14 @@ void carve_gemv(void* ws, unsigned char* body, GemvArgs& a) {
 }  // namespace
 
 namespace sfx {
+
+static constexpr int kPlanKeys = SFX_PLAN_MMA_CHUNKS + 1;
+static std::atomic<int> g_plan_override[kPlanKeys];
+
+int plan_override(int key) {
+  return (key >= 0 && key < kPlanKeys) ? g_plan_override[key].load(std::memory_order_relaxed) : 0;
+}
+
 int launch_pack_gate_up(const void* W_g, const void* W_u, int, int d, int ffn, void* W_gu,
                         cudaStream_t s) {
   pack_gate_up_kernel<<<sm_count() * 4, 256, 0, s>>>(
@@ -106,6 +114,22 @@ int sfx_gemv_plan(int B, long long K, long long N, int flags, int idx_mode, int*
   out[3] = p.col_tiles;
   out[4] = p.kind == 2 ? p.chunks : 0;
   out[5] = (p.kind == 0 && idx_mode) ? p.list_cap : p.slice;
+  return SFX_OK;
+}
+
+int sfx_set_plan_override(int key, int value) {
+  bool ok = value == 0;
+  switch (key) {
+    case SFX_PLAN_UNION_KERNEL: ok = ok || value == 1 || value == 2; break;
+    case SFX_PLAN_UNION_MIN_B: ok = ok || (value >= 2 && value <= 16); break;
+    case SFX_PLAN_GEMV_NT: ok = ok || value == 256 || value == 512 || value == 1024 || value == 2048; break;
+    case SFX_PLAN_GEMV_S:
+    case SFX_PLAN_UNION_S: ok = ok || value >= 1; break;
+    case SFX_PLAN_MMA_CHUNKS: ok = ok || value == 1 || value == 2 || value == 4 || value == 8; break;
+    default: return SFX_ERR_ARG;
+  }
+  if (!ok) return SFX_ERR_ARG;
+  g_plan_override[key].store(value, std::memory_order_relaxed);
   return SFX_OK;
 }
 

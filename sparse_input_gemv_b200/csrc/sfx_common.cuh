@@ -82,6 +82,16 @@ __device__ __forceinline__ void raise_status(unsigned* status, unsigned bits) {
   if (status) atomicOr(status, bits);
 }
 
+// Split-K arrival on a tile counter, after a CTA barrier: the release half
+// publishes the CTA's partial sums (ordered before it by the barrier), the
+// acquire half lets the last arriver read everyone else's. Returns the count
+// before this arrival.
+__device__ __forceinline__ int arrive_acq_rel(int32_t* counter) {
+  int prev;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(prev) : "l"(counter) : "memory");
+  return prev;
+}
+
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

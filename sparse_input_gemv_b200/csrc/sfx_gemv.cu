@@ -3,7 +3,6 @@
 #include "sfx_gemv_kernel.cuh"
 
 #include <algorithm>
-#include <cstdlib>
 
 namespace sfx {
 
@@ -32,13 +31,6 @@ static int bmax_for(int B) {
 
 static long long round_up(long long v, long long m) { return (v + m - 1) / m * m; }
 
-static int env_int(const char* name, int dflt) {
-  const char* s = std::getenv(name);
-  return (s && *s) ? std::atoi(s) : dflt;
-}
-
-static constexpr size_t kListBudget = 48 * 1024;
-
 GemvPlan plan_gemv(long long K, long long N, int B, bool idx_mode) {
   GemvPlan p;
   p.BMAX = bmax_for(B);
@@ -66,14 +58,14 @@ GemvPlan plan_gemv(long long K, long long N, int B, bool idx_mode) {
       nt = cand;
     }
   }
-  nt = env_int("SFX_GEMV_NT", nt);
+  if (plan_override(SFX_PLAN_GEMV_NT)) nt = plan_override(SFX_PLAN_GEMV_NT);
   p.NT = nt;
   p.col_tiles = (int)((N + nt - 1) / nt);
   long long S = std::max<long long>(1, slots / p.col_tiles);
   S = std::min<long long>(S, std::max<long long>(1, (K + 31) / 32));
-  S = env_int("SFX_GEMV_S", (int)S);
+  if (plan_override(SFX_PLAN_GEMV_S)) S = plan_override(SFX_PLAN_GEMV_S);
   const size_t per_row = 4 * (size_t)(1 + p.BMAX);
-  const long long cap_max = (long long)(kListBudget / per_row) / 32 * 32;
+  const long long cap_max = list_cap_max(p.BMAX);
   long long slice = round_up((K + S - 1) / S, 32);
   if (slice > cap_max) slice = cap_max;
   S = (K + slice - 1) / slice;
@@ -105,7 +97,7 @@ size_t gemv_workspace_bytes(long long K, long long N, int B) {
 }
 
 int union_min_batch() {
-  const int v = env_int("SFX_UNION_MIN_B", 0);  // tuning sweeps only
+  const int v = plan_override(SFX_PLAN_UNION_MIN_B);
   return v >= 2 ? v : (union_uses_mma() ? kMmaMinBatch : kTcMinBatch);
 }
 

@@ -42,6 +42,16 @@ __host__ __device__ constexpr int gemv_threads(int bmax) { return bmax >= 8 ? 25
 // per SM), 8 for the 4-slot kernel (one CTA per SM, with the registers to
 // spare), so that an SM keeps ~64 KB of weight reads in flight either way
 __host__ __device__ constexpr int rows_in_flight(int bmax) { return bmax == 4 ? 8 : 4; }
+// Shared memory of a CTA's active list: one row index plus BMAX fp32 x values
+// per active row, so a K-split holds at most list_cap_max rows.
+constexpr size_t kListBudget = 48 * 1024;
+__host__ __device__ constexpr int list_cap_max(int bmax) {
+  return (int)(kListBudget / (4 * (1 + (size_t)bmax))) / 32 * 32;
+}
+// Rows of the slice one thread tests: each thread owns a contiguous run.
+__host__ __device__ constexpr int rows_per_thread_max(int bmax) {
+  return (list_cap_max(bmax) + gemv_threads(bmax) - 1) / gemv_threads(bmax);
+}
 
 __device__ __forceinline__ float apply_epi(int epi, float v) {
   if (epi == EPI_GELU) return gelu_erf_f(v);
@@ -92,70 +102,75 @@ __global__ void __launch_bounds__(gemv_threads(BMAX), (BMAX <= 2) ? 2 : 1)
 
   // ---------------------------------------------------------------- 1. active list
   if (a.idx == nullptr) {
+    // Every thread tests a contiguous run of at most kPer rows of the slice;
+    // all its x loads are independent, so the CTA pays one L2 round trip for
+    // x. One block scan of the per-thread counts then places each active row,
+    // and the list comes out ascending.
+    constexpr int kPer = rows_per_thread_max(BMAX);
     const long long k0 = (long long)split * a.slice;
     const long long k1 = min(a.K, k0 + a.slice);
+    const int n = (int)max(0LL, k1 - k0);
+    const int r = (n + kThreads - 1) / kThreads;  // <= kPer (slice <= list_cap_max)
+    const long long i0 = k0 + (long long)tid * r;
     const TX* xp = reinterpret_cast<const TX*>(a.x);
-    int base = 0;
-    // x of the next chunk is loaded while the current chunk is compacted
-    float xnext[BMAX];
+    float xv[kPer][BMAX];
 #pragma unroll
-    for (int b = 0; b < BMAX; ++b)
-      xnext[b] = (b < a.B && k0 + tid < k1) ? to_f32(xp[(long long)b * a.K + k0 + tid]) : 0.f;
-    for (long long c0 = k0; c0 < k1; c0 += kThreads) {
-      const long long i = c0 + tid;
-      const bool in = i < k1;
-      float xcur[BMAX];
+    for (int u = 0; u < kPer; ++u)
 #pragma unroll
-      for (int b = 0; b < BMAX; ++b) {
-        xcur[b] = xnext[b];
-        const long long inext = i + kThreads;
-        xnext[b] = (b < a.B && inext < k1) ? to_f32(xp[(long long)b * a.K + inext]) : 0.f;
-      }
-      float xv[BMAX];
-      bool act = false;
+      for (int b = 0; b < BMAX; ++b)
+        xv[u][b] = (u < r && i0 + u < k1 && b < a.B) ? to_f32(xp[(long long)b * a.K + i0 + u]) : 0.f;
+    unsigned act = 0;
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      bool any = false;
 #pragma unroll
       for (int b = 0; b < BMAX; ++b) {
-        float v = 0.f;
-        bool m = false;
-        if (b < a.B) {
-          if (in) {
-            v = xcur[b];
-            m = fabsf(v) > a.t;
-          }
-          if (a.bitmap_out != nullptr && tile == 0) {
-            const unsigned bal = __ballot_sync(0xffffffffu, m);
-            const long long w0 = c0 + (long long)warp * 32;
-            if (lane == 0 && w0 < k1)
-              a.bitmap_out[(long long)b * ((a.K + 31) >> 5) + (w0 >> 5)] = bal;
-          }
-        }
-        act |= m;
-        xv[b] = (m || a.union_mask) ? v : 0.f;
+        const bool m = (u < r && i0 + u < k1 && b < a.B) && fabsf(xv[u][b]) > a.t;
+        any |= m;
+        if (!m && !a.union_mask) xv[u][b] = 0.f;
       }
-      if (a.union_mask && !act) {
-#pragma unroll
-        for (int b = 0; b < BMAX; ++b) xv[b] = 0.f;
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, act);
-      if (lane == 0) s_warp_tot[warp] = __popc(bal);
-      __syncthreads();
-      int woff = 0, tot = 0;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const int c = s_warp_tot[w];
-        woff += (w < warp) ? c : 0;
-        tot += c;
-      }
-      if (act) {
-        const int pos = base + woff + __popc(bal & lanemask_lt());
-        list_row[pos] = (int32_t)i;
-#pragma unroll
-        for (int b = 0; b < BMAX; ++b) list_x[pos * BMAX + b] = xv[b];
-      }
-      base += tot;
-      __syncthreads();
+      if (any) act |= 1u << u;
     }
-    if (tid == 0) s_count = base;
+    // exclusive scan of the counts: warp shuffles, then the warp totals
+    const int mine = __popc(act);
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_warp_tot[warp] = incl;
+    __syncthreads();
+    int pos = incl - mine, tot = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const int c = s_warp_tot[w];
+      pos += (w < warp) ? c : 0;
+      tot += c;
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      if ((act >> u) & 1u) {
+        list_row[pos] = (int32_t)(i0 + u);
+#pragma unroll
+        for (int b = 0; b < BMAX; ++b) list_x[pos * BMAX + b] = xv[u][b];
+        ++pos;
+      }
+    }
+    if (tid == 0) s_count = tot;
+    // the fused mask, if asked for: the first column tile's CTAs write their
+    // slice's bitmap words (k0 is a multiple of 32, so no word is shared)
+    if (a.bitmap_out != nullptr && tile == 0) {
+      const long long words = (a.K + 31) >> 5;
+      for (long long w0 = k0 + (long long)warp * 32; w0 < k1; w0 += kThreads) {
+        const long long i = w0 + lane;
+        for (int b = 0; b < a.B; ++b) {
+          const bool m = i < k1 && fabsf(to_f32(xp[(long long)b * a.K + i])) > a.t;
+          const unsigned bal = __ballot_sync(0xffffffffu, m);
+          if (lane == 0) a.bitmap_out[(long long)b * words + (w0 >> 5)] = bal;
+        }
+      }
+    }
   } else {
     // caller-provided ascending list (B == 1): this split takes an even share
     const long long c = min((long long)max(*a.cnt, 0), a.K);
@@ -265,15 +280,10 @@ __global__ void __launch_bounds__(gemv_threads(BMAX), (BMAX <= 2) ? 2 : 1)
   if (a.S == 1) return;
 
   // last CTA of this column tile sums the S partials in split order
-  __threadfence();
   __syncthreads();
-  if (tid == 0) {
-    const int prev = atomicAdd(&a.counters[tile], 1);
-    s_last = (prev == a.S - 1);
-  }
+  if (tid == 0) s_last = (arrive_acq_rel(&a.counters[tile]) == a.S - 1);
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   // thread = (column group of 4, split group g of 4); split group g sums the
   // splits s = g, g + 4, g + 8, ... in order; the four group sums are then
   // added in group order.
@@ -329,13 +339,9 @@ __global__ void __launch_bounds__(gemv_threads(BMAX), (BMAX <= 2) ? 2 : 1)
 template <typename TW, typename TX, int NT, int BMAX>
 inline int launch_t(const GemvPlan& p, const GemvArgs& a, cudaStream_t stream, bool pdl) {
   auto kern = sparse_gemv_kernel<TW, TX, NT, BMAX>;
-  static size_t configured = 0;
-  if (p.smem > configured) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem) !=
-        cudaSuccess)
-      return SFX_ERR_CUDA;
-    configured = p.smem;
-  }
+  static size_t configured = 0;  // per instantiation; raised under the helper's lock
+  if (ensure_dynamic_smem(reinterpret_cast<const void*>(kern), p.smem, &configured) != SFX_OK)
+    return SFX_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)p.col_tiles, (unsigned)p.S, 1);
   cfg.blockDim = dim3(gemv_threads(BMAX), 1, 1);

@@ -56,6 +56,10 @@ struct GemvPlan {
 
 int sm_count();
 
+// Plan override for `key` (sfx_plan_key) set through sfx_set_plan_override,
+// 0 when the planner chooses.
+int plan_override(int key);
+
 // Raises the kernel's dynamic shared-memory limit to at least `bytes` (never
 // lowers it). *configured remembers the limit set so far; calls from several
 // host threads are serialised, so the remembered limit is never above the one

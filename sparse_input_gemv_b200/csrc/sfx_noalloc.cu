@@ -69,16 +69,16 @@ extern "C" int sfx_sparse_gemv_noalloc(const void* x, int xdt, int B, int K, con
   if (kWsHeader + gemv_workspace_bytes(K, N, B) > kNoAllocScratchBytes)
     return SFX_ERR_UNSUPPORTED;  // partial sums would not fit in the fixed scratch
   const GemvPlan plan = plan_gemv(K, N, B, idx != nullptr);
-  if (plan.col_tiles > kCounterSlots) return SFX_ERR_UNSUPPORTED;
 
   void* scratch = nullptr;
   const int rc = scratch_for_current_device(&scratch);
   if (rc != SFX_OK) return rc;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // The array keeps the previous call's contents: the status word and the
-  // arrival counters must start at zero, so clear them on the caller's stream.
-  if (cudaMemsetAsync(scratch, 0, kWsStatusBytes + (size_t)plan.col_tiles * 4, s) != cudaSuccess)
-    return SFX_ERR_CUDA;
+  // The array keeps the previous call's contents: the status word and every
+  // arrival counter must start at zero, whichever kernel (and so whichever
+  // tile count) the previous call or this one launches, so the whole header
+  // (16.6 KB) is cleared on the caller's stream.
+  if (cudaMemsetAsync(scratch, 0, kWsHeader, s) != cudaSuccess) return SFX_ERR_CUDA;
 
   GemvArgs a = {};
   a.x = x;

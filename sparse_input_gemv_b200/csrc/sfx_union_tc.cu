@@ -41,8 +41,6 @@
 #include "sfx_rowdot.cuh"
 
 #include <algorithm>
-#include <cstdlib>
-#include <cstring>
 
 namespace sfx {
 
@@ -449,12 +447,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) union_gemm_tc_kernel(const TcAr
     for (int b = 0; b < kTcN; ++b)
       if (b < a.B) a.partials[((long long)split * a.B + b) * N + n0 + m] = d[b];
   }
-  __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&a.counters[tile], 1) == a.S - 1);
+  if (tid == 0) s_last = (arrive_acq_rel(&a.counters[tile]) == a.S - 1);
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   const long long vs = (long long)a.B * N;
   // pairs of columns so the SwiGLU epilogue sees (gate, up) together
   for (int e = tid; e < a.B * (kTcM / 2); e += kTcThreads) {
@@ -691,12 +687,10 @@ __global__ void __launch_bounds__(kMmaThreads, 2) union_gemm_mma_kernel(const Tc
   }
   if (a.S == 1) return;
 
-  __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = (atomicAdd(&a.counters[tile], 1) == a.S - 1);
+  if (tid == 0) s_last = (arrive_acq_rel(&a.counters[tile]) == a.S - 1);
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   // the last CTA of the tile sums the S partials in split order, column pairs
   // so that the SwiGLU epilogue sees (gate, up) together
   const long long vs = (long long)a.B * N;
@@ -727,9 +721,8 @@ static constexpr long long kMaxSlice = 6144;       // tcgen05: 24 KB row list in
 static constexpr long long kMmaMaxSlice = 16384;   // mma.sync: 64 KB row list
 
 bool union_uses_mma() {
-  const char* e = std::getenv("SFX_UNION_KERNEL");  // "tc" or "mma"
-  if (e && *e) return std::strcmp(e, "mma") == 0;
-  return kUnionMmaDefault;
+  const int v = plan_override(SFX_PLAN_UNION_KERNEL);  // 1 tcgen05, 2 mma.sync
+  return v ? v == 2 : kUnionMmaDefault;
 }
 
 // Splits of K for `tiles` column tiles: one wave of resident CTAs (two per
@@ -739,8 +732,7 @@ static void plan_splits(GemvPlan& p, long long K, long long max_slice) {
   const long long slots = 2LL * sm_count();
   long long S = std::max<long long>(1, slots / p.col_tiles);
   S = std::min<long long>(S, std::max<long long>(1, K / 256));
-  if (const char* e = std::getenv("SFX_TC_S"))  // tuning sweeps only
-    if (*e) S = std::max(1, std::atoi(e));
+  if (plan_override(SFX_PLAN_UNION_S)) S = plan_override(SFX_PLAN_UNION_S);
   long long slice = rup((K + S - 1) / S, kPackThreads);  // whole 256-row pack chunks
   if (slice > max_slice) slice = max_slice;
   p.S = (int)((K + slice - 1) / slice);
@@ -766,10 +758,8 @@ GemvPlan plan_union_tc(long long K, long long N) {
   // shared by its warps and summed through shared memory).
   p.kind = 2;
   int C = 8;
-  const char* e = std::getenv("SFX_MMA_CHUNKS");  // tuning sweeps only
-  if (e && *e) {
-    C = std::atoi(e);
-    if (C != 1 && C != 2 && C != 4) C = 8;
+  if (plan_override(SFX_PLAN_MMA_CHUNKS)) {
+    C = plan_override(SFX_PLAN_MMA_CHUNKS);
   } else {
     int best_S = 1 << 30;
     for (int cand = 1; cand <= 8; cand *= 2) {

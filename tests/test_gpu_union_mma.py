@@ -30,9 +30,8 @@ def _mma_union(monkeypatch):
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     sb.load()
-    monkeypatch.setenv("SFX_UNION_KERNEL", "mma")
-    monkeypatch.setenv("SFX_UNION_MIN_B", "2")
-    yield
+    with sb.plan_overrides(union_kernel=sb.UNION_MMA, union_min_b=2):
+        yield
     ws = sb.default_workspace()
     if ws.buf is not None:
         assert ws.status() == 0, "device status word raised"
@@ -83,9 +82,9 @@ def test_union_mma_matches_oracle(B, K, N, p, wdt, xdt, out):
 ])
 def test_union_mma_every_tile_width(chunks, B, K, N, p, wdt, xdt, out, flags, monkeypatch):
     # 8 / chunks warps share each 64-column chunk and are summed in shared memory
-    monkeypatch.setenv("SFX_MMA_CHUNKS", str(chunks))
-    assert sb.sfx_gemv_plan(B, K, N, flags)["chunks"] == chunks
-    case(B, K, N, p, wdt, xdt, out, flags=flags, seed=f"mma-c{chunks}")
+    with sb.plan_overrides(mma_chunks=chunks):
+        assert sb.sfx_gemv_plan(B, K, N, flags)["chunks"] == chunks
+        case(B, K, N, p, wdt, xdt, out, flags=flags, seed=f"mma-c{chunks}")
 
 
 def test_union_mma_epilogues():

@@ -16,11 +16,10 @@ SHAPES = {  # (K, N) of the Llama-3 8B / 70B projections and the Phi-2 down proj
 
 
 @pytest.fixture(autouse=True)
-def _lib(monkeypatch):
+def _lib():
     sb.load()
-    for v in ("SFX_UNION_KERNEL", "SFX_UNION_MIN_B", "SFX_MMA_CHUNKS", "SFX_TC_S", "SFX_GEMV_NT",
-              "SFX_GEMV_S"):
-        monkeypatch.delenv(v, raising=False)
+    for k in range(6):
+        sb.sfx_set_plan_override(k, 0)
 
 
 @pytest.mark.parametrize("name", list(SHAPES))
@@ -69,7 +68,7 @@ def test_plan_one_wave_at_batch_one():
             assert p["col_tiles"] * p["S"] <= slots, (K, N, B, p)
 
 
-def test_plan_flags_and_overrides(monkeypatch):
+def test_plan_flags_and_overrides():
     K, N = SHAPES["8b_gate_up"]
     # SFX_FLAG_CUDA_CORES keeps a batch on CUDA cores; an index list is batch 1 only
     assert sb.sfx_gemv_plan(16, K, N, flags=sb.SFX_FLAG_CUDA_CORES)["kernel"] == "cuda_cores"
@@ -79,15 +78,31 @@ def test_plan_flags_and_overrides(monkeypatch):
     with pytest.raises(sb.SfxError):
         sb.sfx_gemv_plan(17, K, N)
     # the tcgen05 union kernel: 128-column tiles, from 5 tokens on
-    monkeypatch.setenv("SFX_UNION_KERNEL", "tc")
-    assert sb.sfx_gemv_plan(4, K, N)["kernel"] == "cuda_cores"
-    p = sb.sfx_gemv_plan(5, K, N)
-    assert p["kernel"] == "union_tcgen05" and p["NT"] == 128 and p["chunks"] == 0
-    monkeypatch.setenv("SFX_UNION_KERNEL", "mma")
-    monkeypatch.setenv("SFX_MMA_CHUNKS", "8")
-    assert sb.sfx_gemv_plan(16, K, N)["NT"] == 512
-    monkeypatch.setenv("SFX_UNION_MIN_B", "2")
-    assert sb.sfx_gemv_plan(2, K, N)["kernel"] == "union_mma"
+    with sb.plan_overrides(union_kernel=sb.UNION_TCGEN05):
+        assert sb.sfx_gemv_plan(4, K, N)["kernel"] == "cuda_cores"
+        p = sb.sfx_gemv_plan(5, K, N)
+        assert p["kernel"] == "union_tcgen05" and p["NT"] == 128 and p["chunks"] == 0
+    with sb.plan_overrides(union_kernel=sb.UNION_MMA, mma_chunks=8):
+        assert sb.sfx_gemv_plan(16, K, N)["NT"] == 512
+        with sb.plan_overrides(union_min_b=2):
+            assert sb.sfx_gemv_plan(2, K, N)["kernel"] == "union_mma"
+    # back to the planner once the overrides are released
+    assert sb.sfx_gemv_plan(16, K, N)["NT"] == 128
+
+
+def test_plan_overrides_reject_out_of_range_values():
+    for key, bad in ((sb.SFX_PLAN_UNION_KERNEL, 3), (sb.SFX_PLAN_UNION_MIN_B, 1),
+                     (sb.SFX_PLAN_UNION_MIN_B, 17), (sb.SFX_PLAN_GEMV_NT, 384),
+                     (sb.SFX_PLAN_GEMV_S, -1), (sb.SFX_PLAN_MMA_CHUNKS, 3), (6, 1), (-1, 0)):
+        with pytest.raises(sb.SfxError):
+            sb.sfx_set_plan_override(key, bad)
+    # the library reads no environment variable for its plans
+    import os
+    os.environ["SFX_MMA_CHUNKS"] = "8"
+    try:
+        assert sb.sfx_gemv_plan(16, *SHAPES["8b_gate_up"])["NT"] == 128
+    finally:
+        del os.environ["SFX_MMA_CHUNKS"]
 
 
 def test_workspace_covers_the_plan():
