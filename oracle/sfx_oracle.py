@@ -40,7 +40,8 @@ __all__ = [
     "corrected_gxo_score_f32", "ffn_static_mask",
     "glass_ranks", "glass_fuse", "glass_mask", "masked_gemv", "silu", "gelu_erf",
     "gelu_tanh", "ffn_swiglu", "ffn_gelu_topk_down",
-    "moe_route", "moe_expert", "moe_layer", "round_to",
+    "moe_route", "moe_expert", "moe_layer", "block_error_curve", "overall_sparsity",
+    "greedy_allocate", "round_to",
 ]
 
 
@@ -355,6 +356,72 @@ def moe_layer(x, logits, W_g, W_upT, W_d, t_e, top_k, Ws_g=None, Ws_u=None, Ws_d
             ys, _, _, _ = ffn_swiglu(x[t:t + 1], -math.inf, Ws_g, Ws_u, Ws_d, -math.inf)
             y[t] += ys[0]
     return y
+
+
+# ----------------------------------------------------------------------------
+# block-wise greedy sparsity allocation                     [TEAL] slide 10
+# ----------------------------------------------------------------------------
+
+def block_error_curve(X, W, levels):
+    """l2 activation error of one block at each sparsity level.
+
+    [TEAL] slide 10 optimises the per-block sparsities against the blocks' l2
+    activation error. Reading: a block is one input site with its weight
+    matrix W [K x N]; at level p its input is masked with the threshold t_p
+    calibrated on the same draws X [S x K] (calibrate_threshold), and the
+    error is the l2 (Frobenius) norm over the S draws of the change in the
+    block output, ||(X * m_p) W - X W||. Returns (err [P], t [P]) in fp64.
+    """
+    X = np.atleast_2d(np.asarray(X, dtype=np.float64))
+    W = np.asarray(W, dtype=np.float64)
+    dense = masked_gemv(X, np.ones_like(X, dtype=bool), W)
+    err, thr = [], []
+    for p in levels:
+        t = calibrate_threshold(X, p)
+        y = masked_gemv(X, magnitude_mask(X, t), W)
+        err.append(float(np.linalg.norm(y - dense)))
+        thr.append(t)
+    return np.array(err), np.array(thr)
+
+
+def overall_sparsity(p, weights):
+    """Model-wide sparsity of per-block sparsities p: sum_i w_i p_i / sum_i w_i.
+
+    Reading of [TEAL] slide 10's overall sparsity constraint: each block counts
+    by its weight w_i, its parameter count, since a block at sparsity p skips
+    that fraction of its weight rows (weights of 1 give the plain mean).
+    """
+    p = np.asarray(p, dtype=np.float64)
+    w = np.asarray(weights, dtype=np.float64)
+    return float((w * p).sum() / w.sum())
+
+
+def greedy_allocate(err, weights, step, target):
+    """Per-block sparsity levels by [TEAL] slide 10's greedy procedure.
+
+    err [M x P]: block i's error at sparsity level j (levels 0, step, 2 step,
+    ..., so err[:, 0] is the dense block). Steps of the slide: every block
+    starts at sparsity 0; each round measures, for every block that can still
+    go one level up, how much its error would grow; the block with the
+    smallest growth goes up one level (equal growths: the lower block index);
+    rounds repeat until the overall sparsity (overall_sparsity with `weights`)
+    reaches `target`, or no block can go further. Returns the level index of
+    each block (sparsity = level * step).
+    """
+    err = np.asarray(err, dtype=np.float64)
+    M, P = err.shape
+    lvl = np.zeros(M, dtype=np.int64)
+    while overall_sparsity(lvl * step, weights) < target - 1e-12:
+        best, best_i = math.inf, -1
+        for i in range(M):
+            if lvl[i] + 1 < P:
+                growth = err[i, lvl[i] + 1] - err[i, lvl[i]]
+                if growth < best:
+                    best, best_i = growth, i
+        if best_i < 0:
+            break
+        lvl[best_i] += 1
+    return lvl
 
 
 # ----------------------------------------------------------------------------

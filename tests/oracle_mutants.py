@@ -129,6 +129,33 @@ def _mutants(O):
         bits = (f.view(np.uint32) >> 16) << 16
         return bits.astype(np.uint32).view(np.float32).astype(np.float64)
     M["bf16_rounding_truncates"] = ("round_to", round_bf16_truncates)
+    def greedy_largest_growth(err, weights, step, target):
+        err = np.asarray(err, np.float64)
+        M_, P = err.shape
+        lvl = np.zeros(M_, np.int64)
+        while O.overall_sparsity(lvl * step, weights) < target - 1e-12:
+            g = [err[i, lvl[i] + 1] - err[i, lvl[i]] if lvl[i] + 1 < P else -math.inf
+                 for i in range(M_)]
+            i = int(np.argmax(g))
+            if g[i] == -math.inf:
+                break
+            lvl[i] += 1
+        return lvl
+    M["greedy_largest_growth"] = ("greedy_allocate", greedy_largest_growth)
+
+    M["overall_unweighted"] = ("overall_sparsity",
+                               lambda p, weights: float(np.mean(np.asarray(p, np.float64))))
+
+    def block_error_output_norm(X, W, levels):
+        X = np.atleast_2d(np.asarray(X, np.float64))
+        err, thr = [], []
+        for p in levels:
+            t = O.calibrate_threshold(X, p)
+            err.append(float(np.linalg.norm(O.masked_gemv(X, O.magnitude_mask(X, t), W))))
+            thr.append(t)
+        return np.array(err), np.array(thr)
+    M["block_error_output_norm"] = ("block_error_curve", block_error_output_norm)
+
     return M
 
 
@@ -140,7 +167,8 @@ MUTANT_NAMES = [
     "layer_drops_shared_expert", "gxo_not_rounded_to_fp32", "corrected_gxo_drops_half",
     "corrected_f32_ranks_abs_gxo", "corrected_f32_norm_is_l1", "corrected_f32_drops_half",
     "static_ffn_ignores_mask",
-    "bf16_rounding_truncates",
+    "bf16_rounding_truncates", "greedy_largest_growth", "overall_unweighted",
+    "block_error_output_norm",
 ]
 
 

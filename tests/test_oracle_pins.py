@@ -418,3 +418,75 @@ def test_round_to_bf16_and_f16():
     assert bf[2] == 1.0
     h = O.round_to(v, "f16")
     assert h[3] == 65504.0 and h[4] == 1.0   # tie -> even
+
+
+# ---------------------------------------------------------------- greedy block allocation
+
+def test_block_error_closed_form_diagonal_weights():
+    # W = diag(d): block output y = x * d, so the error at level p is the l2 norm
+    # of the dropped activations scaled by d: sqrt(sum over |x| <= t_p of (x d)^2)
+    X = _rng(20).laplace(size=(8, 24))
+    d = _rng(21).uniform(0.5, 2.0, size=24)
+    levels = [0.0, 0.25, 0.5, 0.75, 1.0]
+    err, thr = O.block_error_curve(X, np.diag(d), levels)
+    for p, e, t in zip(levels, err, thr):
+        dropped = np.abs(X) <= t
+        assert e == pytest.approx(math.sqrt(((X * d) ** 2)[dropped].sum()), rel=1e-12, abs=1e-15)
+    assert err[0] == 0.0                      # dense: no error
+    assert err[-1] == pytest.approx(np.linalg.norm(X * d), rel=1e-12)  # all dropped
+
+
+def test_block_error_uses_the_full_output_change():
+    # rectangular W: the error is ||(X m) W - X W||, i.e. the norm of the
+    # dropped part pushed through W, row by row in Python
+    X = _rng(22).laplace(size=(3, 6))
+    W = _rng(23).standard_normal((6, 4))
+    err, thr = O.block_error_curve(X, W, [0.5])
+    tot = 0.0
+    for s in range(3):
+        for n in range(4):
+            v = sum(X[s, i] * W[i, n] for i in range(6) if abs(X[s, i]) <= thr[0])
+            tot += v * v
+    assert err[0] == pytest.approx(math.sqrt(tot), rel=1e-12)
+
+
+def _convex_curves(rng, M, P):
+    inc = np.sort(rng.uniform(0.1, 3.0, size=(M, P - 1)), axis=1)  # growing increments
+    return np.concatenate([np.zeros((M, 1)), np.cumsum(inc, axis=1)], axis=1)
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_greedy_is_optimal_on_convex_curves_brute_force(seed):
+    # With equal weights and error curves whose increments grow, raising the
+    # block with the smallest growth one level at a time gives the least total
+    # error among all allocations with the same number of levels (the classic
+    # marginal-allocation result); brute force over every allocation of 3 blocks.
+    M, P, step = 3, 5, 0.25
+    err = _convex_curves(_rng(100 + seed), M, P)
+    for T in range(0, M * (P - 1) + 1):
+        lvl = O.greedy_allocate(err, np.ones(M), step, T * step / M)
+        assert lvl.sum() == T
+        best = min(sum(err[i, a[i]] for i in range(M))
+                   for a in itertools.product(range(P), repeat=M) if sum(a) == T)
+        assert sum(err[i, lvl[i]] for i in range(M)) == pytest.approx(best, rel=1e-12)
+
+
+def test_greedy_weighted_overall_sparsity_and_stop():
+    # weights 1 and 3: one level (0.5) of block 1 already gives overall 0.375,
+    # which is below 0.4; the next level of the cheaper block reaches it
+    err = np.array([[0.0, 1.0, 5.0], [0.0, 0.5, 4.0]])
+    lvl = O.greedy_allocate(err, [1.0, 3.0], 0.5, 0.4)
+    assert lvl.tolist() == [1, 1]
+    assert O.overall_sparsity(lvl * 0.5, [1.0, 3.0]) == pytest.approx(0.5)
+    assert O.overall_sparsity([0.5, 0.0], [1.0, 3.0]) == pytest.approx(0.125)
+    # target 0: every block stays dense; unreachable target: every block ends at its top level
+    assert O.greedy_allocate(err, [1.0, 3.0], 0.5, 0.0).tolist() == [0, 0]
+    assert O.greedy_allocate(err, [1.0, 3.0], 0.5, 2.0).tolist() == [2, 2]
+
+
+def test_greedy_free_block_first_and_ties_to_lower_index():
+    # a block that loses nothing is sparsified first; equal growths go to the
+    # lower block index
+    err = np.array([[0.0, 1.0, 2.0], [0.0, 0.0, 0.0], [0.0, 1.0, 2.0]])
+    assert O.greedy_allocate(err, np.ones(3), 0.5, 1 / 3).tolist() == [0, 2, 0]
+    assert O.greedy_allocate(err, np.ones(3), 0.5, 0.5).tolist() == [1, 2, 0]
