@@ -1,23 +1,26 @@
 #!/usr/bin/env python
 """Benchmark of the activation-sparse decode path on B200.
 
-Workload: Llama-3-8B-shaped decoder-layer projections at batch 1, bf16 weights
-~ N(0, 0.02^2): q/k/v (4096 -> 4096/1024/1024, one fused [4096 x 6144] matrix),
-o (4096 -> 4096), SwiGLU FFN d=4096, ffn=14336 (gate|up interleaved
-[4096 x 28672], down [14336 x 4096]). Inputs are Laplace(0, 1); TEAL magnitude
-thresholds are calibrated per block input (qkv-in, o-in, gate/up-in, down-in)
-on 64 seeded draws for the target sparsity (down-in on the dense FFN's h).
+Headline workload: a Llama-3-70B-shaped SwiGLU FFN layer, d = 8192,
+ffn = 28672, bf16 weights ~ N(0, 0.02^2) (1.41 GB dense per layer), at batch 1
+with TEAL magnitude thresholds on its two block inputs (gate/up-in and
+down-in) calibrated for p = 0.5 on 64 seeded Laplace(0, 1) draws (down-in on
+the dense FFN's h of those draws).
 
-One step = one batch-1 token through a stack of 32 such layers with distinct
-weights (13.9 GB of bf16 weights, far larger than the 126 MB L2, so every
-weight byte comes from HBM). Each layer runs three library calls: sparse GEMV
-(qkv), sparse GEMV (o), sparse SwiGLU FFN (two kernels); the 32-layer step is
+One step = one token through a stack of 8 such layers with distinct weights
+(11.3 GB, far larger than the 126 MB L2, so every weight byte comes from HBM);
+each layer is one sfx_sparse_ffn_swiglu call (two kernels), and the step is
 captured once in a CUDA graph and replayed.
 
 Metric: effective HBM GB/s = algorithmic bytes (active weight rows x row bytes
-+ activations in + outputs) / time, whole job (summed over ranks); also
-us/layer. With --gpus N each rank runs an independent replica (no collective:
-the path does not shard across GPUs here).
++ activations in and out, h written and read) / time, whole job (summed over
+ranks), and µs per layer. The line also carries the metric's sweep (batch 1,
+4, 8, 16 x sparsity 0-0.9 on the same layer, iid and correlated tokens), the
+per-kernel roofline, the cuBLAS dense reference, the fp64 oracle timed on the
+host cores, the mask flips of the GPU path against the oracle, and the other
+workloads of the path (Llama-3-8B decoder layer, single GEMV, Phi-2 top-k
+FFN, 128-expert MoE) as secondary keys. With --gpus N each rank runs an
+independent replica (no collective: the path does not shard across GPUs).
 """
 from __future__ import annotations
 
@@ -37,12 +40,16 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-OTHER_WORKLOADS = ("gemv", "phi2", "moe", "ffn70b")
+OTHER_WORKLOADS = ("llama8b", "gemv", "phi2", "moe")
 METRIC = "sparse FFN µs/layer and effective HBM GB/s vs sparsity at batch 1–16"
+D70, F70 = 8192, 28672
+WORKLOAD = ("Llama-3-70B-shaped SwiGLU FFN layer d=8192 ffn=28672, bf16 weights ~N(0,0.02^2) "
+            "(1.41 GB dense), batch 1, Laplace(0,1) inputs, TEAL thresholds on the gate/up and "
+            "down inputs")
 D, FFN, NQKV = 4096, 14336, 6144
-WORKLOAD = ("Llama-3-8B-shaped decoder layer at batch 1: q/k/v/o 4096->4096/1024/1024/4096, "
-            "SwiGLU FFN d=4096 ffn=14336, bf16 weights ~N(0,0.02^2), Laplace inputs, per-block "
-            "TEAL thresholds on all four block inputs")
+WORKLOAD_8B = ("Llama-3-8B-shaped decoder layer at batch 1: q/k/v/o 4096->4096/1024/1024/4096, "
+               "SwiGLU FFN d=4096 ffn=14336, bf16 weights ~N(0,0.02^2), Laplace inputs, per-block "
+               "TEAL thresholds on all four block inputs")
 
 
 # ---------------------------------------------------------------- helpers
@@ -356,7 +363,7 @@ def bench_other_workloads(stream, dev, which=OTHER_WORKLOADS):
     """The other workloads of the path, short graph-timed runs (not the headline).
 
     `which` selects among "gemv" (single input-sparse GEMV), "phi2" (GeLU FFN with
-    GxO top-k / GLASS), "moe" (128-expert MoE) and "ffn70b" (batch sweep).
+    GxO top-k / GLASS) and "moe" (128-expert MoE).
     """
     from sparse_input_gemv_b200 import binding as sb
     from sparse_input_gemv_b200 import synth
@@ -509,181 +516,296 @@ def bench_other_workloads(stream, dev, which=OTHER_WORKLOADS):
                                                       "weights replayed round-robin (HBM-resident)"}
         del layers
 
-    if "ffn70b" in which:
-        # Llama-3-70B-shaped SwiGLU FFN d=8192, ffn=28672 bf16, batch 1/4/8/16,
-        # per-batch union of magnitude masks, sparsity 0..0.9
-        d, f = 8192, 28672
-        n = 2
-        Wgu = []
-        Wdn = []
-        for c in range(n):
-            Wg = synth.normal((d, f), synth.seed_of("l70", "Wg", c), 0.02, "bf16", dev)
-            Wu = synth.normal((d, f), synth.seed_of("l70", "Wu", c), 0.02, "bf16", dev)
-            Wgu.append(sb.sfx_pack_gate_up(Wg, Wu))
-            del Wg, Wu
-            Wdn.append(synth.normal((f, d), synth.seed_of("l70", "Wd", c), 0.02, "bf16", dev))
-        calib = synth.calib_draws("l70", "x", 64, d, "bf16").to(dev)
-        hc = torch.cat([sb.sfx_sparse_ffn_swiglu(calib[i:i + 16], Wgu[0], Wdn[0], want_h=True, ws=ws)["h"]
-                        for i in range(0, 64, 16)]).contiguous()
-        sweep = []
-        for B in (1, 4, 8, 16):
-            xb = synth.eval_draw("l70", "x", B, d, "bf16").to(dev)
-            yb = torch.empty((B, d), dtype=torch.bfloat16, device=dev)
-            hb = torch.empty((B, f), dtype=torch.float32, device=dev)
-            for p in [i / 10 for i in range(10)]:
-                t_in = sb.sfx_calibrate_thresholds(calib, [p], ws=ws)[0]
-                t_h = sb.sfx_calibrate_thresholds(hc, [p], ws=ws)[0]
-                r = sb.sfx_sparse_ffn_swiglu(xb, Wgu[0], Wdn[0], t_in, t_h, h=hb, y=yb,
-                                             want_bitmaps=True, ws=ws)
-                ux = int(np.unpackbits(r["bitmap_x"].view(torch.uint8).cpu().numpy().reshape(B, -1),
-                                       axis=1).any(0).sum())
-                uh = int(np.unpackbits(r["bitmap_h"].view(torch.uint8).cpu().numpy().reshape(B, -1),
-                                       axis=1).any(0).sum())
-                nbytes = ux * 2 * f * 2 + uh * d * 2 + B * (d * 2 * 2 + f * 4 * 2)
-                us = graph_us([lambda c=c: sb.sfx_sparse_ffn_swiglu(xb, Wgu[c], Wdn[c], t_in, t_h, h=hb,
-                                                                    y=yb, ws=ws) for c in range(n)],
-                              stream, reps=3)
-                sweep.append({"batch": B, "sparsity": p, "us": us, "gbs": nbytes / (us * 1e-6) / 1e9,
-                              "union_frac_in": ux / d, "union_frac_h": uh / f})
-        # the same layer on correlated tokens (shared per-neuron scales; masks of
-        # different tokens overlap with pairwise Jaccard ~0.56 at p = 0.5)
-        ccal = synth.correlated_draws("l70c", "x", 64, d, "bf16", draw=0).to(dev)
-        chc = torch.cat([sb.sfx_sparse_ffn_swiglu(ccal[i:i + 16], Wgu[0], Wdn[0], want_h=True,
-                                                  ws=ws)["h"] for i in range(0, 64, 16)]).contiguous()
-        csweep = []
-        for B in (4, 8, 16):
-            xb = synth.correlated_draws("l70c", "x", B, d, "bf16").to(dev)
-            yb = torch.empty((B, d), dtype=torch.bfloat16, device=dev)
-            hb = torch.empty((B, f), dtype=torch.float32, device=dev)
-            for p in (0.5, 0.7, 0.9):
-                t_in = sb.sfx_calibrate_thresholds(ccal, [p], ws=ws)[0]
-                t_h = sb.sfx_calibrate_thresholds(chc, [p], ws=ws)[0]
-                r = sb.sfx_sparse_ffn_swiglu(xb, Wgu[0], Wdn[0], t_in, t_h, h=hb, y=yb,
-                                             want_bitmaps=True, ws=ws)
-                ux = int(np.unpackbits(r["bitmap_x"].view(torch.uint8).cpu().numpy().reshape(B, -1),
-                                       axis=1).any(0).sum())
-                uh = int(np.unpackbits(r["bitmap_h"].view(torch.uint8).cpu().numpy().reshape(B, -1),
-                                       axis=1).any(0).sum())
-                nbytes = ux * 2 * f * 2 + uh * d * 2 + B * (d * 2 * 2 + f * 4 * 2)
-                us = graph_us([lambda c=c: sb.sfx_sparse_ffn_swiglu(xb, Wgu[c], Wdn[c], t_in, t_h, h=hb,
-                                                                    y=yb, ws=ws) for c in range(n)],
-                              stream, reps=3)
-                csweep.append({"batch": B, "sparsity": p, "us": us, "gbs": nbytes / (us * 1e-6) / 1e9,
-                               "union_frac_in": ux / d, "union_frac_h": uh / f})
-        out["llama3_70b_ffn_bf16_correlated_tokens"] = {
-            "sweep": csweep,
-            "note": "x_bi = exp(1.5 n_i) z_bi (shared per-neuron scales); pairwise mask Jaccard "
-                    "~0.56 at p = 0.5"}
-        # dense library reference: torch.matmul (cuBLAS) for both projections and
-        # torch ops for SiLU(g) * u, every row read
-        lib = []
-        for B in (1, 4, 8, 16):
-            xb = synth.eval_draw("l70", "x", B, d, "bf16").to(dev)
-            gu = torch.empty((B, 2 * f), dtype=torch.bfloat16, device=dev)
-            yb = torch.empty((B, d), dtype=torch.bfloat16, device=dev)
-
-            def dense(c, xb=xb, gu=gu, yb=yb):
-                torch.mm(xb, Wgu[c], out=gu)
-                torch.mm(torch.nn.functional.silu(gu[:, 0::2]) * gu[:, 1::2], Wdn[c], out=yb)
-
-            us = graph_us([lambda c=c: dense(c) for c in range(n)], stream, reps=3)
-            lib.append({"batch": B, "us": us, "gbs": 3 * d * f * 2 / (us * 1e-6) / 1e9})
-        out["llama3_70b_ffn_bf16"] = {"sweep": sweep, "dense_bytes": 3 * d * f * 2,
-                                      "dense_library": lib,
-                                      "note": "2 weight copies (2.8 GB) alternate between calls; "
-                                              "dense_library = torch.matmul (cuBLAS) reference"}
     return out
 
 
-# ---------------------------------------------------------------- CPU oracle leg
+# ---------------------------------------------------------------- the headline: Llama-3-70B FFN
 
-def oracle_layer_pass(W, x, t):
-    """One layer (qkv, o, SwiGLU FFN) of the fp64 oracle as it stands."""
+def ffn_bytes(ux: int, uh: int, B: int, d: int = D70, f: int = F70) -> int:
+    """Algorithmic bytes of one SwiGLU FFN call with `ux` gate/up rows and `uh`
+    down rows read (the batch union): bf16 rows of 4 f and 2 d bytes, x in,
+    y out (bf16), h written and read once (fp32)."""
+    return ux * 4 * f + uh * 2 * d + B * (2 * d * 2 + 2 * f * 4)
+
+
+def union_counts(bitmap: torch.Tensor, B: int, n: int) -> int:
+    """Rows of the batch union in a [B x words] int32 bitmap of n columns."""
+    bits = np.unpackbits(bitmap.view(torch.uint8).cpu().numpy().reshape(B, -1), axis=1,
+                         bitorder="little")[:, :n]
+    return int(bits.any(0).sum())
+
+
+class Ffn70Stack:
+    """L Llama-3-70B-shaped SwiGLU FFN layers with distinct bf16 weights."""
+
+    def __init__(self, layers: int, dev):
+        from sparse_input_gemv_b200 import binding as sb
+        from sparse_input_gemv_b200 import synth
+        self.sb, self.synth, self.L, self.dev = sb, synth, layers, dev
+        self.Wgu, self.Wd = [], []
+        for l in range(layers):
+            Wg = synth.normal((D70, F70), synth.seed_of("l70", "Wg", l), 0.02, "bf16", dev)
+            Wu = synth.normal((D70, F70), synth.seed_of("l70", "Wu", l), 0.02, "bf16", dev)
+            self.Wgu.append(sb.sfx_pack_gate_up(Wg, Wu))
+            del Wg, Wu
+            self.Wd.append(synth.normal((F70, D70), synth.seed_of("l70", "Wd", l), 0.02, "bf16", dev))
+        torch.cuda.synchronize()
+        self.ws = sb.Workspace(dev)
+        self.ws.reserve(max(sb.sfx_workspace_bytes(sb.SFX_OP_FFN_SWIGLU, 16, D70, F70),
+                            sb.sfx_workspace_bytes(sb.SFX_OP_SPARSE_GEMV, 16, D70, 2 * F70, sb.SFX_BF16),
+                            sb.sfx_workspace_bytes(sb.SFX_OP_SPARSE_GEMV, 16, F70, D70, sb.SFX_F32),
+                            sb.sfx_workspace_bytes(sb.SFX_OP_CALIBRATE, 64, F70, 8, sb.SFX_F32)))
+        self.calib = {}
+        self.hcal = {}
+        for kind in ("iid", "corr"):
+            self.calib[kind] = self.draws(kind, 64, draw=0)
+            hs = [sb.sfx_sparse_ffn_swiglu(self.calib[kind][i:i + 16], self.Wgu[0], self.Wd[0],
+                                           want_h=True, ws=self.ws)["h"] for i in range(0, 64, 16)]
+            self.hcal[kind] = torch.cat(hs).contiguous()
+
+    def draws(self, kind, B, draw=64):
+        s = self.synth
+        if kind == "iid":
+            return s.eval_draw("l70", "x", B, D70, "bf16", draw=draw).to(self.dev)
+        return s.correlated_draws("l70c", "x", B, D70, "bf16", draw=draw).to(self.dev)
+
+    def thresholds(self, p, kind="iid"):
+        sb = self.sb
+        return (sb.sfx_calibrate_thresholds(self.calib[kind], [p], ws=self.ws)[0],
+                sb.sfx_calibrate_thresholds(self.hcal[kind], [p], ws=self.ws)[0])
+
+    def call(self, l, x, t_in, t_h, y, h=None):
+        return self.sb.sfx_sparse_ffn_swiglu(x, self.Wgu[l], self.Wd[l], t_in, t_h, y=y, h=h,
+                                             ws=self.ws)
+
+    def active_bytes(self, l, x, t_in, t_h):
+        """(bytes, union rows in, union rows h) of one call, from the fused bitmaps."""
+        B = x.shape[0]
+        r = self.sb.sfx_sparse_ffn_swiglu(x, self.Wgu[l], self.Wd[l], t_in, t_h,
+                                          want_bitmaps=True, ws=self.ws)
+        ux = union_counts(r["bitmap_x"], B, D70)
+        uh = union_counts(r["bitmap_h"], B, F70)
+        return ffn_bytes(ux, uh, B), ux, uh
+
+
+def sweep_70b(stack, stream, batches=(1, 4, 8, 16), ps=None, kind="iid", reps=3):
+    """µs per FFN call over batch x sparsity, the layers replayed round-robin."""
+    ps = ps if ps is not None else [i / 10 for i in range(10)]
+    rows = []
+    for B in batches:
+        xs = [stack.draws(kind, B, draw=64 + 16 * l) for l in range(stack.L)]
+        y = torch.empty((B, D70), dtype=torch.bfloat16, device=stack.dev)
+        for p in ps:
+            t_in, t_h = stack.thresholds(p, kind)
+            nb, ux, uh = stack.active_bytes(0, xs[0], t_in, t_h)
+            us = graph_us([lambda l=l: stack.call(l, xs[l], t_in, t_h, y) for l in range(stack.L)],
+                          stream, reps=reps)
+            rows.append({"batch": B, "sparsity": p, "us": round(us, 2), "bytes": nb,
+                         "gbs": round(nb / (us * 1e-6) / 1e9, 1),
+                         "union_in": round(ux / D70, 4), "union_h": round(uh / F70, 4)})
+    return rows
+
+
+def dense_library_70b(stack, stream, batches=(1, 4, 8, 16), reps=3):
+    """torch.matmul (cuBLAS) for both projections and torch SiLU * mul, every row
+    read: the dense library yardstick, not on the measured path."""
+    out = []
+    for B in batches:
+        x = stack.draws("iid", B)
+        gu = torch.empty((B, 2 * F70), dtype=torch.bfloat16, device=stack.dev)
+        y = torch.empty((B, D70), dtype=torch.bfloat16, device=stack.dev)
+
+        def dense(l):
+            torch.mm(x, stack.Wgu[l], out=gu)
+            torch.mm(torch.nn.functional.silu(gu[:, 0::2]) * gu[:, 1::2], stack.Wd[l], out=y)
+
+        us = graph_us([lambda l=l: dense(l) for l in range(stack.L)], stream, reps=reps)
+        out.append({"batch": B, "us": round(us, 2),
+                    "gbs": round(3 * D70 * F70 * 2 / (us * 1e-6) / 1e9, 1)})
+    return out
+
+
+def stage_kernels_70b(stack, stream, t_in, t_h, reps=10):
+    """Each of the FFN's two kernels alone at batch 1, in graphs of L launches:
+    gate|up with the SiLU(g) * u epilogue (writes h), and down on that h."""
+    sb = stack.sb
+    xs = [stack.draws("iid", 1, draw=64 + 16 * l) for l in range(stack.L)]
+    hs = [torch.empty((1, F70), dtype=torch.float32, device=stack.dev) for _ in range(stack.L)]
+    y = torch.empty((1, D70), dtype=torch.bfloat16, device=stack.dev)
+    fns = {
+        "ffn_gate_up": lambda l: sb.sfx_sparse_gemv(xs[l], stack.Wgu[l], t=t_in,
+                                                    flags=sb.SFX_FLAG_SWIGLU, y=hs[l], ws=stack.ws),
+        "ffn_down": lambda l: sb.sfx_sparse_gemv(hs[l], stack.Wd[l], t=t_h, y=y, ws=stack.ws),
+    }
+    for l in range(stack.L):
+        fns["ffn_gate_up"](l)
+    torch.cuda.synchronize()
+    act_x = [int((xs[l].float().abs() > t_in).sum()) for l in range(stack.L)]
+    act_h = [int((hs[l].abs() > t_h).sum()) for l in range(stack.L)]
+    nbytes = {"ffn_gate_up": sum(a * 4 * F70 + D70 * 2 + F70 * 4 for a in act_x) / stack.L,
+              "ffn_down": sum(a * 2 * D70 + F70 * 4 + D70 * 2 for a in act_h) / stack.L}
+    out = {}
+    for name, fn in fns.items():
+        us = graph_us([lambda l=l: fn(l) for l in range(stack.L)], stream, reps=reps)
+        out[name] = {"us": us, "bytes": nbytes[name], "gbs": nbytes[name] / (us * 1e-6) / 1e9,
+                     "launches_timed": reps * stack.L}
+    return out
+
+
+def oracle_chunks_70b(stack, l, x, t_in, t_h, chunk=2048):
+    """The oracle's FFN on layer l, one block of intermediate neurons at a time.
+
+    h_j depends only on neuron j's gate/up columns and y sums the neurons'
+    down rows, so the oracle's definition (O.ffn_swiglu) runs on blocks of
+    neurons and the block outputs add up to y. Returns (y, h, m_x, m_h) in fp64.
+    """
     import oracle as O
-    O.masked_gemv(x["qkv-in"], O.magnitude_mask(x["qkv-in"], t["qkv-in"]), W["Wqkv"])
-    O.masked_gemv(x["o-in"], O.magnitude_mask(x["o-in"], t["o-in"]), W["Wo"])
-    O.ffn_swiglu(x["ffn-in"], t["ffn-in"], W["Wg"], W["Wu"], W["Wd"], t["down-in"])
+    x64 = x.to("cpu", torch.float64).numpy()
+    y = np.zeros((x64.shape[0], D70))
+    hs, mhs, m_x = [], [], None
+    Wgu = stack.Wgu[l]
+    for j0 in range(0, F70, chunk):
+        j1 = min(F70, j0 + chunk)
+        Wg = Wgu[:, 2 * j0:2 * j1:2].to("cpu", torch.float64).numpy()
+        Wu = Wgu[:, 2 * j0 + 1:2 * j1:2].to("cpu", torch.float64).numpy()
+        Wd = stack.Wd[l][j0:j1].to("cpu", torch.float64).numpy()
+        yc, hc, m_x, mhc = O.ffn_swiglu(x64, t_in, Wg, Wu, Wd, t_h)
+        y += yc
+        hs.append(hc)
+        mhs.append(mhc)
+    return y, np.concatenate(hs, 1), m_x, np.concatenate(mhs, 1)
 
 
-def oracle_cores():
+def flips_vs_oracle(stack, t_in, t_h):
+    """Mask agreement of the GPU path with the oracle on layer 0 at batch 1.
+
+    The oracle takes the GPU's thresholds; the x mask must match bit for bit,
+    the h mask may differ where the fp32 and fp64 h straddle t_h (counted).
+    """
+    import oracle as O
+    sb = stack.sb
+    x = stack.draws("iid", 1)
+    r = sb.sfx_sparse_ffn_swiglu(x, stack.Wgu[0], stack.Wd[0], t_in, t_h, want_bitmaps=True,
+                                 want_h=True, ws=stack.ws)
+    y, h, m_x, m_h = oracle_chunks_70b(stack, 0, x, t_in, t_h)
+    bx = np.unpackbits(r["bitmap_x"].view(torch.uint8).cpu().numpy(), bitorder="little")[:D70]
+    bh = np.unpackbits(r["bitmap_h"].view(torch.uint8).cpu().numpy(), bitorder="little")[:F70]
+    yg = r["y"].to("cpu", torch.float64).numpy()
+    want = O.round_to(y, "bf16")
+    return {"x_mask_flips": int(np.count_nonzero(bx.astype(bool) != m_x[0])),
+            "h_mask_flips": int(np.count_nonzero(bh.astype(bool) != m_h[0])),
+            "h_active": int(m_h.sum()), "x_active": int(m_x.sum()),
+            "y_rel_l2_vs_oracle": float(np.linalg.norm(yg - want) / np.linalg.norm(want)),
+            "note": "layer 0, batch 1; the oracle (fp64, blocks of 2048 neurons) takes the GPU's "
+                    "thresholds, so flips count only where fp32 and fp64 h straddle t_h"}
+
+
+# ---------------------------------------------------------------- CPU oracle legs
+
+def oracle_sample_70b(stack, frac):
+    """Layer 0 of the headline FFN restricted to its first `frac` of the
+    intermediate neurons: fp64 host copies (W_g, W_u [d x n], W_d [n x d])."""
+    n = max(64, int(F70 * frac) // 64 * 64)
+    Wgu = stack.Wgu[0]
+    return {"Wg": Wgu[:, 0:2 * n:2].to("cpu", torch.float64).numpy(),
+            "Wu": Wgu[:, 1:2 * n:2].to("cpu", torch.float64).numpy(),
+            "Wd": stack.Wd[0][:n].to("cpu", torch.float64).numpy(), "n": n}
+
+
+def oracle_pass(W, x64, t_in, t_h):
+    import oracle as O
+    return O.ffn_swiglu(x64, t_in, W["Wg"], W["Wu"], W["Wd"], t_h)
+
+
+def oracle_pass_bytes(W, x64, t_in, t_h):
+    """Algorithmic bytes of one sampled pass, counted as the GPU arm counts them."""
+    _, _, m_x, m_h = oracle_pass(W, x64, t_in, t_h)
+    n = W["n"]
+    return int(m_x.sum()) * 4 * n + int(m_h.sum()) * 2 * D70 + 2 * D70 * 2 + 2 * n * 4
+
+
+def time_oracle(W, x64, t_in, t_h, seconds, threads):
+    """Passes of the sampled oracle FFN in about `seconds`, on `threads` BLAS threads."""
+    from threadpoolctl import threadpool_limits
+    with threadpool_limits(limits=threads):
+        reps, t0 = 0, time.perf_counter()
+        while reps == 0 or time.perf_counter() - t0 < seconds:
+            oracle_pass(W, x64, t_in, t_h)
+            reps += 1
+        el = time.perf_counter() - t0
+    return reps, el
+
+
+def host_cores():
     try:
-        from threadpoolctl import threadpool_info
-        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        return len(os.sched_getaffinity(0))
     except Exception:
         return os.cpu_count() or 1
 
 
-def eval_inputs_fp64():
-    from sparse_input_gemv_b200 import synth
-    return {s: synth.eval_draw("llama3-8b", s, 1, D, "bf16").double().numpy()
-            for s in ("qkv-in", "o-in", "ffn-in")}
-
-
-def layer_bytes_fp64(W, x, t, frac=1.0):
-    """Algorithmic bytes of one layer (bf16 weights), same accounting as the GPU arm."""
-    import oracle as O
-    nq, no_, nf = W["Wqkv"].shape[1], W["Wo"].shape[1], W["Wg"].shape[1]
-    _, h, mx, mh = O.ffn_swiglu(x["ffn-in"], t["ffn-in"], W["Wg"], W["Wu"], W["Wd"], t["down-in"])
-    aq = int((np.abs(x["qkv-in"]) > t["qkv-in"]).sum())
-    ao = int((np.abs(x["o-in"]) > t["o-in"]).sum())
-    return (aq * nq * 2 + D * 2 + nq * 2 + ao * no_ * 2 + D * 2 + no_ * 2
-            + int(mx.sum()) * 2 * nf * 2 + D * 2 + nf * 4 + int(mh.sum()) * D * 2 + nf * 4 + D * 2)
-
-
-def oracle_layer0():
-    """fp64 host copies of layer 0's weights, drawn exactly as the GPU stack draws them."""
-    from sparse_input_gemv_b200 import synth
-    dev = torch.device("cuda")
-    key = ("llama3-8b", 0)
-    out = {}
-    for name, shape in (("Wqkv", (D, NQKV)), ("Wo", (D, D)), ("Wg", (D, FFN)), ("Wu", (D, FFN)),
-                        ("Wd", (FFN, D))):
-        out[name] = synth.normal(shape, synth.seed_of(*key, name), 0.02, "bf16",
-                                 dev).to("cpu", torch.float64).numpy()
-    return out
+def cpu_baseline_70b(stack, t_in, t_h, seconds):
+    """The fp64 oracle as it stands on a bounded sample of the headline layer,
+    on one host thread and on one thread per core (BLAS threads)."""
+    W = oracle_sample_70b(stack, 1 / 16)
+    x64 = stack.draws("iid", 1).to("cpu", torch.float64).numpy()
+    nbytes = oracle_pass_bytes(W, x64, t_in, t_h)
+    cores = host_cores()
+    r1, e1 = time_oracle(W, x64, t_in, t_h, seconds / 2, 1)
+    rn, en = time_oracle(W, x64, t_in, t_h, seconds / 2, cores)
+    return {"value": nbytes * rn / en / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "single_thread_gbs": nbytes * r1 / e1 / 1e9,
+            "us_per_layer_all_cores": en / rn * 1e6 * (F70 / W["n"]),
+            "us_per_layer_single_thread": e1 / r1 * 1e6 * (F70 / W["n"]),
+            "sample": f"layer 0 of the headline FFN on its first {W['n']} of {F70} intermediate "
+                      f"neurons (1/16), batch 1: {r1} passes on 1 thread in {e1:.1f} s, {rn} "
+                      f"passes on {cores} threads in {en:.1f} s; value = the all-core run"}
 
 
 def reference_arm(args):
-    """The oracle, as it stands, timed on the host cores on this workload.
+    """The oracle, as it stands, timed on the host cores on the headline workload.
 
-    Thresholds come from the oracle's own calibration (down-in on its dense
-    FFN h over the 64 calibration draws). One step is one layer pass; if the
-    requested steps would take more than about 150 s, every weight matrix is
-    cut to its first columns (the same fraction for all) so the run stays
-    within a few minutes, and the bytes are counted on that sample.
+    Each step is one pass of the oracle's SwiGLU FFN (fp64, all host cores
+    through BLAS) over a sample of layer 0: its first intermediate neurons,
+    as many as keep the whole run within about two minutes. Thresholds are the
+    oracle's own (calibrated on the same 64 draws; down-in on its h of them).
     """
     import oracle as O
     from sparse_input_gemv_b200 import synth
     p = args.sparsity
-    W = oracle_layer0()
-    t = {s: O.calibrate_threshold(synth.calib_draws("llama3-8b", s, 64, D, "bf16")
-                                  .double().numpy(), p) for s in ("qkv-in", "o-in", "ffn-in")}
-    cf = synth.calib_draws("llama3-8b", "ffn-in", 64, D, "bf16").double().numpy()
-    _, hc, _, _ = O.ffn_swiglu(cf, -math.inf, W["Wg"], W["Wu"], W["Wd"], -math.inf)
-    t["down-in"] = O.calibrate_threshold(hc, p)
-    x = eval_inputs_fp64()
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+
+    class One:
+        pass
+
+    st = One()
+    Wg = synth.normal((D70, F70), synth.seed_of("l70", "Wg", 0), 0.02, "bf16", dev)
+    Wu = synth.normal((D70, F70), synth.seed_of("l70", "Wu", 0), 0.02, "bf16", dev)
+    st.Wgu = [torch.stack([Wg, Wu], 2).reshape(D70, 2 * F70)]
+    del Wg, Wu
+    st.Wd = [synth.normal((F70, D70), synth.seed_of("l70", "Wd", 0), 0.02, "bf16", dev)]
+    calib = synth.calib_draws("l70", "x", 64, D70, "bf16", draw=0).double().numpy()
+    x64 = synth.eval_draw("l70", "x", 1, D70, "bf16").double().numpy()
+    t_in = O.calibrate_threshold(calib, p)
+    W = oracle_sample_70b(st, 1 / 64)
+    _, hc, _, _ = O.ffn_swiglu(calib, -math.inf, W["Wg"], W["Wu"], W["Wd"], -math.inf)
+    t_h = O.calibrate_threshold(hc, p)
     t0 = time.perf_counter()
-    oracle_layer_pass(W, x, t)
-    t_full = time.perf_counter() - t0
-    frac = min(1.0, 150.0 / max(t_full * (args.steps + args.warmup), 1e-9))
-    if frac < 1.0:
-        cut = lambda n: max(8, int(n * frac) // 8 * 8)
-        W = {"Wqkv": np.ascontiguousarray(W["Wqkv"][:, :cut(NQKV)]),
-             "Wo": np.ascontiguousarray(W["Wo"][:, :cut(D)]),
-             "Wg": np.ascontiguousarray(W["Wg"][:, :cut(FFN)]),
-             "Wu": np.ascontiguousarray(W["Wu"][:, :cut(FFN)]),
-             "Wd": np.ascontiguousarray(W["Wd"][:cut(FFN), :])}
+    oracle_pass(W, x64, t_in, t_h)
+    t_one = time.perf_counter() - t0
+    frac = min(0.25, (1 / 64) * 120.0 / max(t_one * (args.steps + args.warmup), 1e-9))
+    if frac > 1 / 64:
+        W = oracle_sample_70b(st, frac)
     for _ in range(args.warmup):
-        oracle_layer_pass(W, x, t)
+        oracle_pass(W, x64, t_in, t_h)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle_layer_pass(W, x, t)
+        oracle_pass(W, x64, t_in, t_h)
     el = time.perf_counter() - t0
-    nbytes = layer_bytes_fp64(W, x, t)
+    nbytes = oracle_pass_bytes(W, x64, t_in, t_h)
     gbs = nbytes * args.steps / el / 1e9
-    cores = oracle_cores()
-    sample = ("one layer pass (qkv, o, SwiGLU FFN) of the fp64 numpy oracle per step on layer 0"
-              + (f", weights cut to the first {frac:.3f} of their columns" if frac < 1 else ""))
+    cores = host_cores()
+    sample = (f"one pass of the fp64 numpy oracle's SwiGLU FFN per step on layer 0, its first "
+              f"{W['n']} of {F70} intermediate neurons, batch 1, BLAS on the host cores")
     return {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -691,7 +813,7 @@ def reference_arm(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": WORKLOAD, "batch": 1, "sparsity": p, "layers_per_step": 1,
                    "parallelism": "host cores"},
-        "us_per_layer": el / max(args.steps, 1) * 1e6 / max(frac, 1e-9),
+        "us_per_layer": el / max(args.steps, 1) * 1e6 * (F70 / W["n"]),
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -700,6 +822,89 @@ def reference_arm(args):
 
 # ---------------------------------------------------------------- main
 
+def measure_step(step_fn, stream, steps, warmup, dist, dev, clocks_index=None, e2e_bufs=None):
+    """Capture `step_fn` in a graph and time `steps` replays (CUDA events,
+    barrier + synchronize on both sides, max over ranks). With `e2e_bufs`
+    = (device inputs, device outputs) also time the same replays with a pinned
+    host->device copy of the inputs and a device->host copy of the outputs."""
+    for _ in range(max(warmup, 1)):
+        step_fn()
+    torch.cuda.synchronize()
+    g = capture(step_fn, stream)
+    for _ in range(2):
+        g.replay()
+    res = {}
+    sampler = ClockSampler(clocks_index) if clocks_index is not None else None
+    if sampler:
+        sampler.__enter__()
+        t_soak = time.perf_counter()
+        while time.perf_counter() - t_soak < 1.0:  # clock soak before the timed region
+            g.replay()
+            torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms = time_graph(g, steps, stream)
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.__exit__()
+        res["clocks"] = sampler.summary()
+    res["ms"] = max_over_ranks(ms, dist, dev)
+    if e2e_bufs is not None:
+        xs, ys = e2e_bufs
+        hx = [x.cpu().pin_memory() for x in xs]
+        hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in ys]
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        start.record(stream)
+        for _ in range(steps):
+            for d_, h_ in zip(xs, hx):
+                d_.copy_(h_, non_blocking=True)
+            g.replay()
+            for h_, d_ in zip(hy, ys):
+                h_.copy_(d_, non_blocking=True)
+        end.record(stream)
+        end.synchronize()
+        res["e2e_ms"] = max_over_ranks(start.elapsed_time(end), dist, dev)
+        res["h2d"] = sum(x.numel() * x.element_size() for x in xs)
+        res["d2h"] = sum(y.numel() * y.element_size() for y in ys)
+    del g
+    return res
+
+
+def llama8b_layer(stream, dev, sparsity, steps, sweep_ps, layers=32):
+    """The Llama-3-8B-shaped decoder layer (qkv, o, SwiGLU FFN) at batch 1,
+    secondary workload: µs per layer at `sparsity` and over a sweep."""
+    stack = Stack(layers, dev, keep_layer0_fp64=False)
+    out = {"workload": WORKLOAD_8B, "layers": layers}
+    sweep = []
+    for p in sweep_ps:
+        stack.set_sparsity(p)
+        r = measure_step(stack.step, stream, steps, 2, None, dev)
+        us = r["ms"] * 1e3 / (steps * layers)
+        sweep.append({"sparsity": p, "us_per_layer": round(us, 2),
+                      "gbs": round(stack.step_bytes() * steps / (r["ms"] * 1e-3) / 1e9, 1)})
+    out["sweep"] = sweep
+    base = next((s["us_per_layer"] for s in sweep if s["sparsity"] == 0), None)
+    if base:
+        for s in sweep:
+            s["time_ratio_vs_p0"] = round(s["us_per_layer"] / base, 3)
+    stack.set_sparsity(sparsity)
+    kernels = {}
+    for name, fn in stack.kernel_fns().items():
+        us = graph_us([lambda l=l: fn(l) for l in range(layers)], stream, reps=5)
+        kb = sum(stack.kernel_bytes(name, l) for l in range(layers)) / layers
+        kernels[name] = {"us": round(us, 2), "gbs": round(kb / (us * 1e-6) / 1e9, 1)}
+    out["kernels_at_sparsity"] = {"sparsity": sparsity, **kernels}
+    out["dense_library_us_per_layer"] = round(dense_library_us_per_layer(stack, stream), 2)
+    del stack
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
@@ -707,14 +912,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["sfx", "reference"], default="sfx")
     ap.add_argument("--sparsity", type=float, default=0.5)
-    ap.add_argument("--layers", type=int, default=32)
-    ap.add_argument("--sweep", default="0,0.25,0.4,0.5,0.65,0.9",
-                    help="comma list of sparsities for the sweep ('' to skip)")
-    ap.add_argument("--sweep-steps", type=int, default=20)
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--layers", type=int, default=8, help="70B FFN layers in the stack")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the batch x sparsity sweep")
+    ap.add_argument("--cpu-seconds", type=float, default=16.0)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-other", action="store_true",
-                    help="skip the other workloads (single GEMV, Phi-2, MoE, Llama-3-70B FFN)")
+                    help="skip the other workloads (" + ", ".join(OTHER_WORKLOADS) + ")")
     ap.add_argument("--other", default=",".join(OTHER_WORKLOADS),
                     help="comma list of the other workloads to run: " + ", ".join(OTHER_WORKLOADS))
     args = ap.parse_args()
@@ -725,8 +928,7 @@ def main():
     dist = None
     if world > 1:
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=dev)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
     if args.impl == "reference":
         if rank == 0:
@@ -737,89 +939,30 @@ def main():
 
     from sparse_input_gemv_b200 import binding as sb
     sb.load()
-    stack = Stack(args.layers, dev, keep_layer0_fp64=(rank == 0 and not args.no_cpu))
     stream = torch.cuda.Stream(dev)
     torch.cuda.set_stream(stream)
+    stack = Ffn70Stack(args.layers, dev)
+    L = args.layers
+    t_in, t_h = stack.thresholds(args.sparsity)
+    xs = [stack.draws("iid", 1, draw=64 + 16 * l) for l in range(L)]
+    ys = [torch.empty((1, D70), dtype=torch.bfloat16, device=dev) for _ in range(L)]
+    layer_bytes = [stack.active_bytes(l, xs[l], t_in, t_h)[0] for l in range(L)]
+    bytes_step = sum(layer_bytes)
 
-    def measure(p, steps, warmup, clocks=False, e2e=False):
-        stack.set_sparsity(p)
-        for _ in range(max(warmup, 1)):
-            stack.step()
-        torch.cuda.synchronize()
-        g = capture(stack.step, stream)
-        for _ in range(2):
-            g.replay()
-        res = {"p": p, "t": dict(stack.t)}
-        sampler = ClockSampler(local_rank) if clocks else None
-        if sampler:
-            sampler.__enter__()
-            t_soak = time.perf_counter()
-            while time.perf_counter() - t_soak < 1.0:  # clock soak before the timed region
-                g.replay()
-                torch.cuda.synchronize()
-        if dist is not None:
-            dist.barrier()
-        torch.cuda.synchronize()
-        ms = time_graph(g, steps, stream)
-        torch.cuda.synchronize()
-        if sampler:
-            sampler.__exit__()
-            res["clocks"] = sampler.summary()
-        res["ms"] = max_over_ranks(ms, dist, dev)
-        res["bytes_step"] = stack.step_bytes()
-        res["graph"] = g
-        if e2e:
-            # same step through host buffers: H2D of the step's inputs, D2H of its outputs
-            xs = [stack.xq, stack.xo, stack.xf]
-            ys = [stack.yq, stack.yo, stack.yf]
-            hx = [x.cpu().pin_memory() for x in xs]
-            hy = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in ys]
-            start = torch.cuda.Event(enable_timing=True)
-            end = torch.cuda.Event(enable_timing=True)
-            if dist is not None:
-                dist.barrier()
-            torch.cuda.synchronize()
-            start.record(stream)
-            for _ in range(steps):
-                for d_, h_ in zip(xs, hx):
-                    d_.copy_(h_, non_blocking=True)
-                g.replay()
-                for h_, d_ in zip(hy, ys):
-                    h_.copy_(d_, non_blocking=True)
-            end.record(stream)
-            end.synchronize()
-            ems = start.elapsed_time(end)
-            res["e2e_ms"] = max_over_ranks(ems, dist, dev)
-            res["h2d"] = sum(x.numel() * x.element_size() for x in xs)
-            res["d2h"] = sum(y.numel() * y.element_size() for y in ys)
-        return res
+    def step():
+        for l in range(L):
+            stack.call(l, xs[l], t_in, t_h, ys[l])
 
-    # headline
-    main_res = measure(args.sparsity, args.steps, args.warmup, clocks=True, e2e=True)
-    ms = main_res["ms"]
+    # headline: K timed steps of the 8-layer stack
     K = args.steps
-    bytes_step = main_res["bytes_step"]
+    main_res = measure_step(step, stream, K, args.warmup, dist, dev, clocks_index=local_rank,
+                            e2e_bufs=(xs, ys))
+    ms = main_res["ms"]
     value = replica_gbs(bytes_step, K, world, ms)
-    us_layer = ms * 1e3 / (K * args.layers)
+    us_layer = ms * 1e3 / (K * L)
 
-    # per-kernel device times: each kernel alone, replayed over the 32 layers
-    kernels = {}
-    fns = stack.kernel_fns()
-    reps = max(3, min(20, args.steps))
-    for name, fn in fns.items():
-        for l in range(args.layers):
-            fn(l)
-        torch.cuda.synchronize()
-        g = capture(lambda: [fn(l) for l in range(args.layers)], stream)
-        g.replay()
-        kms = time_graph(g, reps, stream)
-        avg_us = kms * 1e3 / (reps * args.layers)
-        kb = sum(stack.kernel_bytes(name, l) for l in range(args.layers)) / args.layers
-        kernels[name] = {"us": avg_us, "bytes": kb, "gbs": kb / (avg_us * 1e-6) / 1e9}
-        del g
-    ffn_us = kernels["ffn_gate_up"]["us"] + kernels["ffn_down"]["us"]
-    dense_lib_us = dense_library_us_per_layer(stack, stream)
-
+    # the FFN's two kernels alone (roofline), and p = 0 for the dense reference point
+    kernels = stage_kernels_70b(stack, stream, t_in, t_h)
     peaks = {}
     try:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -831,72 +974,70 @@ def main():
     dom = max(kernels, key=lambda k: kernels[k]["us"])
     roofline = {"bound": "hbm", "kernel": dom, "achieved": kernels[dom]["gbs"], "peak": peak,
                 "unit": "GB/s", "frac": kernels[dom]["gbs"] / peak, "peak_source": peak_src,
-                "traffic": None}
+                "bytes_per_launch": kernels[dom]["bytes"], "traffic": None}
     roofline["traffic"], roofline["traffic_note"] = profiled_traffic(dom, args.sparsity)
+    ffn_roof = {"achieved": bytes_step / L / (us_layer * 1e-6) / 1e9}
+    ffn_roof["frac"] = ffn_roof["achieved"] / peak
 
-    # sweep over sparsity (shorter runs, graph replay only)
-    sweep = []
-    dense_us = None
-    if args.sweep:
-        for p in [float(v) for v in args.sweep.split(",") if v.strip() != ""]:
-            r = measure(p, args.sweep_steps, 2)
-            us = r["ms"] * 1e3 / (args.sweep_steps * args.layers)
-            sweep.append({"sparsity": p, "us_per_layer": us,
-                          "gbs": r["bytes_step"] * args.sweep_steps / (r["ms"] * 1e-3) / 1e9,
-                          "active_bytes_per_layer": r["bytes_step"] / args.layers})
-            if p == 0:
-                dense_us = us
-            del r["graph"]
-        stack.set_sparsity(args.sparsity)
+    sweep = corr = lib = None
+    if not args.no_sweep:
+        sweep = sweep_70b(stack, stream)
+        corr = sweep_70b(stack, stream, batches=(4, 8, 16), ps=(0.5, 0.7, 0.9), kind="corr")
+        lib = dense_library_70b(stack, stream)
+    scaling = None
+    if sweep:
+        b1 = {r["sparsity"]: r["us"] for r in sweep if r["batch"] == 1}
+        dense_b1 = b1.get(0.0)
+        nb1 = {r["sparsity"]: r["bytes"] for r in sweep if r["batch"] == 1}
+        if dense_b1:
+            scaling = [{"sparsity": p, "time_ratio": round(u / dense_b1, 3),
+                        "byte_ratio": round(nb1[p] / nb1[0.0], 3)} for p, u in sorted(b1.items())]
 
-    # CPU oracle baseline on rank 0 (bounded sample of about cpu_seconds)
+    flips = None
     cpu = None
-    if rank == 0 and not args.no_cpu and stack.layer0 is not None:
-        t = dict(stack.t)
-        x = eval_inputs_fp64()
-        reps_o, t0 = 0, time.perf_counter()
-        while reps_o == 0 or time.perf_counter() - t0 < args.cpu_seconds:
-            oracle_layer_pass(stack.layer0, x, t)
-            reps_o += 1
-        el = time.perf_counter() - t0
-        nbytes = layer_bytes_fp64(stack.layer0, x, t)
-        cpu = {"value": nbytes * reps_o / el / 1e9, "unit": "GB/s", "cores": oracle_cores(),
-               "kind": "oracle", "us_per_layer": el / reps_o * 1e6,
-               "sample": f"{reps_o} passes of one layer (qkv, o, SwiGLU FFN) of the fp64 numpy "
-                         f"oracle on layer 0 in {el:.1f} s"}
+    if rank == 0 and not args.no_cpu:
+        flips = flips_vs_oracle(stack, t_in, t_h)
+        cpu = cpu_baseline_70b(stack, t_in, t_h, args.cpu_seconds)
+    e2e_val = replica_gbs(bytes_step, K, world, main_res["e2e_ms"])
+    del stack
+    torch.cuda.empty_cache()
 
     other = None
     if rank == 0 and not args.no_other:
-        other = bench_other_workloads(stream, dev, tuple(w for w in args.other.split(",") if w))
+        which = tuple(w for w in args.other.split(",") if w)
+        other = {}
+        if "llama8b" in which:
+            other["llama3_8b_decoder_layer_b1"] = llama8b_layer(
+                stream, dev, args.sparsity, 20, (0.0, 0.25, 0.4, 0.5, 0.65, 0.9))
+        rest = tuple(w for w in which if w != "llama8b")
+        if rest:
+            other.update(bench_other_workloads(stream, dev, rest))
 
-    e2e_val = replica_gbs(bytes_step, K, world, main_res["e2e_ms"])
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "batch": 1, "sparsity": args.sparsity,
-                   "layers_per_step": args.layers,
-                   "l2": f"inputs larger than L2: {args.layers} distinct layers, "
-                         f"{stack.dense_step_bytes() / 1e9:.1f} GB of weights per step",
+                   "layers_per_step": L,
+                   "l2": f"inputs larger than L2: {L} distinct layers, "
+                         f"{L * 3 * D70 * F70 * 2 / 1e9:.1f} GB of weights per step",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "us_per_layer": us_layer, "us_per_layer_ffn": ffn_us,
-        "dense_us_per_layer": dense_us,
-        "speedup_vs_dense": (dense_us / us_layer) if dense_us else None,
-        "dense_library_us_per_layer": dense_lib_us,
-        "speedup_vs_dense_library": dense_lib_us / us_layer,
-        "thresholds": main_res["t"],
-        "kernels": kernels, "roofline": roofline, "sweep": sweep,
+        "us_per_layer": us_layer, "thresholds": {"gate_up_in": t_in, "down_in": t_h},
+        "active_bytes_per_layer": bytes_step / L, "dense_bytes_per_layer": 3 * D70 * F70 * 2,
+        "ffn_roofline": ffn_roof,
+        "kernels": kernels, "roofline": roofline,
+        "sweep": sweep, "scaling_b1": scaling, "sweep_correlated": corr, "dense_library": lib,
+        "mask_flips": flips,
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": main_res["h2d"],
                 "d2h_bytes_per_step": main_res["d2h"], "ms_per_step": main_res["e2e_ms"] / K,
-                "path": "CUDA graph of the public entry points + pinned host copies"},
-        "gpu_launches": 4 * args.layers * K,
+                "path": "CUDA graph of sfx_sparse_ffn_swiglu calls + pinned host copies"},
+        "gpu_launches": 2 * L * K,
         "clocks": main_res.get("clocks"),
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
     if other is not None:
         line["other_workloads"] = other
-    del main_res["graph"]
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

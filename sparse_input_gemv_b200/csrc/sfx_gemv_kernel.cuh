@@ -68,6 +68,41 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p, uint64_t pol) {
   return v;
 }
 
+// x[i .. i+3] as floats (0 past `lim`): one 8- or 16-byte load when `vec`
+// (the four are 4-element aligned) and all four lie below `lim`.
+__device__ __forceinline__ void unpack4(const uint2& q, float (&v)[4], __nv_bfloat16) {
+  v[0] = __uint_as_float(q.x << 16);
+  v[1] = __uint_as_float(q.x & 0xffff0000u);
+  v[2] = __uint_as_float(q.y << 16);
+  v[3] = __uint_as_float(q.y & 0xffff0000u);
+}
+__device__ __forceinline__ void unpack4(const uint2& q, float (&v)[4], __half) {
+  const float2 lo = __half22float2(*reinterpret_cast<const __half2*>(&q.x));
+  const float2 hi = __half22float2(*reinterpret_cast<const __half2*>(&q.y));
+  v[0] = lo.x;
+  v[1] = lo.y;
+  v[2] = hi.x;
+  v[3] = hi.y;
+}
+template <typename TX>
+__device__ __forceinline__ void load4(const TX* p, long long i, long long lim, bool vec,
+                                      float (&v)[4]) {
+  if (vec && i + 3 < lim) {
+    if constexpr (sizeof(TX) == 4) {
+      const float4 q = *reinterpret_cast<const float4*>(p + i);
+      v[0] = q.x;
+      v[1] = q.y;
+      v[2] = q.z;
+      v[3] = q.w;
+    } else {
+      unpack4(*reinterpret_cast<const uint2*>(p + i), v, TX());
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) v[j] = (i + j < lim) ? to_f32(p[i + j]) : 0.f;
+  }
+}
+
 template <typename TW, typename TX, int NT, int BMAX>
 __global__ void __launch_bounds__(gemv_threads(BMAX), (BMAX <= 2) ? 2 : 1)
     sparse_gemv_kernel(const GemvArgs a) {
@@ -102,34 +137,48 @@ __global__ void __launch_bounds__(gemv_threads(BMAX), (BMAX <= 2) ? 2 : 1)
 
   // ---------------------------------------------------------------- 1. active list
   if (a.idx == nullptr) {
-    // Every thread tests a contiguous run of at most kPer rows of the slice;
-    // all its x loads are independent, so the CTA pays one L2 round trip for
-    // x. One block scan of the per-thread counts then places each active row,
-    // and the list comes out ascending.
-    constexpr int kPer = rows_per_thread_max(BMAX);
+    // Every active thread tests a contiguous run of r rows of the slice, r a
+    // multiple of 4 and at least 4, in groups of four whose x values come in
+    // one vector load; all of a thread's loads are independent, so the CTA
+    // pays one L2 round trip for x. Runs of at least four rows keep the
+    // number of threads (and instructions) that take part small: on B200 the
+    // compaction of a few hundred rows is bound by instruction issue, not by
+    // memory. One block scan of the per-thread counts then places the active
+    // rows, ascending.
+    constexpr int KG = (rows_per_thread_max(BMAX) + 3) / 4;  // groups of 4 per thread
     const long long k0 = (long long)split * a.slice;
     const long long k1 = min(a.K, k0 + a.slice);
     const int n = (int)max(0LL, k1 - k0);
-    const int r = (n + kThreads - 1) / kThreads;  // <= kPer (slice <= list_cap_max)
+    const int r = 4 * ((n + 4 * kThreads - 1) / (4 * kThreads));  // <= 4 KG
     const long long i0 = k0 + (long long)tid * r;
     const TX* xp = reinterpret_cast<const TX*>(a.x);
-    float xv[kPer][BMAX];
-#pragma unroll
-    for (int u = 0; u < kPer; ++u)
-#pragma unroll
-      for (int b = 0; b < BMAX; ++b)
-        xv[u][b] = (u < r && i0 + u < k1 && b < a.B) ? to_f32(xp[(long long)b * a.K + i0 + u]) : 0.f;
+    const bool vec = (reinterpret_cast<uintptr_t>(a.x) % (4 * sizeof(TX))) == 0 &&
+                     (a.B == 1 || (a.K & 3) == 0);
+    float xv[4 * KG][BMAX];
     unsigned act = 0;
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      bool any = false;
+    for (int g = 0; g < KG; ++g) {
+      const long long i = i0 + 4 * g;
+      if (4 * g < r && i < k1) {
 #pragma unroll
-      for (int b = 0; b < BMAX; ++b) {
-        const bool m = (u < r && i0 + u < k1 && b < a.B) && fabsf(xv[u][b]) > a.t;
-        any |= m;
-        if (!m && !a.union_mask) xv[u][b] = 0.f;
+        for (int b = 0; b < BMAX; ++b) {
+          float v[4] = {0.f, 0.f, 0.f, 0.f};
+          if (b < a.B) load4(xp + (long long)b * a.K, i, k1, vec, v);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) xv[4 * g + j][b] = v[j];
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          bool any = false;
+#pragma unroll
+          for (int b = 0; b < BMAX; ++b) {
+            const bool m = b < a.B && i + j < k1 && fabsf(xv[4 * g + j][b]) > a.t;
+            any |= m;
+            if (!m && !a.union_mask) xv[4 * g + j][b] = 0.f;
+          }
+          if (any) act |= 1u << (4 * g + j);
+        }
       }
-      if (any) act |= 1u << u;
     }
     // exclusive scan of the counts: warp shuffles, then the warp totals
     const int mine = __popc(act);
@@ -149,12 +198,17 @@ __global__ void __launch_bounds__(gemv_threads(BMAX), (BMAX <= 2) ? 2 : 1)
       tot += c;
     }
 #pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      if ((act >> u) & 1u) {
-        list_row[pos] = (int32_t)(i0 + u);
+    for (int g = 0; g < KG; ++g) {
+      if ((act >> (4 * g)) & 0xFu) {
 #pragma unroll
-        for (int b = 0; b < BMAX; ++b) list_x[pos * BMAX + b] = xv[u][b];
-        ++pos;
+        for (int j = 0; j < 4; ++j) {
+          if ((act >> (4 * g + j)) & 1u) {
+            list_row[pos] = (int32_t)(i0 + 4 * g + j);
+#pragma unroll
+            for (int b = 0; b < BMAX; ++b) list_x[pos * BMAX + b] = xv[4 * g + j][b];
+            ++pos;
+          }
+        }
       }
     }
     if (tid == 0) s_count = tot;
@@ -295,21 +349,22 @@ __global__ void __launch_bounds__(gemv_threads(BMAX), (BMAX <= 2) ? 2 : 1)
     const float4* pb = reinterpret_cast<const float4*>(a.partials + (long long)b * N + n0);
     for (int e = tid; e < 4 * nv; e += kThreads) {
       const int g = e / nv, v = e - g * nv;
+      // up to eight of the group's partials are loaded at once, then added
+      // in split order
       float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
-      int s = g;
-      for (; s + 12 < a.S; s += 16) {
-        const float4 q0 = __ldcg(pb + (long long)(s + 0) * vs + v);
-        const float4 q1 = __ldcg(pb + (long long)(s + 4) * vs + v);
-        const float4 q2 = __ldcg(pb + (long long)(s + 8) * vs + v);
-        const float4 q3 = __ldcg(pb + (long long)(s + 12) * vs + v);
-        acc4.x += q0.x; acc4.y += q0.y; acc4.z += q0.z; acc4.w += q0.w;
-        acc4.x += q1.x; acc4.y += q1.y; acc4.z += q1.z; acc4.w += q1.w;
-        acc4.x += q2.x; acc4.y += q2.y; acc4.z += q2.z; acc4.w += q2.w;
-        acc4.x += q3.x; acc4.y += q3.y; acc4.z += q3.z; acc4.w += q3.w;
-      }
-      for (; s < a.S; s += 4) {
-        const float4 q0 = __ldcg(pb + (long long)s * vs + v);
-        acc4.x += q0.x; acc4.y += q0.y; acc4.z += q0.z; acc4.w += q0.w;
+      for (int s0 = g; s0 < a.S; s0 += 32) {
+        float4 q[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int s = s0 + 4 * u;
+          q[u] = s < a.S ? __ldcg(pb + (long long)s * vs + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (s0 + 4 * u < a.S) {
+            acc4.x += q[u].x; acc4.y += q[u].y; acc4.z += q[u].z; acc4.w += q[u].w;
+          }
+        }
       }
       gsum[g * nv + v] = acc4;
     }

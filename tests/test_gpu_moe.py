@@ -115,7 +115,8 @@ def test_moe_top1_of_1():
     run_case("moe-one", 4, 1, 128, 32, 1, 0, 0.5)
 
 
-@pytest.mark.parametrize("B,p", [(1, 0.5), (4, 0.8), (8, 0.5)])
+@pytest.mark.parametrize("B,p", [(1, 0.5), (4, 0.8), (8, 0.5), (16, 0.5), (16, 0.9), (1, 0.9)])
 def test_moe_128_experts_full_size(B, p):
-    # 128 experts, d = 2048, expert ffn = 768 SwiGLU, top-8, shared ffn = 2048
+    # 128 experts, d = 2048, expert ffn = 768 SwiGLU, top-8, shared ffn = 2048,
+    # at the batches and sparsities the bench times (16 tokens touch ~80 experts)
     run_case("moe-config", B, 128, 2048, 768, 8, 2048, p)

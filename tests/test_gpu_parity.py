@@ -356,8 +356,9 @@ def test_workspace_shared_across_operations():
 # (the tcgen05 kernel; the default mma.sync kernel has its own test file)
 
 @pytest.fixture
-def tc_union(monkeypatch):
-    monkeypatch.setenv("SFX_UNION_KERNEL", "tc")
+def tc_union():
+    with sb.plan_overrides(union_kernel=sb.UNION_TCGEN05):
+        yield
 
 
 @pytest.mark.parametrize("B,K,N,p,wdt,xdt,out", [
@@ -443,3 +444,39 @@ def test_ffn_swiglu_llama3_70b_full_size_sampled(B):
     Wd_cols = Wd[:, torch.from_numpy(cols).cuda()].float().cpu().numpy().astype(np.float64)
     want = O.masked_gemv(h, m_h, Wd_cols)
     assert_close(to64(out["y"])[:, cols], O.round_to(want, "bf16"), "y sampled columns (70B)")
+
+
+# ---------------------------------------------------------------- Phi-2 chain end to end
+
+@pytest.mark.parametrize("keep,sel", [(0.3, "gxo"), (0.5, "gxo"), (0.7, "gxo"), (0.3, "cgxo")])
+def test_phi2_gelu_ffn_chain_end_to_end(keep, sel):
+    # Phi-2-shaped GeLU FFN at batch 1, fp16: the dense up GEMV with the GeLU
+    # epilogue, the GxO (or corrected GxO) top-k on the GPU's own h, then the
+    # index-list down GEMV -- all three on the GPU, compared with the oracle's
+    # own chain (fp64 h, its own top-k). The kept set may differ only where the
+    # fp32 and fp64 scores straddle the k-th score ("Attribution-based Sparse
+    # Activation in Large Language Models", "implementation": top fraction per
+    # layer); the flips are counted and y is within the float tolerance.
+    d, f = 2560, 10240
+    x = synth.eval_draw("phi2-chain", "x", 1, d, "f16")[0]
+    W1 = weights(d, f, "phi2-chain-W1", "f16")
+    W2 = weights(f, d, "phi2-chain-W2", "f16")
+    g = synth.normal((f,), synth.seed_of("phi2-chain", "g"), 1.0, "f32")
+    k = O.keep_count(keep, f)
+    h_gpu = sb.sfx_sparse_gemv(dev(x), dev(W1), flags=sb.SFX_FLAG_GELU, out_dtype=torch.float32)
+    mode = sb.SFX_SEL_TOPK_GXO if sel == "gxo" else sb.SFX_SEL_TOPK_CGXO
+    s = sb.sfx_mask_compact(h_gpu[None], mode, k=k, score_l=dev(g)[None])
+    y = sb.sfx_sparse_gemv(h_gpu, dev(W2), idx=s["idx"][0], cnt=s["cnt"], out_dtype=torch.float16)
+    # the oracle's chain on the same x, W1, g, W2
+    h = O.gelu_erf(to64(x) @ to64(W1))
+    h32 = h.astype(np.float32)
+    score = O.gxo_score(g.numpy(), h32) if sel == "gxo" else O.corrected_gxo_score_f32(g.numpy(), h32)
+    m = O.topk_mask(score, k)
+    got = np.zeros(f, bool)
+    got[s["idx"][0, :int(s["cnt"][0])].cpu().numpy()] = True
+    assert int(s["cnt"][0]) == k
+    flips = int(np.count_nonzero(got != m))
+    assert flips <= 4, flips
+    assert_close(to64(h_gpu), O.round_to(h, "f32"), "h")
+    want = O.masked_gemv(h[None], m[None], to64(W2))[0]
+    assert_close(to64(y), O.round_to(want, "f16"), f"y keep={keep} {sel} ({flips} flips)")
