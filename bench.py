@@ -820,6 +820,43 @@ def reference_arm(args):
     }
 
 
+# ---------------------------------------------------------------- profiling cases
+
+PROFILE_CASES = {
+    "ffn_gate_up": "the headline gate|up GEMV (SiLU(g) * u epilogue), batch 1",
+    "ffn_down": "the headline down GEMV on the gate|up stage's h, batch 1",
+    "ffn": "the headline SwiGLU FFN call, batch 1",
+    "union_gate_up_b16": "the gate|up product of 16 tokens (batch-union kernels), same layer",
+}
+
+
+def profile_case(name, p, dev, launches=6):
+    """One layer of the headline FFN on the device; `launches` calls of one
+    kernel (or call), then exit. The ncu captures in profiles/ run this."""
+    stack = Ffn70Stack(1, dev)
+    sb = stack.sb
+    t_in, t_h = stack.thresholds(p)
+    x = stack.draws("iid", 1)
+    h = torch.empty((1, F70), dtype=torch.float32, device=dev)
+    y = torch.empty((1, D70), dtype=torch.bfloat16, device=dev)
+    sb.sfx_sparse_gemv(x, stack.Wgu[0], t=t_in, flags=sb.SFX_FLAG_SWIGLU, y=h, ws=stack.ws)
+    x16 = stack.draws("iid", 16)
+    h16 = torch.empty((16, F70), dtype=torch.float32, device=dev)
+    for _ in range(launches):
+        if name == "ffn_gate_up":
+            sb.sfx_sparse_gemv(x, stack.Wgu[0], t=t_in, flags=sb.SFX_FLAG_SWIGLU, y=h, ws=stack.ws)
+        elif name == "ffn_down":
+            sb.sfx_sparse_gemv(h, stack.Wd[0], t=t_h, y=y, ws=stack.ws)
+        elif name == "ffn":
+            stack.call(0, x, t_in, t_h, y)
+        elif name == "union_gate_up_b16":
+            sb.sfx_sparse_gemv(x16, stack.Wgu[0], t=t_in, flags=sb.SFX_FLAG_SWIGLU, y=h16,
+                               ws=stack.ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_case": name, "sparsity": p, "launches": launches,
+                      "what": PROFILE_CASES[name]}), flush=True)
+
+
 # ---------------------------------------------------------------- main
 
 def measure_step(step_fn, stream, steps, warmup, dist, dev, clocks_index=None, e2e_bufs=None):
@@ -920,6 +957,9 @@ def main():
                     help="skip the other workloads (" + ", ".join(OTHER_WORKLOADS) + ")")
     ap.add_argument("--other", default=",".join(OTHER_WORKLOADS),
                     help="comma list of the other workloads to run: " + ", ".join(OTHER_WORKLOADS))
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None,
+                    help="run one kernel of the headline layer a few times and exit (the small "
+                         "case an ncu capture runs: one 1.4 GB layer on the device)")
     args = ap.parse_args()
 
     rank, local_rank, world = env_rank()
@@ -941,6 +981,9 @@ def main():
     sb.load()
     stream = torch.cuda.Stream(dev)
     torch.cuda.set_stream(stream)
+    if args.profile_case:
+        profile_case(args.profile_case, args.sparsity, dev)
+        return
     stack = Ffn70Stack(args.layers, dev)
     L = args.layers
     t_in, t_h = stack.thresholds(args.sparsity)

@@ -152,6 +152,11 @@ int sfx_gemv_plan(int B, long long K, long long N, int flags, int idx_mode, int*
  *                         may still raise it)
  *  SFX_PLAN_UNION_S       batch-union K splits (>= 1, same caveat)
  *  SFX_PLAN_MMA_CHUNKS    mma.sync union tile in 64-column chunks: 1, 2, 4, 8
+ *  SFX_PLAN_DENSE         batches of 3-16 tokens: 1 always the union kernels
+ *                         (gathered union rows), 2 always the dense kernel
+ *                         (every row; rows no token keeps multiply zeros),
+ *                         3 the dense kernel on tcgen05 (kept for comparison);
+ *                         0 lets the device choose by the union's row count
  * Returns SFX_OK, or SFX_ERR_ARG for an unknown key or a value out of range. */
 typedef enum {
   SFX_PLAN_UNION_KERNEL = 0,
@@ -159,7 +164,8 @@ typedef enum {
   SFX_PLAN_GEMV_NT = 2,
   SFX_PLAN_GEMV_S = 3,
   SFX_PLAN_UNION_S = 4,
-  SFX_PLAN_MMA_CHUNKS = 5
+  SFX_PLAN_MMA_CHUNKS = 5,
+  SFX_PLAN_DENSE = 6
 } sfx_plan_key;
 int sfx_set_plan_override(int key, int value);
 

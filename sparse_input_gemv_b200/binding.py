@@ -355,7 +355,8 @@ def sfx_device_sm_count() -> int:
 GEMV_KERNELS = ("cuda_cores", "union_tcgen05", "union_mma")
 
 SFX_PLAN_UNION_KERNEL, SFX_PLAN_UNION_MIN_B, SFX_PLAN_GEMV_NT, SFX_PLAN_GEMV_S, SFX_PLAN_UNION_S, \
-    SFX_PLAN_MMA_CHUNKS = range(6)
+    SFX_PLAN_MMA_CHUNKS, SFX_PLAN_DENSE = range(7)
+DENSE_UNION_ONLY, DENSE_ONLY, DENSE_ONLY_TCGEN05 = 1, 2, 3
 UNION_TCGEN05, UNION_MMA = 1, 2
 
 
@@ -370,7 +371,8 @@ class plan_overrides:
     def __init__(self, **kv):
         names = {"union_kernel": SFX_PLAN_UNION_KERNEL, "union_min_b": SFX_PLAN_UNION_MIN_B,
                  "gemv_nt": SFX_PLAN_GEMV_NT, "gemv_s": SFX_PLAN_GEMV_S,
-                 "union_s": SFX_PLAN_UNION_S, "mma_chunks": SFX_PLAN_MMA_CHUNKS}
+                 "union_s": SFX_PLAN_UNION_S, "mma_chunks": SFX_PLAN_MMA_CHUNKS,
+                 "dense": SFX_PLAN_DENSE}
         self.kv = {names[k]: v for k, v in kv.items()}
 
     def __enter__(self):

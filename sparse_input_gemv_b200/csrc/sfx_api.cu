@@ -55,7 +55,7 @@ void carve_gemv(void* ws, unsigned char* body, GemvArgs& a) {
 
 namespace sfx {
 
-static constexpr int kPlanKeys = SFX_PLAN_MMA_CHUNKS + 1;
+static constexpr int kPlanKeys = SFX_PLAN_DENSE + 1;
 static std::atomic<int> g_plan_override[kPlanKeys];
 
 int plan_override(int key) {
@@ -126,6 +126,7 @@ int sfx_set_plan_override(int key, int value) {
     case SFX_PLAN_GEMV_S:
     case SFX_PLAN_UNION_S: ok = ok || value >= 1; break;
     case SFX_PLAN_MMA_CHUNKS: ok = ok || value == 1 || value == 2 || value == 4 || value == 8; break;
+    case SFX_PLAN_DENSE: ok = ok || (value >= 1 && value <= 3); break;
     default: return SFX_ERR_ARG;
   }
   if (!ok) return SFX_ERR_ARG;

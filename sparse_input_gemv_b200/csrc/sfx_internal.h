@@ -82,6 +82,10 @@ GemvPlan plan_union_tc(long long K, long long N);
 // (union_gemm_mma_kernel) instead of tcgen05 (union_gemm_tc_kernel).
 constexpr bool kUnionMmaDefault = true;
 bool union_uses_mma();
+// Batch-union products: 0 the union kernels only, 1 the device chooses between
+// the union kernels and the dense kernel by the union's row count, 2 the dense
+// kernel only (plan override SFX_PLAN_DENSE).
+int dense_mode();
 size_t union_tc_workspace_bytes(long long K, long long N, int B);
 int launch_union_tc(int wdt, int xdt, const GemvPlan& plan, const GemvArgs& a, cudaStream_t stream);
 

@@ -40,7 +40,11 @@
 #include "sfx_internal.h"
 #include "sfx_rowdot.cuh"
 
+#include <cuda.h>  // CUtensorMap (the encoder is fetched at run time; no driver library link)
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <mutex>
 
 namespace sfx {
 
@@ -61,6 +65,12 @@ constexpr int kStageBytes = kSub * kSubBytes;  // 20 KB
 constexpr int kTmemCols = 64;         // four 16-column accumulators (one per K-step of a stage)
 constexpr int kPackThreads = 256;
 
+// Which product a batch-union launch runs: the union kernels (the rows any
+// token keeps, gathered) or the dense kernel (every row, streamed as 2-D
+// tiles). With DENSE_AUTO both are launched and the one not chosen returns at
+// once; the choice is made on the device from the union's row count.
+enum DenseMode { DENSE_NEVER = 0, DENSE_AUTO = 1, DENSE_ALWAYS = 2 };
+
 struct TcArgs {
   GemvArgs g;
   int32_t* rows;      // [S x slice] union rows per split
@@ -70,7 +80,25 @@ struct TcArgs {
   int split_b;        // 1 if x is fp32 (hi + lo tiles)
   int frag;           // 1: x tiles in mma.sync A-fragment order (union_gemm_mma_kernel)
   int chunks;         // union_gemm_mma_kernel: 64-column chunks per CTA (1, 2, 4 or 8)
+  int dense_mode;     // DenseMode
+  int switch_rows;    // DENSE_AUTO: the dense kernel runs when the union has more rows
+  int dense_frag;     // the dense kernel's x tiles in A-fragment order (mma.sync warps)
 };
+
+// Union rows of the whole batch, from the count kernel's per-chunk counts
+// (every lane of the calling warp gets the sum).
+__device__ __forceinline__ long long union_total(const TcArgs& t, int lane) {
+  const int chunks = (int)((t.g.K + kPackThreads - 1) / kPackThreads);
+  long long sum = 0;
+  for (int c = lane; c < chunks; c += 32) sum += t.chunk_counts[c];
+#pragma unroll
+  for (int o = 16; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  return sum;
+}
+
+__device__ __forceinline__ bool dense_chosen(int mode, int switch_rows, long long total) {
+  return mode == DENSE_ALWAYS || (mode == DENSE_AUTO && total > switch_rows);
+}
 
 __device__ __forceinline__ void cp_async16_zfill(uint32_t dst, const void* src, bool valid,
                                                  uint64_t pol) {
@@ -217,12 +245,16 @@ __global__ void __launch_bounds__(kPackThreads) union_pack_kernel(const TcArgs t
   int32_t* rows = t.rows + (long long)split * a.slice;
   const int tile_elems = 256 * (t.split_b ? 2 : 1);  // per 16-row K-step
   uint16_t* pack = t.pack + (long long)split * (a.slice / kTcK) * tile_elems;
+  __shared__ int s_dense;
   pdl_wait();  // chunk counts of pass 1
   if (warp == 0) {
     int s = 0;
     for (int c = first + lane; c < chunk; c += 32) s += t.chunk_counts[c];
     for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if (lane == 0) s_base = s;
+    const bool dense = t.dense_mode != DENSE_NEVER &&
+                       dense_chosen(t.dense_mode, t.switch_rows, union_total(t, lane));
+    if (lane == 0) s_dense = dense ? 1 : 0;
   }
   float xv[kTcN];
   uint32_t bits = row_bits<TX>(a, i, in, xv);
@@ -230,6 +262,25 @@ __global__ void __launch_bounds__(kPackThreads) union_pack_kernel(const TcArgs t
   const unsigned bal = __ballot_sync(0xffffffffu, act);
   if (lane == 0) s_warp_tot[warp] = __popc(bal);
   __syncthreads();
+  if (s_dense) {
+    // the dense kernel's x operand: every row at its own position (tile
+    // i / 16 overall, in the layout its consumers read), zero where no token
+    // keeps the row and past K
+    const long long pos = i - (long long)split * a.slice;
+    uint16_t* tl = pack + (pos / kTcK) * tile_elems;
+    const int kk = (int)(pos % kTcK);
+    if (a.union_mask && bits) bits = (1u << a.B) - 1u;
+#pragma unroll
+    for (int b = 0; b < kTcN; ++b) {
+      const float v = ((bits >> b) & 1u) ? xv[b] : 0.f;
+      const uint16_t hi = to_bits16<TW>(v);
+      const int off = xtile_off(t.dense_frag != 0, b, kk);
+      tl[off] = hi;
+      if (t.split_b) tl[256 + off] = to_bits16<TW>(v - from_bits16<TW>(hi));
+    }
+    pdl_launch_dependents();
+    return;
+  }
   int woff = 0, tot = 0;
 #pragma unroll
   for (int w = 0; w < kPackThreads / 32; ++w) {
@@ -551,6 +602,18 @@ __global__ void __launch_bounds__(kMmaThreads, 2) union_gemm_mma_kernel(const Tc
   const int g = lane >> 2, q = lane & 3;  // fragment role
 
   pdl_wait();  // the pack kernel's rows, counts and x tiles
+  if (t.dense_mode != DENSE_NEVER) {  // the dense kernel may run this product instead
+    __shared__ int s_skip;
+    if (warp == 0) {
+      const bool dense = dense_chosen(t.dense_mode, t.switch_rows, union_total(t, lane));
+      if (lane == 0) s_skip = dense ? 1 : 0;
+    }
+    __syncthreads();
+    if (s_skip) {
+      pdl_launch_dependents();
+      return;
+    }
+  }
   const int nrows = min(max(t.counts[split], 0), a.slice);
   for (int r = tid; r < nrows; r += kMmaThreads) list_row[r] = t.rows[(long long)split * a.slice + r];
   __syncthreads();
@@ -714,6 +777,544 @@ __global__ void __launch_bounds__(kMmaThreads, 2) union_gemm_mma_kernel(const Tc
   if (tid == 0) a.counters[tile] = 0;
 }
 
+// ---------------------------------------------------------------- 4. dense TMA + tcgen05 GEMM
+
+// When the union keeps most rows, reading every row as a dense tile is cheaper
+// than gathering the union: the rows of a 128-column tile arrive as two 2-D
+// TMA boxes of 64 columns x 128 rows (16 KB each, 128-byte swizzle), and a
+// 16-byte-gather cannot move bytes as fast (measured on B200: 16 KB 2-D boxes
+// from two issuing lanes stream 6.9 TB/s; 16-byte gathers into shared memory
+// 3.5 TB/s). The x operand for all K rows comes from the pack kernel as the
+// same 16 x 16 K-major tiles, with the rows no token keeps holding zeros, so
+// the product is the same masked one as the union kernels compute.
+//
+// One persistent CTA per SM; CTA c streams stages [W c / G, W (c + 1) / G) of
+// the (column tile, 128-row stage) sequence, so every CTA moves the same
+// number of bytes. Warp 4 lanes 0 and 1 issue the two boxes of a stage (lane
+// 0 also the stage's x tiles, a 1-D bulk copy) into a 4-stage ring; warp 5
+// lane 0 issues tcgen05.mma, M = 128 columns (A: the stage, MN-major, 128-byte
+// swizzle), N = 16 tokens (B: the x tiles, K-major), K = 16, one accumulator
+// per K-step of the stage, into one of two TMEM accumulator sets per run of
+// stages on one tile (a "segment"); warps 0-3 read a finished segment's
+// accumulators (TMEM lane = column), sum them in K-step order and either
+// write the tile (a segment that covers all of K) or its partial, after
+// which the last segment of the tile to arrive adds the partials in segment
+// order (deterministic). Every wait is bounded; on timeout the kernel raises
+// SFX_DEV_TIMEOUT, waits (bounded) for its copies and MMAs, frees its TMEM and
+// returns.
+constexpr int kDM = 128;                          // output columns per tile
+constexpr int kDRows = 128;                       // rows of W per stage
+constexpr int kDSteps = kDRows / kTcK;            // 8 K-steps per stage
+constexpr int kDStages = 4;
+constexpr int kDBoxBytes = 64 * kDRows * 2;       // one 64-column box: 16 KB
+constexpr int kDABytes = 2 * kDBoxBytes;          // 32 KB of W per stage
+constexpr int kDThreads = 192;                    // warps 0-3 epilogue, 4 TMA, 5 MMA
+constexpr int kDTmemCols = 256;                   // two sets of 8 accumulators x 16 columns
+__host__ __device__ constexpr int dense_b_bytes(bool split) { return kDSteps * kBBytes * (split ? 2 : 1); }
+__host__ __device__ constexpr int dense_stage_bytes(bool split) { return kDABytes + dense_b_bytes(split); }
+__host__ __device__ constexpr size_t dense_smem_bytes(bool split) {
+  return (size_t)kDStages * dense_stage_bytes(split) + 1024;  // + alignment slack
+}
+
+struct DenseArgs {
+  TcArgs t;
+  long long T;          // column tiles of kDM columns
+  long long SPT;        // stages per tile (ceil(K / kDRows))
+  long long W;          // T * SPT
+  int max_seg;          // partial slots per tile
+};
+
+// Barrier 1 over the four epilogue warps (128 threads), returning the OR of
+// `pred` over them.
+__device__ __forceinline__ bool named_barrier_or(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&d)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+               : "r"(addr)
+               : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return smem_desc(addr, lbo, sbo) | (2ull << 61);  // layout: 128-byte swizzle
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar, uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(map), "r"(c0), "r"(c1), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// CTA holding stage-iteration w of the stream-K split over G CTAs:
+// CTA c covers [W c / G, W (c + 1) / G).
+__device__ __forceinline__ long long dense_cta_of(long long w, long long W, long long G) {
+  return ((w + 1) * G - 1) / W;
+}
+
+template <typename TW, bool SPLIT>
+__global__ void __launch_bounds__(kDThreads, 1)
+    dense_gemm_tma_kernel(const __grid_constant__ CUtensorMap wmap, const DenseArgs d) {
+  const TcArgs& t = d.t;
+  const GemvArgs& a = t.g;
+  constexpr int SB = dense_stage_bytes(SPLIT);
+  constexpr int BB = dense_b_bytes(SPLIT);
+  constexpr int kTileElems = 256 * (SPLIT ? 2 : 1);
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t s_full[kDStages];
+  __shared__ __align__(8) uint64_t s_empty[kDStages];
+  __shared__ __align__(8) uint64_t s_acc_full[2];
+  __shared__ __align__(8) uint64_t s_acc_empty[2];
+  __shared__ uint32_t s_tmem;
+  __shared__ int s_abort;
+  __shared__ int s_last;
+  __shared__ int s_skip;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;  // 128-byte swizzle atoms
+  const long long G = gridDim.x, c = blockIdx.x;
+  const long long w0 = d.W * c / G, w1 = d.W * (c + 1) / G;
+  const long long n = w1 - w0;
+
+  pdl_wait();  // the count and pack kernels' results
+  if (warp == 0) {
+    const long long total = union_total(t, lane);
+    if (lane == 0) s_skip = dense_chosen(t.dense_mode, t.switch_rows, total) ? 0 : 1;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kDStages; ++s) {
+      mbar_init(&s_full[s], 2);  // the two issuing lanes
+      mbar_init(&s_empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_acc_full[i], 1);
+      mbar_init(&s_acc_empty[i], 128);
+    }
+    fence_barrier_init();
+    s_abort = 0;
+  }
+  __syncthreads();
+  if (s_skip) {  // the union kernels run this product
+    pdl_launch_dependents();
+    return;
+  }
+  if (warp == 5) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(&s_tmem)),
+                 "r"(kDTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_tmem;
+  const uint16_t* pack = t.pack;  // all K rows, split-major = row-major tiles
+
+  if (warp == 4) {
+    // ------------------------------------------------ TMA producers
+    if (lane < 2) {
+      const uint64_t pol = l2_evict_first_policy();
+      long long j = 0;
+      for (; j < n; ++j) {
+        const int s = (int)(j % kDStages);
+        const uint32_t use = (uint32_t)(j / kDStages);
+        if (use > 0 && !mbar_wait(&s_empty[s], (use - 1) & 1, &s_abort)) {
+          s_abort = 1;
+          raise_status(a.status, SFX_DEV_TIMEOUT);
+          break;
+        }
+        const long long w = w0 + j, tile = w / d.SPT, ks = w - tile * d.SPT;
+        const uint32_t st = base + (uint32_t)(s * SB);
+        const int col = (int)(tile * kDM) + 64 * lane;  // a multiple of 64 elements
+        const int row = (int)(ks * kDRows);
+        mbar_arrive_expect_tx(&s_full[s], kDBoxBytes + (lane == 0 ? BB : 0));
+        tma_load_2d(st + (uint32_t)(lane * kDBoxBytes), &wmap, col, row, &s_full[s], pol);
+        if (lane == 0)
+          bulk_load(st + kDABytes, pack + ks * kDSteps * kTileElems, (uint32_t)BB, &s_full[s]);
+      }
+      // bounded drain: every copy this lane issued has landed before the CTA
+      // may leave (normally the MMAs have consumed them already)
+      for (long long q = (j > kDStages ? j - kDStages : 0); q < j; ++q)
+        mbar_wait(&s_full[q % kDStages], (uint32_t)((q / kDStages) & 1), nullptr, kDrainLimitNs);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = instr_desc(DT<TW>::id == SFX_BF16);
+      long long seg = -1, cur_tile = -1, last_commit = -1;
+      int set = 0;
+      for (long long j = 0; j < n && !*reinterpret_cast<volatile int*>(&s_abort); ++j) {
+        const int s = (int)(j % kDStages);
+        const long long w = w0 + j, tile = w / d.SPT;
+        const bool seg_start = tile != cur_tile;
+        if (seg_start) {
+          ++seg;
+          set = (int)(seg & 1);
+          cur_tile = tile;
+          if (seg >= 2 &&
+              !mbar_wait(&s_acc_empty[set], (uint32_t)(((seg - 2) >> 1) & 1), &s_abort)) {
+            s_abort = 1;
+            raise_status(a.status, SFX_DEV_TIMEOUT);
+            break;
+          }
+        }
+        if (!mbar_wait(&s_full[s], (uint32_t)((j / kDStages) & 1), &s_abort)) {
+          s_abort = 1;
+          raise_status(a.status, SFX_DEV_TIMEOUT);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t st = base + (uint32_t)(s * SB);
+#pragma unroll
+        for (int kk = 0; kk < kDSteps; ++kk) {
+          // A: 16 rows x 128 columns; two 64-column atoms 16 KB apart (LBO),
+          // 8-row groups 1 KB apart (SBO)
+          const uint64_t adesc = smem_desc_sw128(st + (uint32_t)(kk * kTcK * 128), kDBoxBytes, 1024);
+          const uint32_t bst = st + kDABytes + (uint32_t)(kk * kTileElems * 2);
+          const uint32_t dq = tmem + (uint32_t)(set * 128 + kk * kTcN);
+          mma_f16(dq, adesc, smem_desc(bst, 256, 128), idesc, seg_start ? 0u : 1u);
+          if (SPLIT) mma_f16(dq, adesc, smem_desc(bst + kBBytes, 256, 128), idesc, 1u);
+        }
+        mma_commit(&s_empty[s]);
+        last_commit = j;
+        const bool seg_end = (j == n - 1) || ((w + 1) / d.SPT != tile);
+        if (seg_end) mma_commit(&s_acc_full[set]);
+      }
+      // bounded: the last committed MMAs have finished before TMEM is freed
+      if (last_commit >= 0)
+        mbar_wait(&s_empty[last_commit % kDStages], (uint32_t)((last_commit / kDStages) & 1),
+                  nullptr, kDrainLimitNs);
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 0-3)
+    const long long N = a.N;
+    const bool swiglu = a.epi == EPI_SWIGLU;
+    const int m = tid;  // column within the tile = TMEM lane
+    long long seg = -1;
+    for (long long w = w0; w < w1;) {
+      const long long tile = w / d.SPT;
+      const long long we = min(w1, (tile + 1) * d.SPT);
+      const bool whole = (w == tile * d.SPT) && (we == (tile + 1) * d.SPT);
+      ++seg;
+      const int set = (int)(seg & 1);
+      w = we;
+      bool bad = !mbar_wait(&s_acc_full[set], (uint32_t)((seg >> 1) & 1), &s_abort);
+      if (bad) {
+        s_abort = 1;
+        raise_status(a.status, SFX_DEV_TIMEOUT);
+      }
+      // one decision for all four warps (a thread may have seen the abort
+      // flag while another saw the accumulators complete)
+      if (named_barrier_or(bad)) break;
+      tc_fence_after();
+      float acc[kTcN];
+#pragma unroll
+      for (int b = 0; b < kTcN; ++b) acc[b] = 0.f;
+#pragma unroll
+      for (int kk = 0; kk < kDSteps; ++kk) {
+        uint32_t r[16];
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+            "%13,%14,%15}, [%16];"
+            : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+              "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+              "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+            : "r"(tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(set * 128 + kk * kTcN)));
+        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+        for (int b = 0; b < kTcN; ++b) acc[b] += __uint_as_float(r[b]);
+      }
+      tc_fence_before();
+      mbar_arrive(&s_acc_empty[set]);  // the MMA issuer may reuse the set
+      const long long col = tile * kDM + m;
+      if (whole) {
+        // the segment is the whole tile: write it
+#pragma unroll
+        for (int b = 0; b < kTcN; ++b) {
+          if (b >= a.B) break;
+          if (swiglu) {
+            const float up = __shfl_down_sync(0xffffffffu, acc[b], 1);
+            if ((m & 1) == 0 && col < N)
+              reinterpret_cast<float*>(a.y)[(long long)b * (N / 2) + col / 2] = silu_f(acc[b]) * up;
+          } else if (col < N) {
+            store_as(a.y, (long long)b * N + col, a.ydt, epi_f(a.epi, acc[b]));
+          }
+        }
+        continue;
+      }
+      // a part of the tile: its partial, then the tile's last segment adds them up
+      const long long c_first = dense_cta_of(tile * d.SPT, d.W, G);
+      const long long c_last = dense_cta_of((tile + 1) * d.SPT - 1, d.W, G);
+      const int nseg = (int)(c_last - c_first + 1);
+      float* part = a.partials + (tile * d.max_seg) * (long long)a.B * kDM;
+#pragma unroll
+      for (int b = 0; b < kTcN; ++b)
+        if (b < a.B) part[((c - c_first) * a.B + b) * kDM + m] = acc[b];
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (tid == 0) s_last = (arrive_acq_rel(&a.counters[tile]) == nseg - 1);
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!s_last) continue;
+      for (int b = 0; b < a.B; ++b) {
+        float v = 0.f;
+        for (int q = 0; q < nseg; ++q) v += __ldcg(part + ((long long)q * a.B + b) * kDM + m);
+        if (swiglu) {
+          const float up = __shfl_down_sync(0xffffffffu, v, 1);
+          if ((m & 1) == 0 && col < N)
+            reinterpret_cast<float*>(a.y)[(long long)b * (N / 2) + col / 2] = silu_f(v) * up;
+        } else if (col < N) {
+          store_as(a.y, (long long)b * N + col, a.ydt, epi_f(a.epi, v));
+        }
+      }
+      if (tid == 0) a.counters[tile] = 0;
+    }
+  }
+  pdl_launch_dependents();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(kDTmemCols)
+                 : "memory");
+  }
+}
+
+// The dense product with mma.sync consumers (the default dense kernel): the
+// same TMA-fed ring and stream-K split as dense_gemm_tma_kernel, but eight
+// consumer warps multiply each stage, warp w owning columns 16w .. 16w + 15 of
+// the tile for all eight K-blocks: ldmatrix.x4.trans reads the two 8-column
+// blocks of a K-block straight out of the 128-byte-swizzled box (the B
+// fragments of m16n8k16), the x fragment is one 16-byte shared load of the
+// K-block's tile (A-fragment order), and the warp keeps its 16 x 16 partial in
+// eight registers per lane, so no warp-to-warp reduction is needed. Measured
+// on B200 at 16 tokens: tcgen05.mma with N = 16 tokens and an MN-major A took
+// ~0.12 us per 4 KB of A, which held the tcgen05 version of this kernel to
+// 5.2 TB/s; the mma.sync warps keep pace with the TMA stream.
+constexpr int kDMWarps = 8;                        // consumer warps
+constexpr int kDMThreads = (kDMWarps + 1) * 32;    // + the TMA warp
+
+template <typename TW, bool SPLIT>
+__global__ void __launch_bounds__(kDMThreads, 1)
+    dense_gemm_mma_kernel(const __grid_constant__ CUtensorMap wmap, const DenseArgs d) {
+  const TcArgs& t = d.t;
+  const GemvArgs& a = t.g;
+  constexpr int SB = dense_stage_bytes(SPLIT);
+  constexpr int BB = dense_b_bytes(SPLIT);
+  constexpr int kTileElems = 256 * (SPLIT ? 2 : 1);
+  extern __shared__ unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t s_full[kDStages];
+  __shared__ __align__(8) uint64_t s_empty[kDStages];
+  __shared__ int s_abort;
+  __shared__ int s_last;
+  __shared__ int s_skip;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t base = (smem_u32(smem_raw) + 1023u) & ~1023u;  // 128-byte swizzle atoms
+  const long long G = gridDim.x, c = blockIdx.x;
+  const long long w0 = d.W * c / G, w1 = d.W * (c + 1) / G;
+  const long long n = w1 - w0;
+
+  pdl_wait();  // the count and pack kernels' results
+  if (warp == 0) {
+    const long long total = union_total(t, lane);
+    if (lane == 0) s_skip = dense_chosen(t.dense_mode, t.switch_rows, total) ? 0 : 1;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kDStages; ++s) {
+      mbar_init(&s_full[s], 2);         // the two issuing lanes
+      mbar_init(&s_empty[s], kDMWarps);  // one arrival per consumer warp
+    }
+    fence_barrier_init();
+    s_abort = 0;
+  }
+  __syncthreads();
+  if (s_skip) {  // the union kernels run this product
+    pdl_launch_dependents();
+    return;
+  }
+  const uint16_t* pack = t.pack;  // all K rows, split-major = row-major tiles
+
+  if (warp == kDMWarps) {
+    // ------------------------------------------------ TMA producers
+    if (lane < 2) {
+      const uint64_t pol = l2_evict_first_policy();
+      long long j = 0;
+      for (; j < n; ++j) {
+        const int s = (int)(j % kDStages);
+        const uint32_t use = (uint32_t)(j / kDStages);
+        if (use > 0 && !mbar_wait(&s_empty[s], (use - 1) & 1, &s_abort)) {
+          s_abort = 1;
+          raise_status(a.status, SFX_DEV_TIMEOUT);
+          break;
+        }
+        const long long w = w0 + j, tile = w / d.SPT, ks = w - tile * d.SPT;
+        const uint32_t st = base + (uint32_t)(s * SB);
+        const int col = (int)(tile * kDM) + 64 * lane;  // a multiple of 64 elements
+        const int row = (int)(ks * kDRows);
+        mbar_arrive_expect_tx(&s_full[s], kDBoxBytes + (lane == 0 ? BB : 0));
+        tma_load_2d(st + (uint32_t)(lane * kDBoxBytes), &wmap, col, row, &s_full[s], pol);
+        if (lane == 0)
+          bulk_load(st + kDABytes, pack + ks * kDSteps * kTileElems, (uint32_t)BB, &s_full[s]);
+      }
+      // bounded drain: every copy this lane issued has landed before the CTA leaves
+      for (long long q = (j > kDStages ? j - kDStages : 0); q < j; ++q)
+        mbar_wait(&s_full[q % kDStages], (uint32_t)((q / kDStages) & 1), nullptr, kDrainLimitNs);
+    }
+  } else {
+    // ------------------------------------------------ consumers (warps 0-7)
+    const long long N = a.N;
+    const bool swiglu = a.epi == EPI_SWIGLU;
+    const int g = lane >> 2, q = lane & 3;
+    const int box = warp >> 2;                 // columns 0-63: box 0, 64-127: box 1
+    const int nb0 = (2 * warp) & 7;            // the warp's two 8-column blocks in its box
+    const int lm = lane >> 3, li = lane & 7;
+    const int chunk = nb0 + (lm >> 1);         // 16-byte column this lane addresses
+    float acc[2][4];
+    long long cur_tile = -1, seg_first = 0;
+    for (long long j = 0; j < n; ++j) {
+      const int s = (int)(j % kDStages);
+      const long long w = w0 + j, tile = w / d.SPT;
+      if (tile != cur_tile) {
+        cur_tile = tile;
+        seg_first = w;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
+      }
+      bool bad = !mbar_wait(&s_full[s], (uint32_t)((j / kDStages) & 1), &s_abort);
+      bad = __any_sync(0xffffffffu, bad);
+      if (bad) {
+        if (lane == 0) {
+          s_abort = 1;
+          raise_status(a.status, SFX_DEV_TIMEOUT);
+        }
+        break;
+      }
+      const uint32_t st = base + (uint32_t)(s * SB);
+      const uint32_t bx = st + (uint32_t)(box * kDBoxBytes);
+#pragma unroll
+      for (int kb = 0; kb < kDSteps; ++kb) {
+        const int r = kb * kTcK + (lm & 1) * 8 + li;
+        uint32_t b[4];
+        ldmatrix_x4_trans(bx + (uint32_t)(r * 128 + ((chunk ^ li) << 4)), b);
+        const uint32_t xs = st + kDABytes + (uint32_t)(kb * kTileElems * 2 + lane * 16);
+        const uint4 xa = lds128(xs);
+        mma_16816(acc[0], xa.x, xa.y, xa.z, xa.w, b[0], b[1], TW());
+        mma_16816(acc[1], xa.x, xa.y, xa.z, xa.w, b[2], b[3], TW());
+        if (SPLIT) {
+          const uint4 xl = lds128(xs + 512);
+          mma_16816(acc[0], xl.x, xl.y, xl.z, xl.w, b[0], b[1], TW());
+          mma_16816(acc[1], xl.x, xl.y, xl.z, xl.w, b[2], b[3], TW());
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s_empty[s]);  // the stage may be refilled
+      const bool seg_end = (j == n - 1) || ((w + 1) / d.SPT != tile);
+      if (!seg_end) continue;
+      // lane (g, q): acc[h][e] = token g (e < 2) or g + 8 (e >= 2) at tile
+      // column 16 warp + 8 h + 2q + (e & 1)
+      const bool whole = seg_first == tile * d.SPT && w + 1 == (tile + 1) * d.SPT;
+      if (whole) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const long long col = tile * kDM + 16 * warp + 8 * h + 2 * q;
+          if (col >= N) continue;
+#pragma unroll
+          for (int hi = 0; hi < 2; ++hi) {
+            const int b = g + 8 * hi;
+            if (b >= a.B) continue;
+            const float v0 = acc[h][2 * hi], v1 = acc[h][2 * hi + 1];
+            if (swiglu) {
+              reinterpret_cast<float*>(a.y)[(long long)b * (N / 2) + col / 2] = silu_f(v0) * v1;
+            } else {
+              store_as(a.y, (long long)b * N + col, a.ydt, epi_f(a.epi, v0));
+              store_as(a.y, (long long)b * N + col + 1, a.ydt, epi_f(a.epi, v1));
+            }
+          }
+        }
+        continue;
+      }
+      // a part of the tile: the warp writes its 16 columns of the segment's
+      // partial and arrives on the counter of (tile, warp); the last of the
+      // tile's segments to arrive there adds up those 16 columns in segment
+      // order. No barrier between warps: a warp that gives up on a wait cannot
+      // stall the others.
+      const long long c_first = dense_cta_of(tile * d.SPT, d.W, G);
+      const long long c_last = dense_cta_of((tile + 1) * d.SPT - 1, d.W, G);
+      const int nseg = (int)(c_last - c_first + 1);
+      float* part = a.partials + (tile * d.max_seg) * (long long)a.B * kDM;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int hi = 0; hi < 2; ++hi) {
+          const int b = g + 8 * hi;
+          if (b < a.B)
+            *reinterpret_cast<float2*>(part + ((c - c_first) * a.B + b) * kDM + 16 * warp + 8 * h +
+                                       2 * q) = make_float2(acc[h][2 * hi], acc[h][2 * hi + 1]);
+        }
+      __syncwarp();
+      int32_t* counter = a.counters + tile * kDMWarps + warp;
+      int last = 0;
+      if (lane == 0) last = arrive_acq_rel(counter) == nseg - 1;
+      last = __shfl_sync(0xffffffffu, last, 0);
+      __syncwarp();
+      if (!last) continue;
+      for (int e = lane; e < a.B * 8; e += 32) {  // 8 column pairs per token
+        const int b = e >> 3, c2 = 16 * warp + 2 * (e & 7);
+        const long long col = tile * kDM + c2;
+        if (col >= N) continue;
+        float v0 = 0.f, v1 = 0.f;
+        for (int sg = 0; sg < nseg; ++sg) {
+          const float2 v =
+              __ldcg(reinterpret_cast<const float2*>(part + ((long long)sg * a.B + b) * kDM + c2));
+          v0 += v.x;
+          v1 += v.y;
+        }
+        if (swiglu) {
+          reinterpret_cast<float*>(a.y)[(long long)b * (N / 2) + col / 2] = silu_f(v0) * v1;
+        } else {
+          store_as(a.y, (long long)b * N + col, a.ydt, epi_f(a.epi, v0));
+          store_as(a.y, (long long)b * N + col + 1, a.ydt, epi_f(a.epi, v1));
+        }
+      }
+      if (lane == 0) *counter = 0;
+    }
+  }
+  pdl_launch_dependents();
+}
+
 // ------------------------------------------------------------------ host
 
 static long long rup(long long v, long long m) { return (v + m - 1) / m * m; }
@@ -795,10 +1396,118 @@ static TcAux tc_aux(const GemvPlan& p, long long K) {
   return x;
 }
 
+// The dense kernel's stream-K split: T column tiles of kDM columns, SPT
+// stages of kDRows rows per tile, W = T SPT stages over G CTAs (one per SM),
+// and the most CTAs that share one tile (partial slots per tile).
+struct DensePlan {
+  long long T, SPT, W, G;
+  int max_seg;
+};
+static DensePlan plan_dense(long long K, long long N) {
+  DensePlan d;
+  d.T = (N + kDM - 1) / kDM;
+  d.SPT = (K + kDRows - 1) / kDRows;
+  d.W = d.T * d.SPT;
+  d.G = std::min<long long>(sm_count(), d.W);
+  int mx = 1;
+  for (long long tile = 0; tile < d.T; ++tile) {
+    const long long c0 = ((tile * d.SPT + 1) * d.G - 1) / d.W;
+    const long long c1 = (((tile + 1) * d.SPT) * d.G - 1) / d.W;
+    mx = std::max<int>(mx, (int)(c1 - c0 + 1));
+  }
+  d.max_seg = mx;
+  return d;
+}
+
+// The union (sparse) and dense products never both run, so they share the
+// partial-sum area at the front of the workspace body.
+static size_t union_partials_bytes(const GemvPlan& p, long long K, long long N, int B) {
+  const size_t sparse = (size_t)(p.S > 1 ? p.S : 0) * B * N * 4;
+  if (p.kind != 2) return sparse;
+  const DensePlan d = plan_dense(K, N);
+  const size_t dense = (size_t)d.T * d.max_seg * B * kDM * 4;
+  return std::max(sparse, dense);
+}
+
 size_t union_tc_workspace_bytes(long long K, long long N, int B) {
   const GemvPlan p = plan_union_tc(K, N);
-  return (size_t)(p.S > 1 ? p.S : 0) * B * N * 4 + 256 /* alignment */ + tc_aux(p, K).total;
+  return union_partials_bytes(p, K, N, B) + 256 /* alignment */ + tc_aux(p, K).total;
 }
+
+// ------------------------------------------------------------------ tensor maps
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link
+// against the driver library). Maps are cached per (matrix, shape, dtype):
+// encoding one costs host time, and a call captured in a CUDA graph keeps its
+// map by value.
+using EncodeFn = PFN_cuTensorMapEncodeTiled_v12000;
+
+static EncodeFn tensor_map_encoder() {
+  static EncodeFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (EncodeFn) nullptr;
+    return reinterpret_cast<EncodeFn>(f);
+  }();
+  return fn;
+}
+
+struct MapKey {
+  const void* W;
+  long long K, N;
+  int dt;
+  bool operator==(const MapKey& o) const { return W == o.W && K == o.K && N == o.N && dt == o.dt; }
+};
+
+// The weight matrix W [K x N] (16-bit) as a 2-D tensor, boxes of 64 columns x
+// kDRows rows with the 128-byte swizzle; reads past N or K fill zeros.
+static int weight_tensor_map(const void* W, long long K, long long N, int dt, CUtensorMap* out) {
+  static std::mutex mu;
+  static MapKey keys[64];
+  static CUtensorMap maps[64];
+  static int used = 0, next = 0;
+  const MapKey key{W, K, N, dt};
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (keys[i] == key) {
+      *out = maps[i];
+      return SFX_OK;
+    }
+  EncodeFn enc = tensor_map_encoder();
+  if (!enc) return SFX_ERR_CUDA;
+  CUtensorMap m;
+  const cuuint64_t dims[2] = {(cuuint64_t)N, (cuuint64_t)K};
+  const cuuint64_t strides[1] = {(cuuint64_t)N * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kDRows};
+  const cuuint32_t es[2] = {1, 1};
+  if (enc(&m, dt == SFX_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+          const_cast<void*>(W), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return SFX_ERR_CUDA;
+  keys[next] = key;
+  maps[next] = m;
+  next = (next + 1) % 64;
+  used = std::min(used + 1, 64);
+  *out = m;
+  return SFX_OK;
+}
+
+// The union row count above which the dense kernel runs. Measured on B200 at
+// 4-16 tokens, the union kernels stream gathered rows at 4.6-5.6 TB/s and the
+// dense kernel every row at 4.9-6.5 TB/s, a ratio of 0.84-0.95 across the
+// Llama-3 8B / 70B FFN shapes: the dense product wins once the union keeps
+// more than about 85 % of the rows.
+static constexpr double kDenseSwitchFraction = 0.85;
+
+int dense_mode() {
+  // 1 union kernels only, 2 dense kernel only, 3 the tcgen05 dense kernel only
+  const int v = plan_override(SFX_PLAN_DENSE);
+  return v == 1 ? DENSE_NEVER : v >= 2 ? DENSE_ALWAYS : DENSE_AUTO;
+}
+static bool dense_on_tcgen05() { return plan_override(SFX_PLAN_DENSE) == 3; }
 
 // One opt-in per kernel (shared by the bf16/f16 and fp32 activation paths):
 // the largest dynamic shared memory any plan asks for.
@@ -826,6 +1535,21 @@ static int configure_mma_kernel() {
   return rc;
 }
 
+template <typename TW>
+static int configure_dense_kernels() {
+  const auto set = [](const void* k, bool split) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)dense_smem_bytes(split)) == cudaSuccess;
+  };
+  static int rc = (set((const void*)dense_gemm_mma_kernel<TW, false>, false) &&
+                   set((const void*)dense_gemm_mma_kernel<TW, true>, true) &&
+                   set((const void*)dense_gemm_tma_kernel<TW, false>, false) &&
+                   set((const void*)dense_gemm_tma_kernel<TW, true>, true))
+                      ? SFX_OK
+                      : SFX_ERR_CUDA;
+  return rc;
+}
+
 template <typename TW, typename TX>
 static int launch_tc(const GemvPlan& p, TcArgs t, cudaStream_t s) {
   cudaLaunchAttribute attr[1];
@@ -846,7 +1570,30 @@ static int launch_tc(const GemvPlan& p, TcArgs t, cudaStream_t s) {
     cfg.blockDim = dim3(kMmaThreads, 1, 1);
     auto kern = t.split_b ? union_gemm_mma_kernel<TW, true> : union_gemm_mma_kernel<TW, false>;
     if (configure_mma_kernel<TW>() != SFX_OK) return SFX_ERR_CUDA;
-    return cudaLaunchKernelEx(&cfg, kern, t) == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
+    if (t.dense_mode != DENSE_ALWAYS && cudaLaunchKernelEx(&cfg, kern, t) != cudaSuccess)
+      return SFX_ERR_CUDA;
+    if (t.dense_mode == DENSE_NEVER) return SFX_OK;
+    // the dense product: one CTA per SM over the stream-K split
+    DenseArgs d;
+    d.t = t;
+    const DensePlan dp = plan_dense(t.g.K, t.g.N);
+    d.T = dp.T;
+    d.SPT = dp.SPT;
+    d.W = dp.W;
+    d.max_seg = dp.max_seg;
+    CUtensorMap wmap;
+    if (weight_tensor_map(t.g.W, t.g.K, t.g.N, DT<TW>::id, &wmap) != SFX_OK) return SFX_ERR_CUDA;
+    if (configure_dense_kernels<TW>() != SFX_OK) return SFX_ERR_CUDA;
+    cfg.gridDim = dim3((unsigned)dp.G, 1, 1);
+    cfg.dynamicSmemBytes = dense_smem_bytes(t.split_b != 0);
+    if (dense_on_tcgen05()) {
+      cfg.blockDim = dim3(kDThreads, 1, 1);
+      auto dk = t.split_b ? dense_gemm_tma_kernel<TW, true> : dense_gemm_tma_kernel<TW, false>;
+      return cudaLaunchKernelEx(&cfg, dk, wmap, d) == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
+    }
+    cfg.blockDim = dim3(kDMThreads, 1, 1);
+    auto dk = t.split_b ? dense_gemm_mma_kernel<TW, true> : dense_gemm_mma_kernel<TW, false>;
+    return cudaLaunchKernelEx(&cfg, dk, wmap, d) == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
   }
   auto kern = union_gemm_tc_kernel<TW>;
   if (configure_tc_kernel<TW>() != SFX_OK) return SFX_ERR_CUDA;
@@ -861,9 +1608,9 @@ int launch_union_tc(int wdt, int xdt, const GemvPlan& p, const GemvArgs& a, cuda
   t.g.S = p.S;
   t.g.slice = p.slice;
   t.g.list_cap = p.list_cap;
-  // auxiliary buffers follow the split-K partials in the workspace
+  // auxiliary buffers follow the partial sums in the workspace
   unsigned char* aux = reinterpret_cast<unsigned char*>(a.partials) +
-                       (size_t)(p.S > 1 ? p.S : 0) * a.B * a.N * 4;
+                       union_partials_bytes(p, a.K, a.N, a.B);
   aux = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(aux) + 255) & ~uintptr_t(255));
   const TcAux lay = tc_aux(p, a.K);
   t.rows = reinterpret_cast<int32_t*>(aux + lay.rows);
@@ -872,6 +1619,15 @@ int launch_union_tc(int wdt, int xdt, const GemvPlan& p, const GemvArgs& a, cuda
   t.pack = reinterpret_cast<uint16_t*>(aux + lay.pack);
   t.split_b = xdt == SFX_F32 ? 1 : 0;
   t.frag = p.kind == 2 ? 1 : 0;
+  // the sparse/dense switch: with the mma.sync union kernel, the dense kernel
+  // takes the product when the union keeps more than kDenseSwitchFraction of
+  // the rows (decided on the device from the union count)
+  t.dense_mode = p.kind == 2 ? dense_mode() : DENSE_NEVER;
+  t.switch_rows = (int)std::min<long long>(a.K, (long long)(kDenseSwitchFraction * (double)a.K));
+  t.dense_frag = dense_on_tcgen05() ? 0 : 1;
+  // counters: one per tile (tcgen05 kernel) or per tile and consumer warp
+  if (t.dense_mode != DENSE_NEVER && plan_dense(a.K, a.N).T * kDMWarps > kCounterSlots)
+    t.dense_mode = DENSE_NEVER;
   t.chunks = p.chunks;
   if (wdt == SFX_BF16) {
     if (xdt == SFX_BF16) return launch_tc<__nv_bfloat16, __nv_bfloat16>(p, t, s);
