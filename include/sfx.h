@@ -157,6 +157,9 @@ int sfx_gemv_plan(int B, long long K, long long N, int flags, int idx_mode, int*
  *                         (every row; rows no token keeps multiply zeros),
  *                         3 the dense kernel on tcgen05 (kept for comparison);
  *                         0 lets the device choose by the union's row count
+ *  SFX_PLAN_TEST_STALL    tests only: 1 makes the dense kernels leave their
+ *                         first ring stage incomplete, so every wait on it
+ *                         runs out (see sfx_set_wait_limit_ns)
  * Returns SFX_OK, or SFX_ERR_ARG for an unknown key or a value out of range. */
 typedef enum {
   SFX_PLAN_UNION_KERNEL = 0,
@@ -165,9 +168,22 @@ typedef enum {
   SFX_PLAN_GEMV_S = 3,
   SFX_PLAN_UNION_S = 4,
   SFX_PLAN_MMA_CHUNKS = 5,
-  SFX_PLAN_DENSE = 6
+  SFX_PLAN_DENSE = 6,
+  SFX_PLAN_TEST_STALL = 7
 } sfx_plan_key;
 int sfx_set_plan_override(int key, int value);
+
+/* Limit of the kernels' bounded waits, in nanoseconds, for calls made after
+ * this one returns (host only, process-wide). Kernels that hand data between
+ * warps through mbarriers (the batch-union tcgen05 kernel and the dense
+ * kernels of the batch path) never wait longer than this: a wait that runs
+ * out raises SFX_DEV_TIMEOUT in the workspace status word, waits (at most
+ * 20 ms) for the copies and MMAs it started, releases its tensor memory and
+ * returns, so the context stays usable; the output is then incomplete.
+ * After a timeout the workspace's arrival counters may be left mid-count:
+ * re-initialise it (sfx_workspace_init) before its next use.
+ * 0 restores the default of 2 s. Returns SFX_OK. */
+int sfx_set_wait_limit_ns(unsigned long long ns);
 
 /* ------------------------------------------------------------------------
  * a1. Threshold calibration                                 [TEAL] slide 8

@@ -41,6 +41,7 @@ _SIGS = {
     "sfx_build_info": (ctypes.c_char_p, []),
     "sfx_gemv_plan": (_I, [_I, _LL, _LL, _I, _I, _VP]),
     "sfx_set_plan_override": (_I, [_I, _I]),
+    "sfx_set_wait_limit_ns": (_I, [ctypes.c_ulonglong]),
     "sfx_calibrate_thresholds": (_I, [_VP, _I, _LL, _LL, _VP, _I, _VP, _VP, _SZ, _VP]),
     "sfx_mask_compact": (_I, [_VP, _I, _I, _I, _I, _F, _I, _VP, _VP, _D, _VP, _VP, _VP, _VP, _VP,
                               _VP, _SZ, _VP]),
@@ -355,7 +356,7 @@ def sfx_device_sm_count() -> int:
 GEMV_KERNELS = ("cuda_cores", "union_tcgen05", "union_mma")
 
 SFX_PLAN_UNION_KERNEL, SFX_PLAN_UNION_MIN_B, SFX_PLAN_GEMV_NT, SFX_PLAN_GEMV_S, SFX_PLAN_UNION_S, \
-    SFX_PLAN_MMA_CHUNKS, SFX_PLAN_DENSE = range(7)
+    SFX_PLAN_MMA_CHUNKS, SFX_PLAN_DENSE, SFX_PLAN_TEST_STALL = range(8)
 DENSE_UNION_ONLY, DENSE_ONLY, DENSE_ONLY_TCGEN05 = 1, 2, 3
 UNION_TCGEN05, UNION_MMA = 1, 2
 
@@ -365,6 +366,11 @@ def sfx_set_plan_override(key: int, value: int):
     _check("sfx_set_plan_override", load().sfx_set_plan_override(int(key), int(value)))
 
 
+def sfx_set_wait_limit_ns(ns: int):
+    """Limit of the kernels' bounded waits in ns (0: the 2 s default)."""
+    _check("sfx_set_wait_limit_ns", load().sfx_set_wait_limit_ns(int(ns)))
+
+
 class plan_overrides:
     """Context manager: set plan overrides {key: value} and restore the planner on exit."""
 
@@ -372,7 +378,7 @@ class plan_overrides:
         names = {"union_kernel": SFX_PLAN_UNION_KERNEL, "union_min_b": SFX_PLAN_UNION_MIN_B,
                  "gemv_nt": SFX_PLAN_GEMV_NT, "gemv_s": SFX_PLAN_GEMV_S,
                  "union_s": SFX_PLAN_UNION_S, "mma_chunks": SFX_PLAN_MMA_CHUNKS,
-                 "dense": SFX_PLAN_DENSE}
+                 "dense": SFX_PLAN_DENSE, "test_stall": SFX_PLAN_TEST_STALL}
         self.kv = {names[k]: v for k, v in kv.items()}
 
     def __enter__(self):

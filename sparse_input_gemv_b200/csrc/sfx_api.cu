@@ -55,7 +55,13 @@ void carve_gemv(void* ws, unsigned char* body, GemvArgs& a) {
 
 namespace sfx {
 
-static constexpr int kPlanKeys = SFX_PLAN_DENSE + 1;
+static constexpr int kPlanKeys = SFX_PLAN_TEST_STALL + 1;
+static std::atomic<unsigned long long> g_wait_limit_ns{0};
+
+unsigned long long wait_limit_ns() {
+  const unsigned long long v = g_wait_limit_ns.load(std::memory_order_relaxed);
+  return v ? v : kWaitLimitNs;
+}
 static std::atomic<int> g_plan_override[kPlanKeys];
 
 int plan_override(int key) {
@@ -127,10 +133,16 @@ int sfx_set_plan_override(int key, int value) {
     case SFX_PLAN_UNION_S: ok = ok || value >= 1; break;
     case SFX_PLAN_MMA_CHUNKS: ok = ok || value == 1 || value == 2 || value == 4 || value == 8; break;
     case SFX_PLAN_DENSE: ok = ok || (value >= 1 && value <= 3); break;
+    case SFX_PLAN_TEST_STALL: ok = ok || value == 1; break;
     default: return SFX_ERR_ARG;
   }
   if (!ok) return SFX_ERR_ARG;
   g_plan_override[key].store(value, std::memory_order_relaxed);
+  return SFX_OK;
+}
+
+int sfx_set_wait_limit_ns(unsigned long long ns) {
+  g_wait_limit_ns.store(ns, std::memory_order_relaxed);
   return SFX_OK;
 }
 
@@ -271,6 +283,7 @@ int sfx_sparse_gemv(const void* x, int xdt, int B, int K, const void* W, int wdt
   a.union_mask = (flags & SFX_FLAG_UNION_MASK) ? 1 : 0;
   a.no_tc = (flags & SFX_FLAG_CUDA_CORES) ? 1 : 0;
   a.t = t;
+  a.wait_ns = wait_limit_ns();
   return launch_sparse_gemv(wdt, xdt, plan, a, as_stream(stream), false);
 }
 
@@ -303,6 +316,7 @@ int sfx_sparse_ffn_swiglu(const void* x, int dt, int B, int d, int ffn, const vo
   a.union_mask = umask;
   a.no_tc = (flags & SFX_FLAG_CUDA_CORES) ? 1 : 0;
   a.t = t_in;
+  a.wait_ns = wait_limit_ns();
   carve_gemv(ws, gbody, a);
   int rc = launch_sparse_gemv(dt, dt, plan_gemv(a.K, a.N, B, false), a, s, false);
   if (rc != SFX_OK) return rc;
@@ -321,6 +335,7 @@ int sfx_sparse_ffn_swiglu(const void* x, int dt, int B, int d, int ffn, const vo
   b.union_mask = umask;
   b.no_tc = a.no_tc;
   b.t = t_h;
+  b.wait_ns = a.wait_ns;
   carve_gemv(ws, gbody, b);
   return launch_sparse_gemv(dt, SFX_F32, plan_gemv(b.K, b.N, B, false), b, s, true);
 }

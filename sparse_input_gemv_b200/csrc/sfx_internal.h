@@ -40,6 +40,7 @@ struct GemvArgs {
   int union_mask;         // every token uses the batch-union mask
   int no_tc;              // keep B >= 4 on the CUDA-core kernel
   float t;                // magnitude threshold (threshold mode)
+  unsigned long long wait_ns;  // limit of every bounded wait in the kernel
 };
 
 struct GemvPlan {
@@ -55,6 +56,9 @@ struct GemvPlan {
 };
 
 int sm_count();
+
+// Limit of the kernels' bounded waits (sfx_set_wait_limit_ns; 2 s by default).
+unsigned long long wait_limit_ns();
 
 // Plan override for `key` (sfx_plan_key) set through sfx_set_plan_override,
 // 0 when the planner chooses.

@@ -101,5 +101,6 @@ extern "C" int sfx_sparse_gemv_noalloc(const void* x, int xdt, int B, int K, con
   a.union_mask = (flags & SFX_FLAG_UNION_MASK) ? 1 : 0;
   a.no_tc = (flags & SFX_FLAG_CUDA_CORES) ? 1 : 0;
   a.t = t;
+  a.wait_ns = wait_limit_ns();
   return launch_sparse_gemv(wdt, xdt, plan, a, s, false);
 }

@@ -83,6 +83,8 @@ struct TcArgs {
   int dense_mode;     // DenseMode
   int switch_rows;    // DENSE_AUTO: the dense kernel runs when the union has more rows
   int dense_frag;     // the dense kernel's x tiles in A-fragment order (mma.sync warps)
+  int stall_test;     // test hook: the dense kernels' second TMA lane skips stage 0, so
+                      // that stage's barrier never completes and every wait on it runs out
 };
 
 // Union rows of the whole batch, from the count kernel's per-chunk counts
@@ -371,7 +373,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) union_gemm_tc_kernel(const TcAr
     const TW* Wp = reinterpret_cast<const TW*>(a.W);
     for (int c = 0; c < nit; ++c) {
       const int s = c % kStages, use = c / kStages;
-      if (use > 0 && !mbar_wait(&s_empty[s], (use - 1) & 1, &s_abort)) {
+      if (use > 0 && !mbar_wait(&s_empty[s], (use - 1) & 1, &s_abort, a.wait_ns)) {
         s_abort = 1;
         raise_status(a.status, SFX_DEV_TIMEOUT);
         break;
@@ -404,9 +406,10 @@ __global__ void __launch_bounds__(kTcThreads, 2) union_gemm_tc_kernel(const TcAr
   } else if (lane == 0) {
     // ------------------------------------------------ MMA issuer
     constexpr uint32_t idesc = instr_desc(DT<TW>::id == SFX_BF16);
+    int last_commit = -1;
     for (int c = 0; c < nit; ++c) {
       const int s = c % kStages;
-      if (!mbar_wait(&s_full[s], (c / kStages) & 1, &s_abort)) {
+      if (!mbar_wait(&s_full[s], (c / kStages) & 1, &s_abort, a.wait_ns)) {
         s_abort = 1;
         raise_status(a.status, SFX_DEV_TIMEOUT);
         break;
@@ -424,12 +427,18 @@ __global__ void __launch_bounds__(kTcThreads, 2) union_gemm_tc_kernel(const TcAr
         if (t.split_b) mma_f16(dq, adesc, smem_desc(st + kABytes + kBBytes, 256, 128), idesc, 1u);
       }
       mma_commit(&s_empty[s]);
+      last_commit = c;
     }
+    // bounded, also after a timeout: the MMAs issued so far have finished
+    // before TMEM can be freed
+    if (last_commit >= 0)
+      mbar_wait(&s_empty[last_commit % kStages], (last_commit / kStages) & 1, nullptr,
+                kDrainLimitNs);
   }
   // all MMAs done: the last commit covers every earlier MMA
   if (nit > 0 && !s_abort) {
     const int c = nit - 1;
-    if (!mbar_wait(&s_empty[c % kStages], (c / kStages) & 1, &s_abort)) {
+    if (!mbar_wait(&s_empty[c % kStages], (c / kStages) & 1, &s_abort, a.wait_ns)) {
       s_abort = 1;
       raise_status(a.status, SFX_DEV_TIMEOUT);
     }
@@ -949,11 +958,12 @@ __global__ void __launch_bounds__(kDThreads, 1)
       for (; j < n; ++j) {
         const int s = (int)(j % kDStages);
         const uint32_t use = (uint32_t)(j / kDStages);
-        if (use > 0 && !mbar_wait(&s_empty[s], (use - 1) & 1, &s_abort)) {
+        if (use > 0 && !mbar_wait(&s_empty[s], (use - 1) & 1, &s_abort, a.wait_ns)) {
           s_abort = 1;
           raise_status(a.status, SFX_DEV_TIMEOUT);
           break;
         }
+        if (t.stall_test && lane == 1 && j == 0) continue;
         const long long w = w0 + j, tile = w / d.SPT, ks = w - tile * d.SPT;
         const uint32_t st = base + (uint32_t)(s * SB);
         const int col = (int)(tile * kDM) + 64 * lane;  // a multiple of 64 elements
@@ -983,13 +993,14 @@ __global__ void __launch_bounds__(kDThreads, 1)
           set = (int)(seg & 1);
           cur_tile = tile;
           if (seg >= 2 &&
-              !mbar_wait(&s_acc_empty[set], (uint32_t)(((seg - 2) >> 1) & 1), &s_abort)) {
+              !mbar_wait(&s_acc_empty[set], (uint32_t)(((seg - 2) >> 1) & 1), &s_abort,
+                         a.wait_ns)) {
             s_abort = 1;
             raise_status(a.status, SFX_DEV_TIMEOUT);
             break;
           }
         }
-        if (!mbar_wait(&s_full[s], (uint32_t)((j / kDStages) & 1), &s_abort)) {
+        if (!mbar_wait(&s_full[s], (uint32_t)((j / kDStages) & 1), &s_abort, a.wait_ns)) {
           s_abort = 1;
           raise_status(a.status, SFX_DEV_TIMEOUT);
           break;
@@ -1029,7 +1040,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
       ++seg;
       const int set = (int)(seg & 1);
       w = we;
-      bool bad = !mbar_wait(&s_acc_full[set], (uint32_t)((seg >> 1) & 1), &s_abort);
+      bool bad = !mbar_wait(&s_acc_full[set], (uint32_t)((seg >> 1) & 1), &s_abort, a.wait_ns);
       if (bad) {
         s_abort = 1;
         raise_status(a.status, SFX_DEV_TIMEOUT);
@@ -1173,11 +1184,12 @@ __global__ void __launch_bounds__(kDMThreads, 1)
       for (; j < n; ++j) {
         const int s = (int)(j % kDStages);
         const uint32_t use = (uint32_t)(j / kDStages);
-        if (use > 0 && !mbar_wait(&s_empty[s], (use - 1) & 1, &s_abort)) {
+        if (use > 0 && !mbar_wait(&s_empty[s], (use - 1) & 1, &s_abort, a.wait_ns)) {
           s_abort = 1;
           raise_status(a.status, SFX_DEV_TIMEOUT);
           break;
         }
+        if (t.stall_test && lane == 1 && j == 0) continue;
         const long long w = w0 + j, tile = w / d.SPT, ks = w - tile * d.SPT;
         const uint32_t st = base + (uint32_t)(s * SB);
         const int col = (int)(tile * kDM) + 64 * lane;  // a multiple of 64 elements
@@ -1213,7 +1225,7 @@ __global__ void __launch_bounds__(kDMThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) acc[h][e] = 0.f;
       }
-      bool bad = !mbar_wait(&s_full[s], (uint32_t)((j / kDStages) & 1), &s_abort);
+      bool bad = !mbar_wait(&s_full[s], (uint32_t)((j / kDStages) & 1), &s_abort, a.wait_ns);
       bad = __any_sync(0xffffffffu, bad);
       if (bad) {
         if (lane == 0) {
@@ -1625,6 +1637,7 @@ int launch_union_tc(int wdt, int xdt, const GemvPlan& p, const GemvArgs& a, cuda
   t.dense_mode = p.kind == 2 ? dense_mode() : DENSE_NEVER;
   t.switch_rows = (int)std::min<long long>(a.K, (long long)(kDenseSwitchFraction * (double)a.K));
   t.dense_frag = dense_on_tcgen05() ? 0 : 1;
+  t.stall_test = plan_override(SFX_PLAN_TEST_STALL) ? 1 : 0;
   // counters: one per tile (tcgen05 kernel) or per tile and consumer warp
   if (t.dense_mode != DENSE_NEVER && plan_dense(a.K, a.N).T * kDMWarps > kCounterSlots)
     t.dense_mode = DENSE_NEVER;
