@@ -95,7 +95,8 @@ typedef enum {
   SFX_OP_SPARSE_GEMV = 2,
   SFX_OP_FFN_SWIGLU = 3,
   SFX_OP_MOE = 4,
-  SFX_OP_STATIC_FFN = 5
+  SFX_OP_STATIC_FFN = 5,
+  SFX_OP_ERROR_CURVE = 6
 } sfx_op;
 
 /* Bytes of workspace an operation needs (>= 256: the status header).
@@ -106,6 +107,8 @@ typedef enum {
  *  MOE:           a = B, b = d,     c = E,            d = ffn (expert), e = top_k,
  *                 f = ffn_shared
  *  STATIC_FFN:    a = B, b = d,     c = ffn
+ *  ERROR_CURVE:   a = S (draws), b = K, c = N,       d = dtype of the draws,
+ *                 e = P (number of levels)
  * Returns 0 for an unknown op or invalid sizes. */
 size_t sfx_workspace_bytes(int op, long long a, long long b, long long c, long long d,
                            long long e, long long f);
@@ -405,6 +408,47 @@ int sfx_moe_expert_sparse(const void* x, int dt, const float* logits, int B, int
 int sfx_static_ffn(const void* x, int dt, int B, int d, int ffn, const void* W_aT,
                    const void* W_bT, const void* W_d, const int32_t* idx, const int32_t* cnt,
                    int flags, void* y, int ydt, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
+ * Block-wise greedy sparsity allocation        [TEAL] slide 10
+ *
+ * "TEAL: Training-Free Activation Sparsity in Large Language Models",
+ * slide 10 ("block-wise greedy optimization"): the sparsity of each block is
+ * chosen to minimise the blocks' l2 activation error under a model-wide
+ * sparsity target. Every block starts dense; each round raises by one step
+ * the block whose error would grow least; rounds repeat until the target.
+ *
+ * sfx_block_error_curve: one block's error curve. The block is an input site
+ * with its weight matrix W [K x N]; calib [S x K] are the site's calibration
+ * draws. For each level p_j the threshold t_j is calibrated on calib exactly
+ * as sfx_calibrate_thresholds does, and
+ *   err_out[j] = || (calib * m_j) W - calib W ||   (Frobenius, over the S draws)
+ * with m_j = 1[|calib| > t_j]; the products run through sfx_sparse_gemv (fp32
+ * outputs) and the squared changes are summed in fp64 in a fixed order.
+ *  calib  (dev)  [S x K] dtype xdt (f16, bf16 or f32); W (dev) [K x N] wdt
+ *  levels (host) [P] sparsities in [0, 1], 1 <= P <= 64
+ *  err_out (host) [P] double; thr_out (host, optional) [P] float thresholds
+ *  ws     (dev)  sfx_workspace_bytes(SFX_OP_ERROR_CURVE, S, K, N, xdt, P),
+ *                zeroed once (sfx_workspace_init)
+ * Synchronises `stream` (the curve is returned on the host).
+ * ---------------------------------------------------------------------- */
+int sfx_block_error_curve(const void* calib, int xdt, long long S, long long K, const void* W,
+                          int wdt, long long N, const double* levels, int P, double* err_out,
+                          float* thr_out, void* ws, size_t ws_bytes, void* stream);
+
+/* sfx_greedy_allocate (host only): the greedy rounds on given error curves.
+ *  err     (host) [M x P] block i's error at level j, levels 0, step, 2 step,
+ *          ... (err[i * P] is the dense block)
+ *  weights (host) [M] the blocks' weights in the model-wide sparsity
+ *          sum_i w_i p_i / sum_i w_i (their parameter counts: the weight rows a
+ *          block's sparsity skips)
+ * Each round raises by one level the block with the smallest error growth
+ * err[i][l_i + 1] - err[i][l_i] (equal growths: the lower block index) among
+ * the blocks below level P - 1, until the model-wide sparsity reaches
+ * `target` or no block can go further. level_out (host) [M] receives l_i
+ * (block sparsity = l_i * step). Returns SFX_OK or SFX_ERR_ARG. */
+int sfx_greedy_allocate(const double* err, const double* weights, int M, int P, double step,
+                        double target, int* level_out);
 
 #ifdef __cplusplus
 }

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_PKG, "libsfx.so")
 SFX_F16, SFX_BF16, SFX_F32 = 0, 1, 2
 SFX_SEL_THRESHOLD, SFX_SEL_TOPK_GXO, SFX_SEL_TOPK_GLASS, SFX_SEL_TOPK_CGXO = 0, 1, 2, 3
 SFX_OP_CALIBRATE, SFX_OP_MASK_COMPACT, SFX_OP_SPARSE_GEMV, SFX_OP_FFN_SWIGLU, SFX_OP_MOE, \
-    SFX_OP_STATIC_FFN = range(6)
+    SFX_OP_STATIC_FFN, SFX_OP_ERROR_CURVE = range(7)
 SFX_FLAG_GELU, SFX_FLAG_GELU_TANH, SFX_FLAG_UNION_MASK, SFX_FLAG_NO_RENORM, SFX_FLAG_CUDA_CORES = \
     0x1, 0x2, 0x4, 0x8, 0x10
 SFX_FLAG_SWIGLU = 0x20
@@ -42,6 +42,9 @@ _SIGS = {
     "sfx_gemv_plan": (_I, [_I, _LL, _LL, _I, _I, _VP]),
     "sfx_set_plan_override": (_I, [_I, _I]),
     "sfx_set_wait_limit_ns": (_I, [ctypes.c_ulonglong]),
+    "sfx_block_error_curve": (_I, [_VP, _I, _LL, _LL, _VP, _I, _LL, _VP, _I, _VP, _VP, _VP, _SZ,
+                                   _VP]),
+    "sfx_greedy_allocate": (_I, [_VP, _VP, _I, _I, _D, _D, _VP]),
     "sfx_calibrate_thresholds": (_I, [_VP, _I, _LL, _LL, _VP, _I, _VP, _VP, _SZ, _VP]),
     "sfx_mask_compact": (_I, [_VP, _I, _I, _I, _I, _F, _I, _VP, _VP, _D, _VP, _VP, _VP, _VP, _VP,
                               _VP, _SZ, _VP]),
@@ -347,6 +350,41 @@ def sfx_static_ffn(x, W_aT, W_d, idx, cnt, W_bT=None, flags=0, out_dtype=None, y
         _ptr(x2), _DT[x2.dtype], B, d, ffn, _ptr(W_aT), _ptr(W_bT), _ptr(W_d), _ptr(idx), _ptr(cnt),
         int(flags), _ptr(y), _DT[y.dtype], _ptr(buf), buf.numel(), _stream(stream)))
     return y[0] if squeeze and y.dim() == 2 else y
+
+
+def sfx_block_error_curve(calib, W, levels, ws: Workspace | None = None, stream=None):
+    """A block's l2 output error at each sparsity level (TEAL slide 10).
+
+    calib [S x K] (GPU, the site's calibration draws), W [K x N] (GPU).
+    Returns (err: list of floats, thresholds: list of floats)."""
+    _need_cuda(calib, W)
+    S, K = calib.shape
+    K2, N = W.shape
+    if K2 != K:
+        raise ValueError("calib and W disagree on K")
+    P = len(levels)
+    nbytes = sfx_workspace_bytes(SFX_OP_ERROR_CURVE, S, K, N, _DT[calib.dtype], P)
+    ws, buf = _ws(ws, nbytes, calib.device)
+    lv = (ctypes.c_double * P)(*[float(p) for p in levels])
+    err = (ctypes.c_double * P)()
+    thr = (ctypes.c_float * P)()
+    _check("sfx_block_error_curve", load().sfx_block_error_curve(
+        _ptr(calib), _DT[calib.dtype], S, K, _ptr(W), _DT[W.dtype], N,
+        ctypes.cast(lv, ctypes.c_void_p), P, ctypes.cast(err, ctypes.c_void_p),
+        ctypes.cast(thr, ctypes.c_void_p), _ptr(buf), buf.numel(), _stream(stream)))
+    return [float(v) for v in err], [float(v) for v in thr]
+
+
+def sfx_greedy_allocate(err, weights, step, target):
+    """Per-block levels from the greedy rounds (host only). err: [M][P] nested lists."""
+    M, P = len(err), len(err[0])
+    e = (ctypes.c_double * (M * P))(*[float(v) for row in err for v in row])
+    w = (ctypes.c_double * M)(*[float(v) for v in weights])
+    out = (ctypes.c_int * M)()
+    _check("sfx_greedy_allocate", load().sfx_greedy_allocate(
+        ctypes.cast(e, ctypes.c_void_p), ctypes.cast(w, ctypes.c_void_p), M, P, float(step),
+        float(target), ctypes.cast(out, ctypes.c_void_p)))
+    return [int(v) for v in out]
 
 
 def sfx_device_sm_count() -> int:

@@ -167,6 +167,8 @@ size_t sfx_workspace_bytes(int op, long long a, long long b, long long c, long l
     case SFX_OP_STATIC_FFN:
       if (a < 1 || b < 8 || c < 1) return 0;
       return kWsHeader + static_ffn_workspace_bytes((int)a, (int)b, (int)c);
+    case SFX_OP_ERROR_CURVE:
+      return error_curve_workspace_bytes(a, b, c, (int)d, (int)e);
   }
   return 0;
 }

@@ -120,6 +120,10 @@ int run_static_ffn(const void* x, int dt, int B, int d, int ffn, const void* WaT
                    const void* Wd, const int32_t* idx, const int32_t* cnt, int act, void* y,
                    int ydt, unsigned char* ws_body, unsigned* status, cudaStream_t stream);
 
+// block error curves for the greedy allocation (sfx_alloc.cu); the whole
+// workspace, headers of its sub-workspaces included
+size_t error_curve_workspace_bytes(long long S, long long K, long long N, int xdt, int P);
+
 // gate/up interleave (sfx_api.cu)
 int launch_pack_gate_up(const void* W_g, const void* W_u, int dt, int d, int ffn, void* W_gu,
                         cudaStream_t stream);
