@@ -402,20 +402,24 @@ def greedy_allocate(err, weights, step, target):
     err [M x P]: block i's error at sparsity level j (levels 0, step, 2 step,
     ..., so err[:, 0] is the dense block). Steps of the slide: every block
     starts at sparsity 0; each round measures, for every block that can still
-    go one level up, how much its error would grow; the block with the
-    smallest growth goes up one level (equal growths: the lower block index);
+    go one level up, how much its error would grow; the block whose error
+    grows least goes up one level (equal growths: the lower block index);
     rounds repeat until the overall sparsity (overall_sparsity with `weights`)
-    reaches `target`, or no block can go further. Returns the level index of
-    each block (sparsity = level * step).
+    reaches `target`, or no block can go further. Reading: blocks of unequal
+    weight buy unequal amounts of overall sparsity with one level, so the
+    growth is compared per unit of overall sparsity gained, growth / w_i
+    (with equal weights this is the raw growth the slide compares). Returns
+    the level index of each block (sparsity = level * step).
     """
     err = np.asarray(err, dtype=np.float64)
+    w = np.asarray(weights, dtype=np.float64)
     M, P = err.shape
     lvl = np.zeros(M, dtype=np.int64)
-    while overall_sparsity(lvl * step, weights) < target - 1e-12:
+    while overall_sparsity(lvl * step, w) < target - 1e-12:
         best, best_i = math.inf, -1
         for i in range(M):
-            if lvl[i] + 1 < P:
-                growth = err[i, lvl[i] + 1] - err[i, lvl[i]]
+            if lvl[i] + 1 < P and w[i] > 0:
+                growth = (err[i, lvl[i] + 1] - err[i, lvl[i]]) / w[i]
                 if growth < best:
                     best, best_i = growth, i
         if best_i < 0:

@@ -143,6 +143,20 @@ def _mutants(O):
         return lvl
     M["greedy_largest_growth"] = ("greedy_allocate", greedy_largest_growth)
 
+    def greedy_raw_growth(err, weights, step, target):
+        err = np.asarray(err, np.float64)
+        M_, P = err.shape
+        lvl = np.zeros(M_, np.int64)
+        while O.overall_sparsity(lvl * step, weights) < target - 1e-12:
+            g = [err[i, lvl[i] + 1] - err[i, lvl[i]] if lvl[i] + 1 < P else math.inf
+                 for i in range(M_)]
+            i = int(np.argmin(g))
+            if g[i] == math.inf:
+                break
+            lvl[i] += 1
+        return lvl
+    M["greedy_raw_growth"] = ("greedy_allocate", greedy_raw_growth)
+
     M["overall_unweighted"] = ("overall_sparsity",
                                lambda p, weights: float(np.mean(np.asarray(p, np.float64))))
 
@@ -167,7 +181,7 @@ MUTANT_NAMES = [
     "layer_drops_shared_expert", "gxo_not_rounded_to_fp32", "corrected_gxo_drops_half",
     "corrected_f32_ranks_abs_gxo", "corrected_f32_norm_is_l1", "corrected_f32_drops_half",
     "static_ffn_ignores_mask",
-    "bf16_rounding_truncates", "greedy_largest_growth", "overall_unweighted",
+    "bf16_rounding_truncates", "greedy_largest_growth", "greedy_raw_growth", "overall_unweighted",
     "block_error_output_norm",
 ]
 

@@ -484,6 +484,17 @@ def test_greedy_weighted_overall_sparsity_and_stop():
     assert O.greedy_allocate(err, [1.0, 3.0], 0.5, 2.0).tolist() == [2, 2]
 
 
+def test_greedy_compares_growth_per_unit_of_overall_sparsity():
+    # block 1 weighs 4x block 0: one level of block 1 gains 4x the overall
+    # sparsity, so its growth of 2 counts as 0.5 per unit against block 0's 1;
+    # going up on block 1 reaches the 40 % target with half the error of the
+    # allocation that raw growths would pick ([2, 1], error 4)
+    err = np.array([[0.0, 1.0, 2.0], [0.0, 2.0, 4.0]])
+    lvl = O.greedy_allocate(err, [1.0, 4.0], 0.5, 0.4)
+    assert lvl.tolist() == [0, 1]
+    assert err[0, lvl[0]] + err[1, lvl[1]] == 2.0
+
+
 def test_greedy_free_block_first_and_ties_to_lower_index():
     # a block that loses nothing is sparsified first; equal growths go to the
     # lower block index
