@@ -242,11 +242,15 @@ class Stack:
                                                self.Wd[0], want_h=True, ws=self.ws)["h"])
         self.calib["down-in"] = torch.cat(hc).contiguous()
 
-    def set_sparsity(self, p: float):
+    SITES = ("qkv-in", "o-in", "ffn-in", "down-in")
+
+    def set_sparsity(self, p):
+        """One sparsity for every site, or a dict {site: p} (a per-site allocation)."""
         sb = self.sb
         self.p = p
-        self.t = {s: sb.sfx_calibrate_thresholds(self.calib[s], [p], ws=self.ws)[0]
-                  for s in ("qkv-in", "o-in", "ffn-in", "down-in")}
+        ps = p if isinstance(p, dict) else {s: p for s in self.SITES}
+        self.t = {s: sb.sfx_calibrate_thresholds(self.calib[s], [ps[s]], ws=self.ws)[0]
+                  for s in self.SITES}
         # active rows per layer and site (for the algorithmic byte count)
         xq, xo, xf = self.xq.float(), self.xo.float(), self.xf.float()
         self.act_q = (xq.abs() > self.t["qkv-in"]).sum(1).tolist()
@@ -912,6 +916,36 @@ def measure_step(step_fn, stream, steps, warmup, dist, dev, clocks_index=None, e
     return res
 
 
+def greedy_allocation_8b(stack, stream, steps, target, step=0.05):
+    """TEAL slide 10 on the 8B layer: per-site sparsities from the greedy rounds on
+    the sites' l2 error curves (GPU, layer 0's weights and calibration draws), at
+    the model-wide target (sites weighted by their parameter counts), then the
+    layer timed at that allocation next to the uniform one."""
+    sb = stack.sb
+    levels = [round(step * i, 4) for i in range(int(round(0.95 / step)) + 1)]
+    weights_of = {"qkv-in": stack.Wqkv[0], "o-in": stack.Wo[0], "ffn-in": stack.Wgu[0],
+                  "down-in": stack.Wd[0]}
+    curves, weights = [], []
+    for site in stack.SITES:
+        W = weights_of[site]
+        err, _ = sb.sfx_block_error_curve(stack.calib[site].contiguous(), W, levels)
+        curves.append(err)
+        weights.append(W.shape[0] * W.shape[1])  # the weights the site's sparsity skips
+    lv = sb.sfx_greedy_allocate(curves, weights, step, target)
+    alloc = {site: round(l * step, 4) for site, l in zip(stack.SITES, lv)}
+    stack.set_sparsity(alloc)
+    r = measure_step(stack.step, stream, steps, 2, None, stack.dev)
+    us = r["ms"] * 1e3 / (steps * stack.L)
+    overall = sum(w * alloc[s] for s, w in zip(stack.SITES, weights)) / sum(weights)
+    return {"target": target, "step": step, "allocation": alloc, "overall_sparsity": overall,
+            "us_per_layer": round(us, 2),
+            "gbs": round(stack.step_bytes() * steps / (r["ms"] * 1e-3) / 1e9, 1),
+            "error_at_allocation": {s: curves[i][lv[i]] for i, s in enumerate(stack.SITES)},
+            "error_uniform": {s: curves[i][int(round(target / step))]
+                              for i, s in enumerate(stack.SITES)},
+            "note": "l2 output error of each site on its 64 calibration draws (layer 0)"}
+
+
 def llama8b_layer(stream, dev, sparsity, steps, sweep_ps, layers=32):
     """The Llama-3-8B-shaped decoder layer (qkv, o, SwiGLU FFN) at batch 1,
     secondary workload: µs per layer at `sparsity` and over a sweep."""
@@ -937,6 +971,7 @@ def llama8b_layer(stream, dev, sparsity, steps, sweep_ps, layers=32):
         kernels[name] = {"us": round(us, 2), "gbs": round(kb / (us * 1e-6) / 1e9, 1)}
     out["kernels_at_sparsity"] = {"sparsity": sparsity, **kernels}
     out["dense_library_us_per_layer"] = round(dense_library_us_per_layer(stack, stream), 2)
+    out["greedy_allocation"] = greedy_allocation_8b(stack, stream, steps, target=sparsity)
     del stack
     torch.cuda.empty_cache()
     return out

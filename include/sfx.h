@@ -416,7 +416,8 @@ int sfx_static_ffn(const void* x, int dt, int B, int d, int ffn, const void* W_a
  * slide 10 ("block-wise greedy optimization"): the sparsity of each block is
  * chosen to minimise the blocks' l2 activation error under a model-wide
  * sparsity target. Every block starts dense; each round raises by one step
- * the block whose error would grow least; rounds repeat until the target.
+ * the block whose error would grow least (per unit of model-wide sparsity);
+ * rounds repeat until the target.
  *
  * sfx_block_error_curve: one block's error curve. The block is an input site
  * with its weight matrix W [K x N]; calib [S x K] are the site's calibration
@@ -442,11 +443,13 @@ int sfx_block_error_curve(const void* calib, int xdt, long long S, long long K, 
  *  weights (host) [M] the blocks' weights in the model-wide sparsity
  *          sum_i w_i p_i / sum_i w_i (their parameter counts: the weight rows a
  *          block's sparsity skips)
- * Each round raises by one level the block with the smallest error growth
- * err[i][l_i + 1] - err[i][l_i] (equal growths: the lower block index) among
- * the blocks below level P - 1, until the model-wide sparsity reaches
- * `target` or no block can go further. level_out (host) [M] receives l_i
- * (block sparsity = l_i * step). Returns SFX_OK or SFX_ERR_ARG. */
+ * Each round raises by one level the block with the smallest error growth per
+ * unit of model-wide sparsity, (err[i][l_i + 1] - err[i][l_i]) / w_i (equal
+ * values: the lower block index), among the blocks below level P - 1 with
+ * w_i > 0, until the model-wide sparsity reaches `target` or no block can go
+ * further. With equal weights this is the slide's rule: the smallest growth.
+ * level_out (host) [M] receives l_i (block sparsity = l_i * step). Returns
+ * SFX_OK or SFX_ERR_ARG. */
 int sfx_greedy_allocate(const double* err, const double* weights, int M, int P, double step,
                         double target, int* level_out);
 

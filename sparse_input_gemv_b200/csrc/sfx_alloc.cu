@@ -2,7 +2,9 @@
 // Sparsity in Large Language Models", slide 10): every block starts dense;
 // each round measures, for every block, how much its l2 activation error
 // would grow if its sparsity went one step up, and raises the block whose
-// error grows least, until the model-wide sparsity reaches the target.
+// error grows least -- per unit of model-wide sparsity the step buys, since
+// blocks weigh differently in it -- until the model-wide sparsity reaches
+// the target.
 //
 // sfx_block_error_curve measures a block's error curve on the GPU: for each
 // sparsity level, the threshold calibrated on the block's own draws (the exact
@@ -169,8 +171,10 @@ int sfx_greedy_allocate(const double* err, const double* weights, int M, int P, 
     int pick = -1;
     double least = INFINITY;
     for (int i = 0; i < M; ++i) {
-      if (lvl[i] + 1 >= P) continue;  // already at the top level
-      const double growth = err[(size_t)i * P + lvl[i] + 1] - err[(size_t)i * P + lvl[i]];
+      if (lvl[i] + 1 >= P || !(weights[i] > 0.0)) continue;  // top level, or buys nothing
+      // error growth per unit of model-wide sparsity the step buys
+      const double growth =
+          (err[(size_t)i * P + lvl[i] + 1] - err[(size_t)i * P + lvl[i]]) / weights[i];
       if (growth < least) {  // strict: equal growths keep the lower block
         least = growth;
         pick = i;

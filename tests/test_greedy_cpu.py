@@ -2,7 +2,8 @@
 
 "TEAL: Training-Free Activation Sparsity in Large Language Models", slide 10:
 every block starts dense and each round raises the block whose l2 error grows
-least until the model-wide sparsity reaches the target. The library's host
+least (per unit of model-wide sparsity bought) until the model-wide sparsity
+reaches the target. The library's host
 routine and the oracle are separate implementations; on the same error curves
 they must pick the same level for every block.
 """
