@@ -132,7 +132,7 @@ class ClockSampler:
 KERNEL_SOURCES = ("sparse_input_gemv_b200/csrc/sfx_gemv_kernel.cuh",
                   "sparse_input_gemv_b200/csrc/sfx_gemv.cu",
                   "sparse_input_gemv_b200/csrc/sfx_common.cuh")
-PROFILE_SUMMARIES = {"ffn_gate_up": "profiles/sparse_gemv_gate_up_llama3_8b.md"}
+PROFILE_SUMMARIES = {"ffn_gate_up": "profiles/sparse_gemv_gate_up_llama3_70b_p50.md"}
 
 
 def _code_only(src: str) -> str:
