@@ -542,10 +542,12 @@ def union_counts(bitmap: torch.Tensor, B: int, n: int) -> int:
 class Ffn70Stack:
     """L Llama-3-70B-shaped SwiGLU FFN layers with distinct bf16 weights."""
 
-    def __init__(self, layers: int, dev):
+    def __init__(self, layers: int, dev, table=None):
         from sparse_input_gemv_b200 import binding as sb
         from sparse_input_gemv_b200 import synth
+        from sparse_input_gemv_b200.thresholds import ThresholdTable
         self.sb, self.synth, self.L, self.dev = sb, synth, layers, dev
+        self.table = table if table is not None else ThresholdTable()
         self.Wgu, self.Wd = [], []
         for l in range(layers):
             Wg = synth.normal((D70, F70), synth.seed_of("l70", "Wg", l), 0.02, "bf16", dev)
@@ -574,9 +576,12 @@ class Ffn70Stack:
         return s.correlated_draws("l70c", "x", B, D70, "bf16", draw=draw).to(self.dev)
 
     def thresholds(self, p, kind="iid"):
-        sb = self.sb
-        return (sb.sfx_calibrate_thresholds(self.calib[kind], [p], ws=self.ws)[0],
-                sb.sfx_calibrate_thresholds(self.hcal[kind], [p], ws=self.ws)[0])
+        """(t_in, t_h) for sparsity p, from the threshold table (calibrated on a miss)."""
+        seed = "draws 0-63"
+        return (self.table.calibrate(f"l70-{kind}", "gate_up-in", self.calib[kind], [p], seed,
+                                     ws=self.ws)[0],
+                self.table.calibrate(f"l70-{kind}", "down-in", self.hcal[kind], [p], seed,
+                                     ws=self.ws)[0])
 
     def call(self, l, x, t_in, t_h, y, h=None):
         return self.sb.sfx_sparse_ffn_swiglu(x, self.Wgu[l], self.Wd[l], t_in, t_h, y=y, h=h,
@@ -992,6 +997,9 @@ def main():
                     help="skip the other workloads (" + ", ".join(OTHER_WORKLOADS) + ")")
     ap.add_argument("--other", default=",".join(OTHER_WORKLOADS),
                     help="comma list of the other workloads to run: " + ", ".join(OTHER_WORKLOADS))
+    ap.add_argument("--threshold-table", default=None,
+                    help="JSON threshold table to read (if present) and write: the headline "
+                         "layer's calibrated thresholds keyed by (config, site, p, seed)")
     ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES), default=None,
                     help="run one kernel of the headline layer a few times and exit (the small "
                          "case an ncu capture runs: one 1.4 GB layer on the device)")
@@ -1019,7 +1027,9 @@ def main():
     if args.profile_case:
         profile_case(args.profile_case, args.sparsity, dev)
         return
-    stack = Ffn70Stack(args.layers, dev)
+    from sparse_input_gemv_b200.thresholds import ThresholdTable
+    table = ThresholdTable(args.threshold_table)
+    stack = Ffn70Stack(args.layers, dev, table)
     L = args.layers
     t_in, t_h = stack.thresholds(args.sparsity)
     xs = [stack.draws("iid", 1, draw=64 + 16 * l) for l in range(L)]
@@ -1117,6 +1127,8 @@ def main():
     if other is not None:
         line["other_workloads"] = other
     if rank == 0:
+        if args.threshold_table:
+            table.save()
         print(json.dumps(line), flush=True)
     if dist is not None:
         dist.barrier()

@@ -61,6 +61,21 @@ def test_calibration_bit_exact(dtype, S, K, ps):
             assert frac >= p - 1e-12
 
 
+def test_threshold_table_calibrates_once_and_reloads(tmp_path):
+    from sparse_input_gemv_b200.thresholds import ThresholdTable
+    calib = dev(synth.calib_draws("table", "x", 64, 4096, "bf16"))
+    ps = [0.0, 0.25, 0.5, 0.9]
+    path = str(tmp_path / "table.json")
+    tab = ThresholdTable(path)
+    t1 = tab.calibrate("cfg", "ffn-in", calib, ps, seed=3)
+    assert t1 == sb.sfx_calibrate_thresholds(calib, ps)
+    tab.save()
+    # a reloaded table answers without the calibration draws
+    back = ThresholdTable(path)
+    assert back.calibrate("cfg", "ffn-in", None, ps, seed=3) == t1
+    assert t1[2] == O.calibrate_threshold(to64(calib.cpu()), 0.5)
+
+
 def test_calibration_heavy_ties_f32():
     # values on a coarse grid: the order statistic sits inside long runs of ties
     x = torch.from_numpy(np.round(np.random.default_rng(0).laplace(size=(32, 500)) * 4) / 4)
