@@ -231,11 +231,18 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
     n_gt += (j < nt && k > 0 && key[j] > T);
     n_eq += (j < nt && k > 0 && key[j] == T);
   }
-  int tot;
-  const int eq_before = block_excl_scan(n_eq, s_w, &tot);
+  // one scan of (n_gt, n_eq) packed in 16-bit halves (K <= 32768): the threads
+  // before this one keep all their larger keys and the first `remaining` of
+  // the ties, so this thread writes from gt_before + min(eq_before, remaining)
+  int packed_tot;
+  const int packed = block_excl_scan((n_gt << 16) | n_eq, s_w, &packed_tot);
+  const int gt_before = packed >> 16, eq_before = packed & 0xffff;
   int eq_keep = (int)remaining - eq_before;
   eq_keep = eq_keep < 0 ? 0 : (eq_keep > n_eq ? n_eq : eq_keep);
-  const int pos0 = block_excl_scan(n_gt + eq_keep, s_w, &tot);
+  const int pos0 = gt_before + (eq_before < (int)remaining ? eq_before : (int)remaining);
+  const int tot = (packed_tot >> 16) + ((packed_tot & 0xffff) < (int)remaining
+                                            ? (packed_tot & 0xffff)
+                                            : (int)remaining);
   int32_t* out = idx ? idx + (long long)b * K : nullptr;
   int pos = pos0, eq_seen = 0;
   uint32_t word = 0;  // bits of the current bitmap word gathered by this thread

@@ -111,6 +111,13 @@ def test_moe_most_experts_and_tokens():
     run_case("moe-wide", 16, 1024, 128, 32, 4, 64, 0.5)
 
 
+def test_moe_x_staged_after_routing():
+    # 16 tokens of d = 6144 (the largest B * d) with 512 experts: x and the
+    # logits do not fit in shared memory side by side, so the logits overlay x
+    # and x is staged once routing is done
+    run_case("moe-tall", 16, 512, 6144, 16, 2, 0, 0.5)
+
+
 def test_moe_top1_of_1():
     run_case("moe-one", 4, 1, 128, 32, 1, 0, 0.5)
 
