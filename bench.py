@@ -836,12 +836,88 @@ PROFILE_CASES = {
     "ffn_down": "the headline down GEMV on the gate|up stage's h, batch 1",
     "ffn": "the headline SwiGLU FFN call, batch 1",
     "union_gate_up_b16": "the gate|up product of 16 tokens (batch-union kernels), same layer",
+    "union_mma_gate_up_8b_b16": "a Llama-3-8B-shaped gate|up product (W 4096 x 28672) of 16 "
+                                "correlated tokens on the gathered-union mma.sync kernel",
+    "union_tc_gate_up_8b_b16": "the same product on the tcgen05 union kernel (kept for comparison)",
+    "moe_b1": "the 128-expert MoE layer (d=2048, expert ffn=768, top-8, shared ffn=2048), batch 1",
+    "topk_phi2": "the Phi-2-shaped GeLU up GEMV (2560 -> 10240) and the GxO top-k select, keep "
+                 "1 - sparsity",
+    "static_up_phi2": "the Phi-2-shaped FFN on a static GLASS set (keep 1 - sparsity) on both "
+                      "projections, batch 1",
 }
 
 
+def profile_other(name, p, dev, launches):
+    """The small cases of profile_case outside the headline layer."""
+    from sparse_input_gemv_b200 import binding as sb
+    from sparse_input_gemv_b200 import synth
+    ws = sb.Workspace(dev)
+    if name in ("union_mma_gate_up_8b_b16", "union_tc_gate_up_8b_b16"):
+        K, N = 4096, 28672
+        W = synth.normal((K, N), synth.seed_of("prof-8b", "Wgu"), 0.02, "bf16", dev)
+        x = synth.correlated_draws("prof-8b", "x", 16, K, "bf16").to(dev)
+        calib = synth.calib_draws("prof-8b", "x", 64, K, "bf16").to(dev)
+        t = sb.sfx_calibrate_thresholds(calib, [p], ws=ws)[0]
+        h = torch.empty((16, N // 2), dtype=torch.float32, device=dev)
+        kern = sb.UNION_MMA if name.startswith("union_mma") else sb.UNION_TCGEN05
+        with sb.plan_overrides(union_kernel=kern, dense=sb.DENSE_UNION_ONLY):
+            for _ in range(launches):
+                sb.sfx_sparse_gemv(x, W, t=t, flags=sb.SFX_FLAG_SWIGLU, y=h, ws=ws)
+    elif name == "moe_b1":
+        E, d, f, fs, top = 128, 2048, 768, 2048, 8
+        WgT = synth.normal((E, f, d), synth.seed_of("prof-moe", "WgT"), 0.02, "bf16", dev)
+        WuT = synth.normal((E, f, d), synth.seed_of("prof-moe", "WuT"), 0.02, "bf16", dev)
+        Wd = synth.normal((E, f, d), synth.seed_of("prof-moe", "Wd"), 0.02, "bf16", dev)
+        Sg = synth.normal((fs, d), synth.seed_of("prof-moe", "SgT"), 0.02, "bf16", dev)
+        Su = synth.normal((fs, d), synth.seed_of("prof-moe", "SuT"), 0.02, "bf16", dev)
+        Sd = synth.normal((fs, d), synth.seed_of("prof-moe", "Sd"), 0.02, "bf16", dev)
+        # per-expert thresholds: the gate activations of 16 calibration tokens routed to
+        # every expert, calibrated per expert
+        xc = synth.calib_draws("prof-moe", "x", 16, d, "bf16").to(dev)
+        ninf = torch.full((E,), -math.inf, dtype=torch.float32, device=dev)
+        a = sb.sfx_moe_expert_sparse(xc, torch.zeros((16, E), dtype=torch.float32, device=dev),
+                                     WgT, WuT, Wd, ninf, E, want_a=True, ws=ws)["a"]
+        a_e = a.permute(1, 0, 2).contiguous()
+        te = torch.tensor([sb.sfx_calibrate_thresholds(a_e[e], [p], ws=ws)[0] for e in range(E)],
+                          dtype=torch.float32, device=dev)
+        x = synth.eval_draw("prof-moe", "x", 1, d, "bf16").to(dev)
+        logits = synth.normal((1, E), synth.seed_of("prof-moe", "logits"), 1.0, "f32", dev)
+        y = torch.empty((1, d), dtype=torch.bfloat16, device=dev)
+        for _ in range(launches):
+            sb.sfx_moe_expert_sparse(x, logits, WgT, WuT, Wd, te, top, Ws_gT=Sg, Ws_upT=Su,
+                                     Ws_d=Sd, y=y, ws=ws)
+    else:  # the Phi-2-shaped FFN cases
+        d, f = 2560, 10240
+        k = int((1.0 - p) * f + 0.5)
+        W1 = synth.normal((d, f), synth.seed_of("prof-phi2", "W1"), 0.02, "f16", dev)
+        W2 = synth.normal((f, d), synth.seed_of("prof-phi2", "W2"), 0.02, "f16", dev)
+        x = synth.eval_draw("prof-phi2", "x", 1, d, "f16").to(dev)
+        g = synth.normal((1, f), synth.seed_of("prof-phi2", "g"), 1.0, "f32", dev)
+        h = torch.empty((1, f), dtype=torch.float32, device=dev)
+        if name == "topk_phi2":
+            for _ in range(launches):
+                sb.sfx_sparse_gemv(x, W1, flags=sb.SFX_FLAG_GELU, y=h, ws=ws)
+                sb.sfx_mask_compact(h, sb.SFX_SEL_TOPK_GXO, k=k, score_l=g, ws=ws)
+        else:
+            sl = synth.abs_normal((1, f), synth.seed_of("prof-phi2", "local"), device=dev)
+            sgl = synth.abs_normal((1, f), synth.seed_of("prof-phi2", "global"), device=dev)
+            gl = sb.sfx_mask_compact(None, sb.SFX_SEL_TOPK_GLASS, k=k, score_l=sl, score_g=sgl,
+                                     lam=0.5, ws=ws)
+            W1T = W1.t().contiguous()
+            y = torch.empty((1, d), dtype=torch.float16, device=dev)
+            for _ in range(launches):
+                sb.sfx_static_ffn(x, W1T, W2, gl["idx"][0], gl["cnt"], y=y, ws=ws)
+    torch.cuda.synchronize()
+
+
 def profile_case(name, p, dev, launches=6):
-    """One layer of the headline FFN on the device; `launches` calls of one
-    kernel (or call), then exit. The ncu captures in profiles/ run this."""
+    """One kernel (or call) of a small case, `launches` times, then exit: the
+    headline layer's, or another workload's. The ncu captures in profiles/ run this."""
+    if name not in ("ffn_gate_up", "ffn_down", "ffn", "union_gate_up_b16"):
+        profile_other(name, p, dev, launches)
+        print(json.dumps({"profile_case": name, "sparsity": p, "launches": launches,
+                          "what": PROFILE_CASES[name]}), flush=True)
+        return
     stack = Ffn70Stack(1, dev)
     sb = stack.sb
     t_in, t_h = stack.thresholds(p)
