@@ -163,6 +163,9 @@ int sfx_gemv_plan(int B, long long K, long long N, int flags, int idx_mode, int*
  *  SFX_PLAN_TEST_STALL    tests only: 1 makes the dense kernels leave their
  *                         first ring stage incomplete, so every wait on it
  *                         runs out (see sfx_set_wait_limit_ns)
+ *  SFX_PLAN_MOE_CHUNK     MoE expert kernel: intermediate neurons per routed
+ *                         work item, 16..64 (the shared expert's items take
+ *                         2/3 as many)
  * Returns SFX_OK, or SFX_ERR_ARG for an unknown key or a value out of range. */
 typedef enum {
   SFX_PLAN_UNION_KERNEL = 0,
@@ -172,7 +175,8 @@ typedef enum {
   SFX_PLAN_UNION_S = 4,
   SFX_PLAN_MMA_CHUNKS = 5,
   SFX_PLAN_DENSE = 6,
-  SFX_PLAN_TEST_STALL = 7
+  SFX_PLAN_TEST_STALL = 7,
+  SFX_PLAN_MOE_CHUNK = 8
 } sfx_plan_key;
 int sfx_set_plan_override(int key, int value);
 

@@ -394,7 +394,7 @@ def sfx_device_sm_count() -> int:
 GEMV_KERNELS = ("cuda_cores", "union_tcgen05", "union_mma")
 
 SFX_PLAN_UNION_KERNEL, SFX_PLAN_UNION_MIN_B, SFX_PLAN_GEMV_NT, SFX_PLAN_GEMV_S, SFX_PLAN_UNION_S, \
-    SFX_PLAN_MMA_CHUNKS, SFX_PLAN_DENSE, SFX_PLAN_TEST_STALL = range(8)
+    SFX_PLAN_MMA_CHUNKS, SFX_PLAN_DENSE, SFX_PLAN_TEST_STALL, SFX_PLAN_MOE_CHUNK = range(9)
 DENSE_UNION_ONLY, DENSE_ONLY, DENSE_ONLY_TCGEN05 = 1, 2, 3
 UNION_TCGEN05, UNION_MMA = 1, 2
 
@@ -416,7 +416,8 @@ class plan_overrides:
         names = {"union_kernel": SFX_PLAN_UNION_KERNEL, "union_min_b": SFX_PLAN_UNION_MIN_B,
                  "gemv_nt": SFX_PLAN_GEMV_NT, "gemv_s": SFX_PLAN_GEMV_S,
                  "union_s": SFX_PLAN_UNION_S, "mma_chunks": SFX_PLAN_MMA_CHUNKS,
-                 "dense": SFX_PLAN_DENSE, "test_stall": SFX_PLAN_TEST_STALL}
+                 "dense": SFX_PLAN_DENSE, "test_stall": SFX_PLAN_TEST_STALL,
+                 "moe_chunk": SFX_PLAN_MOE_CHUNK}
         self.kv = {names[k]: v for k, v in kv.items()}
 
     def __enter__(self):

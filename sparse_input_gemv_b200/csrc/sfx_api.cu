@@ -55,7 +55,7 @@ void carve_gemv(void* ws, unsigned char* body, GemvArgs& a) {
 
 namespace sfx {
 
-static constexpr int kPlanKeys = SFX_PLAN_TEST_STALL + 1;
+static constexpr int kPlanKeys = SFX_PLAN_MOE_CHUNK + 1;
 static std::atomic<unsigned long long> g_wait_limit_ns{0};
 
 unsigned long long wait_limit_ns() {
@@ -134,6 +134,7 @@ int sfx_set_plan_override(int key, int value) {
     case SFX_PLAN_MMA_CHUNKS: ok = ok || value == 1 || value == 2 || value == 4 || value == 8; break;
     case SFX_PLAN_DENSE: ok = ok || (value >= 1 && value <= 3); break;
     case SFX_PLAN_TEST_STALL: ok = ok || value == 1; break;
+    case SFX_PLAN_MOE_CHUNK: ok = ok || (value >= 16 && value <= 64); break;
     default: return SFX_ERR_ARG;
   }
   if (!ok) return SFX_ERR_ARG;

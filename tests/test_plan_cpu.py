@@ -18,7 +18,7 @@ SHAPES = {  # (K, N) of the Llama-3 8B / 70B projections and the Phi-2 down proj
 @pytest.fixture(autouse=True)
 def _lib():
     sb.load()
-    for k in range(8):
+    for k in range(9):
         sb.sfx_set_plan_override(k, 0)
 
 
@@ -94,7 +94,8 @@ def test_plan_overrides_reject_out_of_range_values():
     for key, bad in ((sb.SFX_PLAN_UNION_KERNEL, 3), (sb.SFX_PLAN_UNION_MIN_B, 1),
                      (sb.SFX_PLAN_UNION_MIN_B, 17), (sb.SFX_PLAN_GEMV_NT, 384),
                      (sb.SFX_PLAN_GEMV_S, -1), (sb.SFX_PLAN_MMA_CHUNKS, 3), (sb.SFX_PLAN_DENSE, 4),
-                     (sb.SFX_PLAN_TEST_STALL, 2), (8, 1), (-1, 0)):
+                     (sb.SFX_PLAN_TEST_STALL, 2), (sb.SFX_PLAN_MOE_CHUNK, 15),
+                     (sb.SFX_PLAN_MOE_CHUNK, 65), (9, 1), (-1, 0)):
         with pytest.raises(sb.SfxError):
             sb.sfx_set_plan_override(key, bad)
     # the library reads no environment variable for its plans
