@@ -1364,13 +1364,15 @@ GemvPlan plan_union_tc(long long K, long long N) {
     p.smem = (size_t)kStages * kStageBytes + (size_t)p.slice * 4;
     return p;
   }
-  // mma.sync: the CTA tile (1, 2, 4 or 8 chunks of 64 columns) that needs the
-  // fewest K splits, 2 chunks among equals, else the narrowest. Measured on
-  // B200 at 16 tokens: the serial sum of many split partials by the last CTA
-  // of a tile costs more than narrow tiles do (the K-blocks of a chunk are
-  // shared by its warps and summed through shared memory).
+  // mma.sync: among the CTA tiles (1, 2, 4 or 8 chunks of 64 columns) that
+  // need the fewest K splits, the widest that still gives at least 1.5 CTAs
+  // per SM, else the narrowest. Measured on B200 at 4-16 tokens: the serial sum
+  // of many split partials by the last CTA of a tile costs more than narrow
+  // tiles do, and among tiles without extra splits wider ones win down to
+  // ~1.5 CTAs per SM (70B gate|up: 256 columns 4-6 % faster than 128; 8B
+  // gate|up: 128 columns, 224 CTAs, fastest; 70B down: 64 columns, 2 splits).
   p.kind = 2;
-  int C = 8;
+  int C = 1;
   if (plan_override(SFX_PLAN_MMA_CHUNKS)) {
     C = plan_override(SFX_PLAN_MMA_CHUNKS);
   } else {
@@ -1379,10 +1381,14 @@ GemvPlan plan_union_tc(long long K, long long N) {
       GemvPlan q;
       q.col_tiles = (int)((N + 64LL * cand - 1) / (64LL * cand));
       plan_splits(q, K, kMmaMaxSlice);
-      if (q.S < best_S || (q.S == best_S && cand == 2)) {
-        best_S = q.S;
-        C = cand;
-      }
+      best_S = std::min(best_S, q.S);
+    }
+    const long long min_ctas = (3LL * sm_count() + 1) / 2;
+    for (int cand = 1; cand <= 8; cand *= 2) {
+      GemvPlan q;
+      q.col_tiles = (int)((N + 64LL * cand - 1) / (64LL * cand));
+      plan_splits(q, K, kMmaMaxSlice);
+      if (q.S == best_S && (cand == 1 || (long long)q.col_tiles * q.S >= min_ctas)) C = cand;
     }
   }
   p.chunks = C;

@@ -51,9 +51,10 @@ def test_plan_pins_measured_choices():
     assert pin(1, "o") == {"NT": 256, "S": 16, "chunks": 0}
     assert pin(1, "8b_gate_up") == {"NT": 512, "S": 5, "chunks": 0}
     assert pin(1, "8b_down") == {"NT": 256, "S": 18, "chunks": 0}
-    # 16 tokens, mma.sync union: fewest K splits, two 64-column chunks among equals
+    # 16 tokens, mma.sync union: fewest K splits; among those the widest tile
+    # with at least 1.5 CTAs per SM (222 at 148 SMs)
     assert pin(16, "8b_gate_up") == {"NT": 128, "S": 1, "chunks": 2}
-    assert pin(16, "70b_gate_up") == {"NT": 128, "S": 1, "chunks": 2}
+    assert pin(16, "70b_gate_up") == {"NT": 256, "S": 1, "chunks": 4}
     assert pin(16, "70b_down") == {"NT": 64, "S": 2, "chunks": 1}
     assert pin(16, "8b_down") == {"NT": 64, "S": 4, "chunks": 1}
     assert pin(16, "qkv") == {"NT": 64, "S": 3, "chunks": 1}
