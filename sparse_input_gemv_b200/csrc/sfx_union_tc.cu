@@ -1513,12 +1513,15 @@ static int weight_tensor_map(const void* W, long long K, long long N, int dt, CU
   return SFX_OK;
 }
 
-// The union row count above which the dense kernel runs. Measured on B200 at
-// 4-16 tokens, the union kernels stream gathered rows at 4.6-5.6 TB/s and the
-// dense kernel every row at 4.9-6.5 TB/s, a ratio of 0.84-0.95 across the
-// Llama-3 8B / 70B FFN shapes: the dense product wins once the union keeps
-// more than about 85 % of the rows.
+// The union row fraction above which the dense kernel runs. Measured on B200
+// at 4-16 tokens, forcing each side on the 70B FFN: with 16-bit x the union
+// kernel streams gathered rows at ~0.85 of the dense kernel's rate, and the
+// gate|up product crosses over at 82-86 % of the rows; with fp32 x the dense
+// kernel's split operand (two MMAs per K-step) slows it down, and the down
+// product's union still wins at 90 % (87.0 against 88.4 us) and loses only
+// near the full union (95.4 against 89.4 us at 99.9 %).
 static constexpr double kDenseSwitchFraction = 0.85;
+static constexpr double kDenseSwitchFractionSplit = 0.93;
 
 int dense_mode() {
   // 1 union kernels only, 2 dense kernel only, 3 the tcgen05 dense kernel only
@@ -1641,7 +1644,9 @@ int launch_union_tc(int wdt, int xdt, const GemvPlan& p, const GemvArgs& a, cuda
   // takes the product when the union keeps more than kDenseSwitchFraction of
   // the rows (decided on the device from the union count)
   t.dense_mode = p.kind == 2 ? dense_mode() : DENSE_NEVER;
-  t.switch_rows = (int)std::min<long long>(a.K, (long long)(kDenseSwitchFraction * (double)a.K));
+  t.switch_rows = (int)std::min<long long>(
+      a.K, (long long)((xdt == SFX_F32 ? kDenseSwitchFractionSplit : kDenseSwitchFraction) *
+                       (double)a.K));
   t.dense_frag = dense_on_tcgen05() ? 0 : 1;
   t.stall_test = plan_override(SFX_PLAN_TEST_STALL) ? 1 : 0;
   // counters: one per tile (tcgen05 kernel) or per tile and consumer warp
