@@ -127,3 +127,11 @@ def test_moe_128_experts_full_size(B, p):
     # 128 experts, d = 2048, expert ffn = 768 SwiGLU, top-8, shared ffn = 2048,
     # at the batches and sparsities the bench times (16 tokens touch ~80 experts)
     run_case("moe-config", B, 128, 2048, 768, 8, 2048, p)
+
+
+@pytest.mark.parametrize("chunk,B", [(16, 4), (24, 16), (48, 1), (64, 8)])
+def test_moe_other_item_sizes(chunk, B):
+    # the planner's 32-neuron items are measured, not required: other sizes
+    # (ragged last chunks, 16-row tiles left partly empty) give the same layer
+    with sb.plan_overrides(moe_chunk=chunk):
+        run_case("moe-chunks", B, 32, 512, 200, 4, 136, 0.5)
