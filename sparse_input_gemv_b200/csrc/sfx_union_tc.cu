@@ -558,7 +558,7 @@ __global__ void __launch_bounds__(kTcThreads, 2) union_gemm_tc_kernel(const TcAr
 constexpr int kMmaWarps = 8;
 constexpr int kMmaThreads = kMmaWarps * 32;
 constexpr int kMmaWarpCols = 64;
-constexpr int kMmaDepth = 2;  // fp32 x: K-blocks loaded per group
+constexpr int kMmaDepth = 1;  // fp32 x: K-blocks loaded per group (1 measured best of 1-3)
 constexpr int kMmaPipe = 3;   // 16-bit x: register slots of the rolling pipeline
 // token row stride of the reduction buffer: 2 (mod 32) words, so that the
 // float2 stores of a half-warp (tokens g = 0..3, column groups q = 0..3) hit
@@ -695,7 +695,8 @@ __global__ void __launch_bounds__(kMmaThreads, 2) union_gemm_mma_kernel(const Tc
   } else {
     // fp32 x (hi + lo fragments, two MMAs per tile): the WPC warps of a chunk
     // take groups of kMmaDepth K-blocks in turn, loaded together, then
-    // multiplied (a rolling pipeline costs this variant more than it saves)
+    // multiplied (a rolling pipeline costs this variant more than it saves;
+    // on the 70B down, groups of one K-block were 2-3.5 % faster than two)
     for (int kb0 = wrow * kMmaDepth; kb0 < nblk; kb0 += WPC * kMmaDepth) {
       uint4 w[kMmaDepth][2][2];
       uint4 xa[kMmaDepth], xl[kMmaDepth];
