@@ -128,23 +128,24 @@ __global__ void __launch_bounds__(256, 4) static_up_rows_kernel(const TW* __rest
                                                                 const int32_t* __restrict__ cnt_p,
                                                                 int act, float* h,
                                                                 unsigned* status) {
-  // 16-byte loads per lane in flight per row (4 KB of one row, or 2 KB of each
-  // of the two SwiGLU rows, per warp); 64 registers keep 32 warps per SM
-  constexpr int kLoads = SWI ? 4 : 8;
+  // 16-byte loads per lane in flight per row (5 KB of one row, a whole Phi-2
+  // row, or 2 KB of each of the two SwiGLU rows, per warp); 64 registers keep
+  // 32 warps per SM
+  constexpr int kLoads = SWI ? 4 : 10;
   pdl_wait();  // x and the list may come from the previous grid
   const int lane = threadIdx.x & 31;
   const int gw = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5);
   const int nw = (int)((gridDim.x * blockDim.x) >> 5);
   const int cnt = min(max(*cnt_p, 0), ffn);
-  // start every row this warp will read towards L2 (one bulk prefetch per row,
-  // spread over the lanes), so the rows stream while the first ones are summed
+  // one matrix: start every row this warp will read towards L2 (one bulk
+  // prefetch per row, spread over the lanes), so the rows stream while the
+  // first ones are summed. Measured on B200: with the two SwiGLU rows per
+  // neuron the prefetches cost more than they save (8B shape, keep 0.5: 36.8
+  // against 41.8 us without / with), with one GeLU row they save 0.7-1 us.
   const uint32_t row_bytes = (uint32_t)((long long)d * sizeof(TW));
-  for (int k = gw + lane * nw; k < cnt; k += 32 * nw) {
+  for (int k = gw + lane * nw; !SWI && k < cnt; k += 32 * nw) {
     const int r = idx[k];
-    if (r >= 0 && r < ffn) {
-      prefetch_l2_bulk(WaT + (long long)r * d, row_bytes);
-      if (WbT) prefetch_l2_bulk(WbT + (long long)r * d, row_bytes);
-    }
+    if (r >= 0 && r < ffn) prefetch_l2_bulk(WaT + (long long)r * d, row_bytes);
   }
   for (int k = gw; k < cnt; k += nw) {
     const int r = idx[k];
