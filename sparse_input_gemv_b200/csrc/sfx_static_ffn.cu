@@ -15,9 +15,8 @@
 // the fp32 accumulator is zeroed (cudaMemsetAsync), then
 // static_ffn_kernel (persistent CTAs, programmatic dependent launch): each CTA
 // takes chunks of S whose size it derives from the device-side count so that
-// the chunks spread over all resident CTAs; a chunk's rows of every matrix are
-// bulk-prefetched to L2 at once (they are known before any arithmetic), the dot
-// products run as tensor-core tiles, and the down projection adds 16-byte
+// the chunks spread over all resident CTAs; the dot products run as
+// tensor-core tiles, and the down projection adds 16-byte
 // float4 atomics into the accumulator (the combine order, hence the last bits
 // of y, may vary between runs); then static_ffn_finalize_kernel writes y.
 #include "sfx_common.cuh"
@@ -51,21 +50,11 @@ __global__ void __launch_bounds__(kRowThreads, 2)
   ch = ch < kSfChunkMin ? kSfChunkMin : (ch > kSfChunkMax ? kSfChunkMax : ch);
   const int n_items = (cnt + ch - 1) / ch;
   if ((int)blockIdx.x >= n_items) return;
-  const long long row_bytes = (long long)d * sizeof(TW);
-  const int nmat = WbT ? 3 : 2;
 
-  // every row of an item is known up front: bulk-prefetch them all to L2
-  auto prefetch_item = [&](int it) {
-    const int j0 = it * ch, nj = min(ch, cnt - j0);
-    for (int k = tid; k < nmat * nj; k += kRowThreads) {
-      const int m = k / nj;
-      const int r = idx[j0 + (k - m * nj)];
-      if (r < 0 || r >= ffn) continue;  // reported when the item runs
-      const TW* base = m == 0 ? WaT : (m == 1 ? Wd : WbT);
-      prefetch_l2_bulk(base + (long long)r * d, (uint32_t)row_bytes);
-    }
-  };
-  prefetch_item(blockIdx.x);
+  // No L2 prefetch of the items' rows: measured on B200 at 4 and 16 tokens
+  // (Phi-2 GeLU and 8B-shaped SwiGLU sets, keep 0.3-0.7), bulk-prefetching
+  // every row of the next item cost up to 14 % more than letting the
+  // row-dot loads stream them.
 
   const int xstride = d + kXPad;
   TW* xs = reinterpret_cast<TW*>(s_xraw);
@@ -90,7 +79,6 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       s_bad[tid] = bad;
     }
     __syncthreads();
-    if (it + (int)gridDim.x < n_items) prefetch_item(it + gridDim.x);
     int n_tiles, ksplit;
     auto row_of = [&](int r) { return (long long)s_list[r]; };
     mma_rows(WaT, row_of, nj, d, xs, xstride, B, s_part, &n_tiles, &ksplit);
