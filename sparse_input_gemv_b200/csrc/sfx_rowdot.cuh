@@ -110,16 +110,19 @@ __device__ __forceinline__ float sum_parts(const float (*s_part)[16][kRowTok], i
 
 // acc[tok(t0 + b)] += sum_k v[k][t0 + b] Wd[s_list[k], :] for NTOK tokens, the
 // warps taking (256-column chunk, row phase) tasks; 16-byte atomics into acc.
+// The chunks start at `rot` (mod the chunk count): callers whose items all add
+// into the same token rows at the same time pass the item index, so that their
+// atomics land on different columns.
 template <typename TW, int NTOK>
 __device__ __forceinline__ void down_pass(const TW* __restrict__ Wd, const int* s_list, int na,
                                           const float (*s_v)[kRowTok], int t0, const int* s_tok,
-                                          int d, float* acc_out) {
+                                          int d, float* acc_out, int rot) {
   constexpr int kWarps = kRowThreads / 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nch = (d + 255) / 256;
   const int nsplit = kWarps >= nch ? kWarps / nch : 1;
   for (int task = warp; task < nch * nsplit; task += kWarps) {
-    const int chk = task % nch, par = task / nch;
+    const int chk = (task + rot) % nch, par = task / nch;
     const int col = chk * 256 + lane * 8;
     if (col >= d) continue;
     float acc[NTOK][8];
@@ -165,13 +168,13 @@ __device__ __forceinline__ void down_pass(const TW* __restrict__ Wd, const int* 
 template <typename TW>
 __device__ __forceinline__ void down_all(const TW* __restrict__ Wd, const int* s_list, int na,
                                          const float (*s_v)[kRowTok], int ne, const int* s_tok,
-                                         int d, float* acc_out) {
+                                         int d, float* acc_out, int rot = 0) {
   for (int t0 = 0; t0 < ne && na > 0; t0 += 4) {
     switch (ne - t0 < 4 ? ne - t0 : 4) {
-      case 1: down_pass<TW, 1>(Wd, s_list, na, s_v, t0, s_tok, d, acc_out); break;
-      case 2: down_pass<TW, 2>(Wd, s_list, na, s_v, t0, s_tok, d, acc_out); break;
-      case 3: down_pass<TW, 3>(Wd, s_list, na, s_v, t0, s_tok, d, acc_out); break;
-      default: down_pass<TW, 4>(Wd, s_list, na, s_v, t0, s_tok, d, acc_out); break;
+      case 1: down_pass<TW, 1>(Wd, s_list, na, s_v, t0, s_tok, d, acc_out, rot); break;
+      case 2: down_pass<TW, 2>(Wd, s_list, na, s_v, t0, s_tok, d, acc_out, rot); break;
+      case 3: down_pass<TW, 3>(Wd, s_list, na, s_v, t0, s_tok, d, acc_out, rot); break;
+      default: down_pass<TW, 4>(Wd, s_list, na, s_v, t0, s_tok, d, acc_out, rot); break;
     }
   }
 }

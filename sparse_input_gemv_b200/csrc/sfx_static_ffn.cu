@@ -45,8 +45,12 @@ __global__ void __launch_bounds__(kRowThreads, 2)
   const int tid = threadIdx.x;
   pdl_wait();  // x, the list and the zeroed accumulator come from earlier work on the stream
   const int cnt = min(max(*cnt_p, 0), ffn);
-  // chunk size from the count: about one item per resident CTA, 16..64 neurons
-  int ch = (cnt + (int)gridDim.x - 1) / (int)gridDim.x;
+  // chunk size from the count: the fewest equal rounds of one item per resident
+  // CTA with at most 64 neurons per item (at least 16). Rounding 10035 neurons
+  // on 148 CTAs to 157 items of 64 left 9 CTAs a second item and doubled the
+  // time; 296 items of 34 take two even rounds.
+  const int rounds = max(1, (cnt + (int)gridDim.x * kSfChunkMax - 1) / ((int)gridDim.x * kSfChunkMax));
+  int ch = (cnt + (int)gridDim.x * rounds - 1) / ((int)gridDim.x * rounds);
   ch = ch < kSfChunkMin ? kSfChunkMin : (ch > kSfChunkMax ? kSfChunkMax : ch);
   const int n_items = (cnt + ch - 1) / ch;
   if ((int)blockIdx.x >= n_items) return;
@@ -101,7 +105,7 @@ __global__ void __launch_bounds__(kRowThreads, 2)
       s_v[r][t] = s_bad[r] ? 0.f : v;
     }
     __syncthreads();
-    down_all(Wd, s_list, nj, s_v, B, s_tok, d, acc);
+    down_all(Wd, s_list, nj, s_v, B, s_tok, d, acc, it);  // all items share the tokens
   }
 }
 
