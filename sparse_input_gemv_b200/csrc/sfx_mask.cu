@@ -132,8 +132,13 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
   __shared__ int s_w[kMaskWarps + 1];
   __shared__ uint32_t s_prefix;
   __shared__ uint32_t s_remaining;
+  __shared__ int s_whole;
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
+  // h comes from the previous kernel (launched as its programmatic dependent);
+  // the next kernel may start its CTAs now: it waits for this grid's results
+  pdl_wait();
+  pdl_launch_dependents();
   const int kpt = (K + kMaskThreads - 1) / kMaskThreads;
   const TX* xb = x + (long long)b * K;
   const float* gb = g + (long long)b * K;
@@ -211,25 +216,32 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
       if (c < remaining && remaining <= c + h1) {
         s_prefix = prefix | ((uint32_t)(2 * tid + 1) << shift);
         s_remaining = remaining - c;
+        s_whole = remaining - c == h1;
       }
       c += h1;
       if (c < remaining && remaining <= c + h0) {
         s_prefix = prefix | ((uint32_t)(2 * tid) << shift);
         s_remaining = remaining - c;
+        s_whole = remaining - c == h0;
       }
       __syncthreads();
       prefix = s_prefix;
       remaining = s_remaining;
       pmask |= dmask << shift;
+      // the bin holding the k-th key is kept whole: every key above it and
+      // every key in it are the top k, so the digits left decide nothing
+      if (s_whole) break;
     }
   }
-  const uint32_t T = prefix;  // k-th largest key; `remaining` of the keys equal to T are kept
+  // T: the k-th largest key on the digits examined (pmask); `remaining` of the
+  // keys equal to T on those digits are kept (all of them after an early stop)
+  const uint32_t T = prefix;
   // ties before this thread, then this thread's kept count and output position
   int n_gt = 0, n_eq = 0;
 #pragma unroll
   for (int j = 0; j < KPT; ++j) {
-    n_gt += (j < nt && k > 0 && key[j] > T);
-    n_eq += (j < nt && k > 0 && key[j] == T);
+    n_gt += (j < nt && k > 0 && (key[j] & pmask) > T);
+    n_eq += (j < nt && k > 0 && (key[j] & pmask) == T);
   }
   // one scan of (n_gt, n_eq) packed in 16-bit halves (K <= 32768): the threads
   // before this one keep all their larger keys and the first `remaining` of
@@ -253,9 +265,9 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
       const int i = e0 + j;
       bool keep = false;
       if (k > 0) {
-        if (key[j] > T) {
+        if ((key[j] & pmask) > T) {
           keep = true;
-        } else if (key[j] == T) {
+        } else if ((key[j] & pmask) == T) {
           keep = eq_seen < eq_keep;
           ++eq_seen;
         }
@@ -328,9 +340,21 @@ template <typename TX, int KPT>
 static int launch_gxo_k(const void* x, const float* g, int B, int K, int k, int corrected,
                         uint32_t* bitmap, int32_t* idx, int32_t* cnt, cudaStream_t s) {
   const size_t smem = (size_t)((K + 31) / 32) * 4;  // the bitmap (<= 4 KB)
-  topk_gxo_kernel<TX, KPT><<<B, kMaskThreads, smem, s>>>(reinterpret_cast<const TX*>(x), g, K, k,
-                                                          corrected, bitmap, idx, cnt);
-  return cudaGetLastError() == cudaSuccess ? SFX_OK : SFX_ERR_CUDA;
+  // a programmatic dependent launch: the kernel waits for its inputs itself
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)B, 1, 1);
+  cfg.blockDim = dim3(kMaskThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, topk_gxo_kernel<TX, KPT>, reinterpret_cast<const TX*>(x), g, K,
+                            k, corrected, bitmap, idx, cnt) == cudaSuccess
+             ? SFX_OK
+             : SFX_ERR_CUDA;
 }
 
 // keys per thread in registers: K <= 1024 KPT (K <= 32768)

@@ -180,6 +180,32 @@ def test_topk_gxo_ties_go_to_lower_index():
             assert np.array_equal(out["idx"][b, :k].cpu().numpy(), O.compact(m)[0]), (k, b)
 
 
+def test_topk_gxo_stops_after_any_digit_pass():
+    # The radix select stops once the bin holding the k-th key is kept whole.
+    # 120 scores 2^-j (one key per 11-bit top digit) over zeros stop after the
+    # first pass for k <= 120 and tie-break the zeros after three passes above;
+    # consecutive floats 1 + j ulp share their top 22 bits in runs of 1024 and
+    # stop after two passes or three; a mix of powers and ulps stops after two
+    # or three depending on k. Each case against the oracle, bit for bit.
+    K = 4096
+    j = np.arange(K)
+    cases = {
+        "powers": np.where(j < 120, np.ldexp(1.0, -np.minimum(j, 119)), 0.0).astype(np.float32),
+        "ulps": (np.float32(1.0) + j.astype(np.float32) * np.float32(2.0 ** -23)).astype(np.float32),
+        "mixed": np.where(j % 2 == 0, np.ldexp(1.0, -(j % 60)),
+                          1.0 + j * 2.0 ** -23).astype(np.float32),
+    }
+    for name, hv in cases.items():
+        h = torch.from_numpy(np.stack([hv, hv[::-1].copy()]))
+        g = torch.ones((2, K), dtype=torch.float32)
+        for k in (1, 5, 120, 121, 511, 1024, 1025, 2048, 4095):
+            out = sb.sfx_mask_compact(dev(h), sb.SFX_SEL_TOPK_GXO, k=k, score_l=dev(g))
+            for b in range(2):
+                m = O.topk_mask(O.gxo_score(h.numpy()[b], g.numpy()[b]), k)
+                assert int(out["cnt"][b]) == k
+                assert np.array_equal(out["idx"][b, :k].cpu().numpy(), O.compact(m)[0]), (name, k, b)
+
+
 @pytest.mark.parametrize("lam,K,keep", [(0.5, 10240, 0.5), (0.0, 2000, 0.3), (1.0, 2000, 0.7),
                                         (0.3, 999, 0.5)])
 def test_glass_bit_exact(lam, K, keep):
