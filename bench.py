@@ -411,30 +411,33 @@ def bench_other_workloads(stream, dev, which=OTHER_WORKLOADS):
         import ctypes
         P = lambda tns: ctypes.c_void_p(tns.data_ptr())
 
-        def select_gxo(k, sel=sb.SFX_SEL_TOPK_GXO):
+        def select_gxo(k, sel=sb.SFX_SEL_TOPK_GXO, with_idx=False):
             lib.sfx_mask_compact(P(h), sb.SFX_F32, 1, f, sel, 0.0, k, P(g), None, 0.5,
-                                 P(bitmap), P(idx), P(cnt), None, None, P(ws.buf), ws.buf.numel(),
+                                 P(bitmap), P(idx) if with_idx else None, P(cnt), None, None,
+                                 P(ws.buf), ws.buf.numel(),
                                  ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+
+        def gxo_steps(k, sel, with_idx):
+            # up GEMV (GeLU) -> top-k select -> down GEMV on the select's bitmap
+            # (or on its ascending index list)
+            steps = []
+            for c in range(n):
+                def step(c=c):
+                    sb.sfx_sparse_gemv(x, W1[c], flags=sb.SFX_FLAG_GELU, y=h, ws=ws)
+                    select_gxo(k, sel, with_idx)
+                    if with_idx:
+                        sb.sfx_sparse_gemv(h[0], W2[c], idx=idx[0], cnt=cnt, y=y[0], ws=ws)
+                    else:
+                        sb.sfx_sparse_gemv_mask(h[0], W2[c], bitmap[0], y=y[0], ws=ws)
+                steps.append(step)
+            return steps
         phi = {}
         for keep in (0.3, 0.5, 0.7):
             k = int(keep * f + 0.5)
-            steps = []
-            for c in range(n):
-                def step(c=c, k=k):
-                    sb.sfx_sparse_gemv(x, W1[c], flags=sb.SFX_FLAG_GELU, y=h, ws=ws)
-                    select_gxo(k)
-                    sb.sfx_sparse_gemv(h[0], W2[c], idx=idx[0], cnt=cnt, y=y[0], ws=ws)
-                steps.append(step)
-            us = graph_us(steps, stream)
+            us = graph_us(gxo_steps(k, sb.SFX_SEL_TOPK_GXO, False), stream)
+            us_idx = graph_us(gxo_steps(k, sb.SFX_SEL_TOPK_GXO, True), stream)
             # the same step with the corrected GxO score (ATTR "correction term")
-            csteps = []
-            for c in range(n):
-                def cstep(c=c, k=k):
-                    sb.sfx_sparse_gemv(x, W1[c], flags=sb.SFX_FLAG_GELU, y=h, ws=ws)
-                    select_gxo(k, sb.SFX_SEL_TOPK_CGXO)
-                    sb.sfx_sparse_gemv(h[0], W2[c], idx=idx[0], cnt=cnt, y=y[0], ws=ws)
-                csteps.append(cstep)
-            us_c = graph_us(csteps, stream)
+            us_c = graph_us(gxo_steps(k, sb.SFX_SEL_TOPK_CGXO, False), stream)
             nbytes = d * f * 2 + k * d * 2 + d * 2 + f * 4 * 3 + d * 2
             # GLASS: the mask is fixed after prefill, so a decode step is up + down only
             sb.sfx_mask_compact(None, sb.SFX_SEL_TOPK_GLASS, k=k, score_l=sl, score_g=sgl, lam=0.5, ws=ws)
@@ -450,6 +453,7 @@ def bench_other_workloads(stream, dev, which=OTHER_WORKLOADS):
                                 for c in range(n)], stream)
             bytes_both = 2 * k * d * 2 + 2 * d * 2
             phi[f"keep{int(keep * 100)}"] = {"us_gxo": us, "us_corrected_gxo": us_c,
+                                             "us_gxo_index_list": us_idx,
                                              "us_glass_static_mask": us_gl,
                                              "us_glass_both_projections": us_both,
                                              "gbs_glass_both_projections":

@@ -281,6 +281,33 @@ int sfx_sparse_gemv(const void* x, int xdt, int B, int K, const void* W, int wdt
                     void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------
+ * a5. Input-sparse GEMV on a given mask       [TEAL] slide 11, [ATTR]
+ *
+ * y[b, n] = sum_{i : m_bi} x[b, i] * W[i, n], accumulated in fp32, with the
+ * mask given as a bitmap in the layout sfx_mask_compact and the fused mask
+ * outputs write (bit i % 32 of word i / 32 of row b; bits at or past K are
+ * ignored). Every CTA reads the mask words of its K-slice in the same round
+ * trip as x and builds its active list itself, so a selection such as the
+ * GxO top-k reaches the product as a bitmap, with no index list in between.
+ * Rows are fetched once for the batch and each token keeps its own rows,
+ * unless SFX_FLAG_UNION_MASK makes every token keep the rows any token keeps
+ * (each with its own x). Every B runs on the CUDA-core kernel; the K-split
+ * sums are added in a fixed order (same bits per call). Epilogue flags, dtypes,
+ * workspace and limits as sfx_sparse_gemv.
+ *
+ *  x     (dev) [B x K] of dtype xdt (f16, bf16, f32); xdt == wdt or f32
+ *  W     (dev) [K x N] of dtype wdt (f16, bf16), row-major, 16-byte aligned
+ *  mask  (dev) [B x ceil(K/32)] uint32
+ *  y     (dev) [B x N] of dtype ydt ([B x N/2] fp32 with SFX_FLAG_SWIGLU)
+ *  ws    (dev) sfx_workspace_bytes(SFX_OP_SPARSE_GEMV, B, K, N, xdt)
+ * Returns SFX_ERR_ARG for a NULL mask or the arguments sfx_sparse_gemv
+ * rejects.
+ * ---------------------------------------------------------------------- */
+int sfx_sparse_gemv_mask(const void* x, int xdt, int B, int K, const void* W, int wdt, int N,
+                         const uint32_t* mask, void* y, int ydt, int flags,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------
  * sfx_sparse_gemv without a workspace. The source pages have no counterpart:
  * this entry point exists for callers, not for the method.
  *

@@ -52,6 +52,7 @@ _SIGS = {
                              _SZ, _VP]),
     "sfx_sparse_gemv_noalloc": (_I, [_VP, _I, _I, _I, _VP, _I, _I, _F, _VP, _VP, _VP, _I, _I,
                                      _VP]),
+    "sfx_sparse_gemv_mask": (_I, [_VP, _I, _I, _I, _VP, _I, _I, _VP, _VP, _I, _I, _VP, _SZ, _VP]),
     "sfx_sparse_ffn_swiglu": (_I, [_VP, _I, _I, _I, _I, _VP, _VP, _F, _F, _VP, _I, _VP, _VP, _VP,
                                    _I, _VP, _SZ, _VP]),
     "sfx_pack_gate_up": (_I, [_VP, _VP, _I, _I, _I, _VP, _VP]),
@@ -176,8 +177,10 @@ def sfx_calibrate_thresholds(calib: torch.Tensor, sparsities, ws: Workspace | No
 
 
 def sfx_mask_compact(x=None, sel=SFX_SEL_THRESHOLD, t=0.0, k=0, score_l=None, score_g=None,
-                     lam=0.5, want_union=False, ws: Workspace | None = None, K=None, B=None):
-    """Masks, ascending index lists and counts. Returns dict(bitmap, idx, cnt[, union_idx, union_cnt])."""
+                     lam=0.5, want_union=False, ws: Workspace | None = None, K=None, B=None,
+                     want_idx=True):
+    """Masks, ascending index lists and counts. Returns dict(bitmap, idx, cnt[, union_idx, union_cnt]);
+    idx is None with want_idx=False (the bitmap and counts only)."""
     ref = x if x is not None else score_l
     _need_cuda(x, score_l, score_g)
     if ref.dim() == 1:
@@ -188,7 +191,7 @@ def sfx_mask_compact(x=None, sel=SFX_SEL_THRESHOLD, t=0.0, k=0, score_l=None, sc
     dev = ref.device
     words = (K + 31) // 32
     bitmap = torch.zeros((B, words), dtype=torch.int32, device=dev)
-    idx = torch.full((B, K), -1, dtype=torch.int32, device=dev)
+    idx = torch.full((B, K), -1, dtype=torch.int32, device=dev) if want_idx else None
     cnt = torch.zeros((B,), dtype=torch.int32, device=dev)
     uidx = torch.full((K,), -1, dtype=torch.int32, device=dev) if want_union else None
     ucnt = torch.zeros((1,), dtype=torch.int32, device=dev) if want_union else None
@@ -228,6 +231,33 @@ def sfx_sparse_gemv(x, W, t=-math.inf, idx=None, cnt=None, out_dtype=None, flags
         _ptr(y), _DT[y.dtype], int(flags), _ptr(bitmap), _ptr(buf), buf.numel(), _stream(stream)))
     y_out = y[0] if squeeze else y
     return (y_out, bitmap) if want_bitmap else y_out
+
+
+def sfx_sparse_gemv_mask(x, W, mask, out_dtype=None, flags=0, y=None,
+                         ws: Workspace | None = None, stream=None):
+    """y = (x * m) W for a given mask bitmap m ([B x ceil(K/32)] int32/uint32 words)."""
+    squeeze = x.dim() == 1
+    x2 = x[None] if squeeze else x
+    mask2 = mask[None] if mask.dim() == 1 else mask
+    _need_cuda(x2, W, mask2)
+    B, K = x2.shape
+    K2, N = W.shape
+    if K2 != K:
+        raise ValueError("x and W disagree on K")
+    if tuple(mask2.shape) != (B, (K + 31) // 32) or mask2.element_size() != 4 \
+            or not mask2.is_contiguous():
+        raise ValueError("mask must be a contiguous [B x ceil(K/32)] tensor of 32-bit words")
+    out_dtype = out_dtype or W.dtype
+    if flags & SFX_FLAG_SWIGLU:
+        out_dtype = torch.float32
+    if y is None:
+        ncol = N // 2 if flags & SFX_FLAG_SWIGLU else N
+        y = torch.empty((B, ncol), dtype=out_dtype, device=W.device)
+    ws, buf = _ws(ws, sfx_workspace_bytes(SFX_OP_SPARSE_GEMV, B, K, N, _DT[x2.dtype]), W.device)
+    _check("sfx_sparse_gemv_mask", load().sfx_sparse_gemv_mask(
+        _ptr(x2), _DT[x2.dtype], B, K, _ptr(W), _DT[W.dtype], N, _ptr(mask2), _ptr(y),
+        _DT[y.dtype], int(flags), _ptr(buf), buf.numel(), _stream(stream)))
+    return y[0] if squeeze else y
 
 
 def sfx_sparse_gemv_noalloc(x, W, t=-math.inf, idx=None, cnt=None, out_dtype=None, flags=0,

@@ -290,6 +290,40 @@ int sfx_sparse_gemv(const void* x, int xdt, int B, int K, const void* W, int wdt
   return launch_sparse_gemv(wdt, xdt, plan, a, as_stream(stream), false);
 }
 
+int sfx_sparse_gemv_mask(const void* x, int xdt, int B, int K, const void* W, int wdt, int N,
+                         const uint32_t* mask, void* y, int ydt, int flags, void* ws,
+                         size_t ws_bytes, void* stream) {
+  if (!x || !W || !y || !mask || B < 1 || B > 16 || K < 1 || N < 8) return SFX_ERR_ARG;
+  if ((flags & SFX_FLAG_GELU) && (flags & SFX_FLAG_GELU_TANH)) return SFX_ERR_ARG;
+  if ((flags & SFX_FLAG_SWIGLU) && (flags & (SFX_FLAG_GELU | SFX_FLAG_GELU_TANH))) return SFX_ERR_ARG;
+  if (!(wdt == SFX_F16 || wdt == SFX_BF16) || !(xdt == wdt || xdt == SFX_F32) || !valid_dtype(ydt))
+    return SFX_ERR_DTYPE;
+  if ((flags & SFX_FLAG_SWIGLU) && ydt != SFX_F32) return SFX_ERR_DTYPE;
+  if (N % 8 != 0 || !aligned16(W)) return SFX_ERR_ALIGN;
+  if (!ws || ws_bytes < sfx_workspace_bytes(SFX_OP_SPARSE_GEMV, B, K, N, xdt, 0, 0))
+    return SFX_ERR_WORKSPACE;
+  GemvArgs a = {};
+  a.x = x;
+  a.W = W;
+  a.y = y;
+  a.mask_in = mask;
+  a.status = reinterpret_cast<unsigned*>(ws);
+  carve_gemv(ws, reinterpret_cast<unsigned char*>(ws) + kWsHeader, a);
+  a.K = K;
+  a.N = N;
+  a.B = B;
+  a.ydt = ydt;
+  a.epi = (flags & SFX_FLAG_SWIGLU) ? EPI_SWIGLU
+        : (flags & SFX_FLAG_GELU)   ? EPI_GELU
+        : (flags & SFX_FLAG_GELU_TANH) ? EPI_GELU_TANH
+                                       : EPI_NONE;
+  a.union_mask = (flags & SFX_FLAG_UNION_MASK) ? 1 : 0;
+  a.no_tc = 1;
+  a.t = 0.f;
+  a.wait_ns = wait_limit_ns();
+  return launch_sparse_gemv(wdt, xdt, plan_gemv(K, N, B, false), a, as_stream(stream), false);
+}
+
 int sfx_sparse_ffn_swiglu(const void* x, int dt, int B, int d, int ffn, const void* W_gu,
                           const void* W_d, float t_in, float t_h, void* y, int ydt, float* h_out,
                           uint32_t* bitmap_x_out, uint32_t* bitmap_h_out, int flags, void* ws,

@@ -118,7 +118,7 @@ int launch_sparse_gemv(int wdt, int xdt, const GemvPlan& p, GemvArgs a, cudaStre
   const bool pdl = true;
   // a batch of union_min_batch() .. 16 tokens in threshold mode: the union
   // tile on the tensor cores
-  if (a.B >= union_min_batch() && a.idx == nullptr && !a.no_tc)
+  if (a.B >= union_min_batch() && a.idx == nullptr && a.mask_in == nullptr && !a.no_tc)
     return launch_union_tc(wdt, xdt, plan_union_tc(a.K, a.N), a, s);
   if (p.col_tiles > kCounterSlots) return SFX_ERR_UNSUPPORTED;
   a.S = p.S;

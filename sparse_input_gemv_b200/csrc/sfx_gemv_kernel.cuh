@@ -154,16 +154,25 @@ __global__ void __launch_bounds__(gemv_threads(BMAX), (BMAX <= 2) ? 2 : 1)
     const TX* xp = reinterpret_cast<const TX*>(a.x);
     const bool vec = (reinterpret_cast<uintptr_t>(a.x) % (4 * sizeof(TX))) == 0 &&
                      (a.B == 1 || (a.K & 3) == 0);
+    // a given mask: the four rows of a group share one word (i % 4 == 0),
+    // loaded together with x
+    const uint32_t* mk = a.mask_in;
+    const long long mwords = (a.K + 31) >> 5;
     float xv[4 * KG][BMAX];
     unsigned act = 0;
 #pragma unroll
     for (int g = 0; g < KG; ++g) {
       const long long i = i0 + 4 * g;
       if (4 * g < r && i < k1) {
+        unsigned mw[BMAX];
 #pragma unroll
         for (int b = 0; b < BMAX; ++b) {
           float v[4] = {0.f, 0.f, 0.f, 0.f};
-          if (b < a.B) load4(xp + (long long)b * a.K, i, k1, vec, v);
+          mw[b] = 0u;
+          if (b < a.B) {
+            load4(xp + (long long)b * a.K, i, k1, vec, v);
+            if (mk != nullptr) mw[b] = __ldg(mk + (long long)b * mwords + (i >> 5)) >> (i & 31);
+          }
 #pragma unroll
           for (int j = 0; j < 4; ++j) xv[4 * g + j][b] = v[j];
         }
@@ -172,7 +181,9 @@ __global__ void __launch_bounds__(gemv_threads(BMAX), (BMAX <= 2) ? 2 : 1)
           bool any = false;
 #pragma unroll
           for (int b = 0; b < BMAX; ++b) {
-            const bool m = b < a.B && i + j < k1 && fabsf(xv[4 * g + j][b]) > a.t;
+            const bool m = b < a.B && i + j < k1 &&
+                           (mk != nullptr ? ((mw[b] >> j) & 1u) != 0u
+                                          : fabsf(xv[4 * g + j][b]) > a.t);
             any |= m;
             if (!m && !a.union_mask) xv[4 * g + j][b] = 0.f;
           }

@@ -25,6 +25,7 @@ struct GemvArgs {
   const void* W;          // [K x N] weights, dtype wdt
   void* y;                // [B x N] (or [B x N/2] fp32 h for EPI_SWIGLU)
   const int32_t* idx;     // optional active list (B == 1)
+  const uint32_t* mask_in;  // optional mask bitmap [B x ceil(K/32)] instead of |x| > t
   const int32_t* cnt;     // device count of idx
   uint32_t* bitmap_out;   // optional fused-mask output [B x ceil(K/32)]
   float* partials;        // [S x B x N] split-K partial sums (workspace)

@@ -189,6 +189,7 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
   for (int w = tid; w < words; w += kMaskThreads) s_bits[w] = 0u;
 
   uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k;
+  int whole = 1;  // the kept keys are all keys >= T on the digits examined
   // each thread owns bins 2 tid and 2 tid + 1: it zeroes them, and after a pass
   // reads and re-zeroes them itself
   hist[2 * tid] = 0u;
@@ -230,7 +231,8 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
       pmask |= dmask << shift;
       // the bin holding the k-th key is kept whole: every key above it and
       // every key in it are the top k, so the digits left decide nothing
-      if (s_whole) break;
+      whole = s_whole;
+      if (whole) break;
     }
   }
   // T: the k-th largest key on the digits examined (pmask); `remaining` of the
@@ -245,16 +247,19 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
   }
   // one scan of (n_gt, n_eq) packed in 16-bit halves (K <= 32768): the threads
   // before this one keep all their larger keys and the first `remaining` of
-  // the ties, so this thread writes from gt_before + min(eq_before, remaining)
-  int packed_tot;
-  const int packed = block_excl_scan((n_gt << 16) | n_eq, s_w, &packed_tot);
-  const int gt_before = packed >> 16, eq_before = packed & 0xffff;
-  int eq_keep = (int)remaining - eq_before;
-  eq_keep = eq_keep < 0 ? 0 : (eq_keep > n_eq ? n_eq : eq_keep);
-  const int pos0 = gt_before + (eq_before < (int)remaining ? eq_before : (int)remaining);
-  const int tot = (packed_tot >> 16) + ((packed_tot & 0xffff) < (int)remaining
-                                            ? (packed_tot & 0xffff)
-                                            : (int)remaining);
+  // the ties, so this thread writes from gt_before + min(eq_before, remaining).
+  // Without an index list and with every tie kept, no offset is needed.
+  int eq_keep = n_eq, pos0 = 0, tot = k;
+  if (idx != nullptr || !whole) {
+    int packed_tot;
+    const int packed = block_excl_scan((n_gt << 16) | n_eq, s_w, &packed_tot);
+    const int gt_before = packed >> 16, eq_before = packed & 0xffff;
+    eq_keep = (int)remaining - eq_before;
+    eq_keep = eq_keep < 0 ? 0 : (eq_keep > n_eq ? n_eq : eq_keep);
+    pos0 = gt_before + (eq_before < (int)remaining ? eq_before : (int)remaining);
+    tot = (packed_tot >> 16) + ((packed_tot & 0xffff) < (int)remaining ? (packed_tot & 0xffff)
+                                                                       : (int)remaining);
+  }
   int32_t* out = idx ? idx + (long long)b * K : nullptr;
   int pos = pos0, eq_seen = 0;
   uint32_t word = 0;  // bits of the current bitmap word gathered by this thread

@@ -321,6 +321,58 @@ def test_gemv_bad_index_is_skipped_and_flagged():
     assert_close(to64(y), O.round_to(O.masked_gemv(to64(x), m, to64(W))[0], "f32"), "bad idx")
 
 
+# ---------------------------------------------------------------- GEMV on a given mask
+
+@pytest.mark.parametrize("B,K,N,dens,wdt,xdt,flags", [
+    (1, 10240, 2560, 0.3, "f16", "f32", 0),          # the Phi-2 down shape, fp32 h
+    (2, 1000, 264, 0.5, "bf16", "bf16", 0),           # ragged K (bits past K set) and N
+    (5, 4096, 1024, 0.2, "bf16", "bf16", 0),          # 5 tokens stay on CUDA cores
+    (3, 2560, 512, 0.4, "f16", "f16", "union"),       # every token on the union's rows
+    (1, 777, 128, 0.6, "bf16", "f32", "gelu"),        # epilogue
+    (16, 4000, 4096, 0.1, "bf16", "bf16", 0),
+])
+def test_gemv_given_mask_matches_oracle(B, K, N, dens, wdt, xdt, flags):
+    rng = np.random.default_rng(K + B)
+    m = rng.random((B, K)) < dens
+    words = pack_bitmap(m)
+    if K % 32:
+        words[:, -1] |= np.int32(-1 << (K % 32))  # bits past K must be ignored
+    x = synth.eval_draw("given-mask", f"x{K}", B, K, xdt)
+    W = weights(K, N, f"given-mask-{K}", wdt)
+    fl = {0: 0, "union": sb.SFX_FLAG_UNION_MASK, "gelu": sb.SFX_FLAG_GELU}[flags]
+    y = sb.sfx_sparse_gemv_mask(dev(x), dev(W), dev(torch.from_numpy(words)),
+                                out_dtype=torch.float32, flags=fl)
+    mm = np.broadcast_to(O.union_mask(m), (B, K)) if flags == "union" else m
+    want = O.masked_gemv(to64(x), mm, to64(W))
+    if flags == "gelu":
+        want = O.gelu_erf(want)
+    assert_close(to64(y), O.round_to(want, "f32"), f"given mask B={B} K={K}")
+
+
+def test_gemv_given_mask_empty_and_full():
+    B, K, N = 2, 3000, 256
+    x = synth.eval_draw("given-mask-ef", "x", B, K, "bf16")
+    W = weights(K, N, "given-mask-ef", "bf16")
+    zero = torch.zeros((B, (K + 31) // 32), dtype=torch.int32)
+    y0 = sb.sfx_sparse_gemv_mask(dev(x), dev(W), dev(zero), out_dtype=torch.float32)
+    assert torch.count_nonzero(y0) == 0
+    full = torch.full((B, (K + 31) // 32), -1, dtype=torch.int32)
+    y1 = sb.sfx_sparse_gemv_mask(dev(x), dev(W), dev(full), out_dtype=torch.float32)
+    y_dense = sb.sfx_sparse_gemv(dev(x), dev(W), t=-math.inf, out_dtype=torch.float32,
+                                 flags=sb.SFX_FLAG_CUDA_CORES)
+    assert torch.equal(y1, y_dense)  # same plan, same split order: the same bits
+
+
+def test_gemv_given_mask_equals_its_own_threshold():
+    # the fused |x| > t mask, written out and passed back in, gives the same bits
+    B, K, N = 2, 8192, 2048
+    x = dev(synth.eval_draw("given-mask-t", "x", B, K, "bf16"))
+    W = dev(weights(K, N, "given-mask-t", "bf16"))
+    y_t, bm = sb.sfx_sparse_gemv(x, W, t=0.8, out_dtype=torch.float32, want_bitmap=True)
+    y_m = sb.sfx_sparse_gemv_mask(x, W, bm, out_dtype=torch.float32)
+    assert torch.equal(y_t, y_m)
+
+
 # ---------------------------------------------------------------- SwiGLU FFN
 
 def ffn_case(B, d, ffn, p, dtype="bf16", seed="ffn"):
@@ -489,11 +541,15 @@ def test_ffn_swiglu_llama3_70b_full_size_sampled(B):
 
 # ---------------------------------------------------------------- Phi-2 chain end to end
 
-@pytest.mark.parametrize("keep,sel", [(0.3, "gxo"), (0.5, "gxo"), (0.7, "gxo"), (0.3, "cgxo")])
-def test_phi2_gelu_ffn_chain_end_to_end(keep, sel):
+@pytest.mark.parametrize("keep,sel,path", [(0.3, "gxo", "idx"), (0.5, "gxo", "idx"),
+                                           (0.7, "gxo", "idx"), (0.3, "cgxo", "idx"),
+                                           (0.3, "gxo", "bitmap"), (0.7, "gxo", "bitmap"),
+                                           (0.5, "cgxo", "bitmap")])
+def test_phi2_gelu_ffn_chain_end_to_end(keep, sel, path):
     # Phi-2-shaped GeLU FFN at batch 1, fp16: the dense up GEMV with the GeLU
     # epilogue, the GxO (or corrected GxO) top-k on the GPU's own h, then the
-    # index-list down GEMV -- all three on the GPU, compared with the oracle's
+    # down GEMV on its index list or on its bitmap (path) -- all three on the
+    # GPU, compared with the oracle's
     # own chain (fp64 h, its own top-k). The kept set may differ only where the
     # fp32 and fp64 scores straddle the k-th score ("Attribution-based Sparse
     # Activation in Large Language Models", "implementation": top fraction per
@@ -506,16 +562,22 @@ def test_phi2_gelu_ffn_chain_end_to_end(keep, sel):
     k = O.keep_count(keep, f)
     h_gpu = sb.sfx_sparse_gemv(dev(x), dev(W1), flags=sb.SFX_FLAG_GELU, out_dtype=torch.float32)
     mode = sb.SFX_SEL_TOPK_GXO if sel == "gxo" else sb.SFX_SEL_TOPK_CGXO
-    s = sb.sfx_mask_compact(h_gpu[None], mode, k=k, score_l=dev(g)[None])
-    y = sb.sfx_sparse_gemv(h_gpu, dev(W2), idx=s["idx"][0], cnt=s["cnt"], out_dtype=torch.float16)
+    s = sb.sfx_mask_compact(h_gpu[None], mode, k=k, score_l=dev(g)[None],
+                            want_idx=(path == "idx"))
+    if path == "idx":
+        y = sb.sfx_sparse_gemv(h_gpu, dev(W2), idx=s["idx"][0], cnt=s["cnt"],
+                               out_dtype=torch.float16)
+    else:
+        y = sb.sfx_sparse_gemv_mask(h_gpu, dev(W2), s["bitmap"][0], out_dtype=torch.float16)
     # the oracle's chain on the same x, W1, g, W2
     h = O.gelu_erf(to64(x) @ to64(W1))
     h32 = h.astype(np.float32)
     score = O.gxo_score(g.numpy(), h32) if sel == "gxo" else O.corrected_gxo_score_f32(g.numpy(), h32)
     m = O.topk_mask(score, k)
-    got = np.zeros(f, bool)
-    got[s["idx"][0, :int(s["cnt"][0])].cpu().numpy()] = True
-    assert int(s["cnt"][0]) == k
+    got = np.unpackbits(s["bitmap"][0].cpu().numpy().view(np.uint8), bitorder="little")[:f] > 0
+    if path == "idx":
+        assert np.array_equal(np.flatnonzero(got), s["idx"][0, :int(s["cnt"][0])].cpu().numpy())
+    assert int(s["cnt"][0]) == k and int(got.sum()) == k
     flips = int(np.count_nonzero(got != m))
     assert flips <= 4, flips
     assert_close(to64(h_gpu), O.round_to(h, "f32"), "h")
