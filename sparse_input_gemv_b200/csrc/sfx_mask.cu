@@ -127,29 +127,31 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
                                                                 int K, int k, int corrected,
                                                                 uint32_t* bitmap, int32_t* idx,
                                                                 int32_t* cnt) {
-  extern __shared__ uint32_t s_bits[];  // the bitmap [ceil(K / 32)]
   __shared__ uint32_t hist[kTopkBins];
   __shared__ int s_w[kMaskWarps + 1];
   __shared__ uint32_t s_prefix;
   __shared__ uint32_t s_remaining;
   __shared__ int s_whole;
   const int b = blockIdx.x;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   // h comes from the previous kernel (launched as its programmatic dependent);
   // the next kernel may start its CTAs now: it waits for this grid's results
   pdl_wait();
   pdl_launch_dependents();
+  // Warp w owns the span of 32 kpt elements starting at 32 kpt w, lane-major:
+  // its slot j holds element 32 kpt w + 32 j + lane. Every load is coalesced,
+  // and slot j of a warp is one 32-bit word of the bitmap.
   const int kpt = (K + kMaskThreads - 1) / kMaskThreads;
+  const int base = 32 * kpt * warp;
   const TX* xb = x + (long long)b * K;
   const float* gb = g + (long long)b * K;
-  const int e0 = tid * kpt;
-  const int nt = K - e0 < 0 ? 0 : (K - e0 < kpt ? K - e0 : kpt);  // this thread's elements
-  // this thread's inputs (a contiguous run: its lines are shared through L1)
   float xv[KPT], gv[KPT];
 #pragma unroll
   for (int j = 0; j < KPT; ++j) {
-    xv[j] = j < nt ? to_f32(xb[e0 + j]) : 0.f;
-    gv[j] = j < nt ? gb[e0 + j] : 0.f;
+    const int e = base + 32 * j + lane;
+    const bool ok = j < kpt && e < K;
+    xv[j] = ok ? to_f32(xb[e]) : 0.f;
+    gv[j] = ok ? gb[e] : 0.f;
   }
   // corrected GxO: n / 2 with n = fl32(sqrt(sum g^2)), the squares exact in
   // double and summed in double (a fixed order: per thread, then warp and
@@ -162,7 +164,7 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
     for (int j = 0; j < KPT; ++j) ss += (double)gv[j] * (double)gv[j];
 #pragma unroll
     for (int o = 16; o; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    if ((tid & 31) == 0) s_d[tid >> 5] = ss;
+    if (lane == 0) s_d[warp] = ss;
     __syncthreads();
     if (tid < 32) {
       double v = s_d[tid];
@@ -174,8 +176,10 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
     half_n = __double2float_rn(sqrt(s_d[0])) * 0.5f;  // exact halving
   }
   uint32_t key[KPT];
+  unsigned valid = 0;  // slots that hold an element
 #pragma unroll
   for (int j = 0; j < KPT; ++j) {
+    if (j < kpt && base + 32 * j + lane < K) valid |= 1u << j;
     if (corrected) {
       // signed score -> unsigned key in the same order
       const float sc = __fadd_rn(__fmul_rn(xv[j], gv[j]), __fmul_rn(fabsf(xv[j]), half_n));
@@ -185,11 +189,8 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
       key[j] = __float_as_uint(fabsf(__fmul_rn(xv[j], gv[j])));
     }
   }
-  const int words = (K + 31) >> 5;
-  for (int w = tid; w < words; w += kMaskThreads) s_bits[w] = 0u;
 
   uint32_t prefix = 0, pmask = 0, remaining = (uint32_t)k;
-  int whole = 1;  // the kept keys are all keys >= T on the digits examined
   // each thread owns bins 2 tid and 2 tid + 1: it zeroes them, and after a pass
   // reads and re-zeroes them itself
   hist[2 * tid] = 0u;
@@ -204,7 +205,8 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
       __syncthreads();  // zeroed bins (or the previous selection) visible
 #pragma unroll
       for (int j = 0; j < KPT; ++j)
-        if (j < nt && (key[j] & pmask) == prefix) atomicAdd(&hist[(key[j] >> shift) & dmask], 1u);
+        if (((valid >> j) & 1u) && (key[j] & pmask) == prefix)
+          atomicAdd(&hist[(key[j] >> shift) & dmask], 1u);
       __syncthreads();
       // keys in bins above this thread's two: total minus the inclusive prefix
       const uint32_t h0 = hist[2 * tid], h1 = hist[2 * tid + 1];
@@ -231,66 +233,62 @@ __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __rest
       pmask |= dmask << shift;
       // the bin holding the k-th key is kept whole: every key above it and
       // every key in it are the top k, so the digits left decide nothing
-      whole = s_whole;
-      if (whole) break;
+      if (s_whole) break;
     }
   }
-  // T: the k-th largest key on the digits examined (pmask); `remaining` of the
-  // keys equal to T on those digits are kept (all of them after an early stop)
+  // T: the k-th largest key on the digits examined (pmask). Kept: every key
+  // above T, and the first `remaining` keys equal to T in index order (after
+  // k = 0 no pass ran: remaining = 0 and nothing is above T = 0 on no digits).
   const uint32_t T = prefix;
-  // ties before this thread, then this thread's kept count and output position
-  int n_gt = 0, n_eq = 0;
+  // per-warp counts of larger and equal keys, then one scan over the warps
+  unsigned w_gt = 0, w_eq = 0;
 #pragma unroll
   for (int j = 0; j < KPT; ++j) {
-    n_gt += (j < nt && k > 0 && (key[j] & pmask) > T);
-    n_eq += (j < nt && k > 0 && (key[j] & pmask) == T);
+    const bool v = (valid >> j) & 1u;
+    w_gt += __popc(__ballot_sync(0xffffffffu, v && (key[j] & pmask) > T));
+    w_eq += __popc(__ballot_sync(0xffffffffu, v && (key[j] & pmask) == T));
   }
-  // one scan of (n_gt, n_eq) packed in 16-bit halves (K <= 32768): the threads
-  // before this one keep all their larger keys and the first `remaining` of
-  // the ties, so this thread writes from gt_before + min(eq_before, remaining).
-  // Without an index list and with every tie kept, no offset is needed.
-  int eq_keep = n_eq, pos0 = 0, tot = k;
-  if (idx != nullptr || !whole) {
-    int packed_tot;
-    const int packed = block_excl_scan((n_gt << 16) | n_eq, s_w, &packed_tot);
-    const int gt_before = packed >> 16, eq_before = packed & 0xffff;
-    eq_keep = (int)remaining - eq_before;
-    eq_keep = eq_keep < 0 ? 0 : (eq_keep > n_eq ? n_eq : eq_keep);
-    pos0 = gt_before + (eq_before < (int)remaining ? eq_before : (int)remaining);
-    tot = (packed_tot >> 16) + ((packed_tot & 0xffff) < (int)remaining ? (packed_tot & 0xffff)
-                                                                       : (int)remaining);
+  if (lane == 0) s_w[warp] = (int)((w_gt << 16) | w_eq);  // both <= K <= 32768
+  __syncthreads();
+  if (warp == 0) {
+    const int wv = s_w[lane];
+    int winc = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, winc, o);
+      if (lane >= o) winc += n;
+    }
+    s_w[lane] = winc - wv;
+    if (lane == 31) s_w[32] = winc;
   }
+  __syncthreads();
+  // larger and equal keys at lower indices, running over the warp's slots
+  unsigned gt_run = (unsigned)s_w[warp] >> 16, eq_run = (unsigned)s_w[warp] & 0xffffu;
+  const unsigned all_gt = (unsigned)s_w[32] >> 16, all_eq = (unsigned)s_w[32] & 0xffffu;
   int32_t* out = idx ? idx + (long long)b * K : nullptr;
-  int pos = pos0, eq_seen = 0;
-  uint32_t word = 0;  // bits of the current bitmap word gathered by this thread
-  int word_id = e0 >> 5;
+  const int words = (K + 31) >> 5;
+  const unsigned lt = lanemask_lt();
 #pragma unroll
   for (int j = 0; j < KPT; ++j) {
-    if (j < nt) {
-      const int i = e0 + j;
-      bool keep = false;
-      if (k > 0) {
-        if ((key[j] & pmask) > T) {
-          keep = true;
-        } else if ((key[j] & pmask) == T) {
-          keep = eq_seen < eq_keep;
-          ++eq_seen;
-        }
+    const int e = base + 32 * j + lane;
+    if (j < kpt && base + 32 * j < K) {  // warp-uniform: the slot's word exists
+      const bool v = (valid >> j) & 1u;
+      const bool gt = v && (key[j] & pmask) > T, eq = v && (key[j] & pmask) == T;
+      const unsigned bg = __ballot_sync(0xffffffffu, gt);
+      const unsigned be = __ballot_sync(0xffffffffu, eq);
+      const unsigned eq_rank = eq_run + __popc(be & lt);
+      const bool keep = gt || (eq && eq_rank < remaining);
+      const unsigned bk = __ballot_sync(0xffffffffu, keep);
+      if (keep && out) {
+        const unsigned gt_rank = gt_run + __popc(bg & lt);
+        out[gt_rank + (eq_rank < remaining ? eq_rank : remaining)] = e;
       }
-      if (keep && out) out[pos++] = i;
-      if ((i >> 5) != word_id) {  // flush a finished word (shared with neighbours: OR)
-        if (word) atomicOr(&s_bits[word_id], word);
-        word = 0;
-        word_id = i >> 5;
-      }
-      if (keep) word |= 1u << (i & 31);
+      if (lane == 0 && bitmap) bitmap[(long long)b * words + ((base + 32 * j) >> 5)] = bk;
+      gt_run += __popc(bg);
+      eq_run += __popc(be);
     }
   }
-  if (word) atomicOr(&s_bits[word_id], word);
-  __syncthreads();
-  if (bitmap)
-    for (int w = tid; w < words; w += kMaskThreads) bitmap[(long long)b * words + w] = s_bits[w];
-  if (tid == 0) cnt[b] = tot;
+  if (tid == 0) cnt[b] = (int)(all_gt + (all_eq < remaining ? all_eq : remaining));
 }
 
 // q_j = #{i : key_i > key_j or (key_i == key_j and i < j)} by counting.
@@ -344,12 +342,11 @@ static int launch_threshold(const void* x, int B, int K, float t, uint32_t* bitm
 template <typename TX, int KPT>
 static int launch_gxo_k(const void* x, const float* g, int B, int K, int k, int corrected,
                         uint32_t* bitmap, int32_t* idx, int32_t* cnt, cudaStream_t s) {
-  const size_t smem = (size_t)((K + 31) / 32) * 4;  // the bitmap (<= 4 KB)
   // a programmatic dependent launch: the kernel waits for its inputs itself
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)B, 1, 1);
   cfg.blockDim = dim3(kMaskThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = 0;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -369,6 +366,9 @@ static int launch_gxo(const void* x, const float* g, int B, int K, int k, int co
   const int kpt = (K + kMaskThreads - 1) / kMaskThreads;
   if (kpt <= 4) return launch_gxo_k<TX, 4>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
   if (kpt <= 8) return launch_gxo_k<TX, 8>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
+  // 12 slots for n = 8193..12288 (10 keys per thread at n = 10240): every
+  // per-key loop is unrolled over the slots, so spare slots cost issue slots
+  if (kpt <= 12) return launch_gxo_k<TX, 12>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
   if (kpt <= 16) return launch_gxo_k<TX, 16>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
   return launch_gxo_k<TX, 32>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
 }
