@@ -444,8 +444,8 @@ def bench_other_workloads(stream, dev, which=OTHER_WORKLOADS):
             gl = sb.sfx_mask_compact(None, sb.SFX_SEL_TOPK_GLASS, k=k, score_l=sl, score_g=sgl, lam=0.5,
                                      ws=ws)
             us_gl = graph_us([lambda c=c: (sb.sfx_sparse_gemv(x, W1[c], flags=sb.SFX_FLAG_GELU, y=h, ws=ws),
-                                           sb.sfx_sparse_gemv(h[0], W2[c], idx=gl["idx"][0],
-                                                              cnt=gl["cnt"], y=y[0], ws=ws))
+                                           sb.sfx_sparse_gemv_mask(h[0], W2[c], gl["bitmap"][0],
+                                                                   y=y[0], ws=ws))
                               for c in range(n)], stream)
             # GLASS set on both projections: up rows and down rows of the kept neurons only
             us_both = graph_us([lambda c=c: sb.sfx_static_ffn(x, W1T[c], W2[c], gl["idx"][0],
