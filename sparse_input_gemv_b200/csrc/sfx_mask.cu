@@ -113,13 +113,14 @@ __device__ __forceinline__ int block_excl_scan(int v, int* s_w, int* total) {
 }
 
 // Exact top-k of s_i = |fl32(x_i * g_i)| (or the corrected GxO score) for one
-// token per CTA. Thread t owns the contiguous elements [t kpt, (t + 1) kpt),
-// kpt <= KPT, and keeps their keys in registers. Three radix passes over the
-// key bits (11, 11 and 10 bits, most significant first; wide digits keep the
-// histogram atomics spread even though the scores share their leading bits)
-// find the k-th largest key T and how many keys equal to T are kept; two block
-// scans then give every thread its ties' ranks and its output position, so the
-// list comes out ascending with ties resolved toward the lower index.
+// token per CTA. Warp w owns the 32 kpt elements from 32 kpt w on, in
+// lane-major slots (kpt <= KPT per thread, keys in registers). Up to three
+// radix passes over the key bits (11, 11 and 10 bits, most significant first;
+// wide digits keep the histogram atomics spread even though the scores share
+// their leading bits) find the k-th largest key T on the digits examined and
+// how many keys equal to it are kept, stopping early once that bin is kept
+// whole. Slot ballots and one scan over the warps then place every kept index,
+// so the list comes out ascending with ties resolved toward the lower index.
 constexpr int kTopkBins = 2048;  // 2 bins per thread
 template <typename TX, int KPT>
 __global__ void __launch_bounds__(kMaskThreads) topk_gxo_kernel(const TX* __restrict__ x,
