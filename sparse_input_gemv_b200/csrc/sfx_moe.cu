@@ -113,7 +113,12 @@ __global__ void __launch_bounds__(512) moe_route_kernel(const float* logits, int
   __shared__ unsigned s_tokmask[1024];  // tokens (B <= 16) that selected each expert
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nthr = blockDim.x, pairs = B * top_k;
-  pdl_launch_dependents();  // the expert grid waits for this grid's results where it needs them
+  // launched as a programmatic dependent: the previous kernel's results (the
+  // logits, x, this workspace's accumulator) are complete after the wait; only
+  // then may the expert grid start (its shared-expert items read x at once and
+  // wait for this grid's results where they need them)
+  pdl_wait();
+  pdl_launch_dependents();
 
   for (int i = tid; i < B * d; i += nthr) w.acc[i] = 0.f;
   if (tid == 0) *w.next_item = 0;
@@ -504,9 +509,21 @@ int run_moe(const void* x, int dt, const float* logits, int B, int d, int E, int
       return SFX_ERR_CUDA;
   }
   const int route_threads = 32 * (B > 4 ? B : 4);
-  moe_route_kernel<<<1, route_threads, route_smem, s>>>(logits, B, E, top_k, renorm, d, w,
-                                                        sel_out);
-  if (cudaGetLastError() != cudaSuccess) return SFX_ERR_CUDA;
+  {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(1, 1, 1);
+    cfg.blockDim = dim3((unsigned)route_threads, 1, 1);
+    cfg.dynamicSmemBytes = route_smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, moe_route_kernel, logits, B, E, top_k, renorm, d, w, sel_out) !=
+        cudaSuccess)
+      return SFX_ERR_CUDA;
+  }
   const int pairs = B * top_k;
   const int max_active = pairs < E ? pairs : E;
   const int ffn_s = Ws_gT ? ffn_shared : 0;
