@@ -11,7 +11,7 @@
 // neuron ([ffn x d]), so a neuron's gate, up and down weights are three
 // contiguous 2d-byte rows.
 //
-// Launches per call (the second and third with programmatic dependent launch):
+// Launches per call (all three programmatic dependent launches):
 //  1. moe_route_kernel (one CTA, one warp per token): softmax over E logits,
 //     top-k by probability (ties to the lower expert index), weights
 //     renormalised over the selection (or raw); the selected (token, slot)
