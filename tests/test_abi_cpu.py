@@ -111,6 +111,28 @@ def test_gemv_rejects_bad_arguments_before_launch(lib):
     assert _gemv(lib, ws_bytes=16) == -4
 
 
+def _gemv_mask(lib, x=0x1000, W=0x2000, mask=0x5000, y=0x3000, B=1, K=64, N=64,
+               wdt=sb.SFX_BF16, xdt=sb.SFX_BF16, ydt=sb.SFX_BF16, flags=0, ws=0x4000,
+               ws_bytes=1 << 20):
+    # fake (never dereferenced) pointers: every case below is rejected on the host
+    return lib.sfx_sparse_gemv_mask(x, xdt, B, K, W, wdt, N, mask, y, ydt, flags, ws, ws_bytes,
+                                    None)
+
+
+def test_gemv_on_a_mask_rejects_bad_arguments_before_launch(lib):
+    assert _gemv_mask(lib, mask=None) == -1
+    assert _gemv_mask(lib, x=None) == -1
+    assert _gemv_mask(lib, B=0) == -1
+    assert _gemv_mask(lib, B=17) == -1
+    assert _gemv_mask(lib, N=4) == -1
+    assert _gemv_mask(lib, flags=sb.SFX_FLAG_SWIGLU | sb.SFX_FLAG_GELU) == -1
+    assert _gemv_mask(lib, wdt=sb.SFX_F32) == -2
+    assert _gemv_mask(lib, flags=sb.SFX_FLAG_SWIGLU) == -2   # SwiGLU writes fp32 h
+    assert _gemv_mask(lib, W=0x2008) == -3                   # not 16-byte aligned
+    assert _gemv_mask(lib, N=68) == -3
+    assert _gemv_mask(lib, ws_bytes=16) == -4
+
+
 def test_other_entry_points_reject_bad_arguments(lib):
     VP = ctypes.c_void_p
     # calibration: P out of range, NaN sparsity
