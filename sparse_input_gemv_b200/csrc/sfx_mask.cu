@@ -367,8 +367,9 @@ static int launch_gxo(const void* x, const float* g, int B, int K, int k, int co
   const int kpt = (K + kMaskThreads - 1) / kMaskThreads;
   if (kpt <= 4) return launch_gxo_k<TX, 4>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
   if (kpt <= 8) return launch_gxo_k<TX, 8>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
-  // 12 slots for n = 8193..12288 (10 keys per thread at n = 10240): every
-  // per-key loop is unrolled over the slots, so spare slots cost issue slots
+  // every per-key loop is unrolled over the slots, so spare slots cost issue
+  // slots: 10 for n = 8193..10240 (10 keys per thread at n = 10240), 12 up to 12288
+  if (kpt <= 10) return launch_gxo_k<TX, 10>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
   if (kpt <= 12) return launch_gxo_k<TX, 12>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
   if (kpt <= 16) return launch_gxo_k<TX, 16>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
   return launch_gxo_k<TX, 32>(x, g, B, K, k, corrected, bitmap, idx, cnt, s);
