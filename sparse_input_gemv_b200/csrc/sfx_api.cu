@@ -252,11 +252,15 @@ int sfx_mask_compact(const void* x, int dt, int B, int K, int sel, float t, int 
                              reinterpret_cast<unsigned*>(ws), as_stream(stream));
 }
 
-int sfx_sparse_gemv(const void* x, int xdt, int B, int K, const void* W, int wdt, int N, float t,
-                    const int32_t* idx, const int32_t* cnt, void* y, int ydt, int flags,
-                    uint32_t* bitmap_out, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Checks shared by the two sparse GEMV entry points, then the launch arguments
+// every mode shares; the caller adds its mask source.
+int check_gemv(const void* x, int xdt, int B, int K, const void* W, int wdt, int N, void* y,
+               int ydt, int flags, void* ws, size_t ws_bytes) {
   if (!x || !W || !y || B < 1 || B > 16 || K < 1 || N < 8) return SFX_ERR_ARG;
-  if (idx && (!cnt || B != 1)) return SFX_ERR_ARG;
   if ((flags & SFX_FLAG_GELU) && (flags & SFX_FLAG_GELU_TANH)) return SFX_ERR_ARG;
   if ((flags & SFX_FLAG_SWIGLU) && (flags & (SFX_FLAG_GELU | SFX_FLAG_GELU_TANH))) return SFX_ERR_ARG;
   if (!(wdt == SFX_F16 || wdt == SFX_BF16) || !(xdt == wdt || xdt == SFX_F32) || !valid_dtype(ydt))
@@ -265,14 +269,15 @@ int sfx_sparse_gemv(const void* x, int xdt, int B, int K, const void* W, int wdt
   if (N % 8 != 0 || !aligned16(W)) return SFX_ERR_ALIGN;
   if (!ws || ws_bytes < sfx_workspace_bytes(SFX_OP_SPARSE_GEMV, B, K, N, xdt, 0, 0))
     return SFX_ERR_WORKSPACE;
-  const GemvPlan plan = plan_gemv(K, N, B, idx != nullptr);
+  return SFX_OK;
+}
+
+GemvArgs gemv_args(const void* x, int B, int K, const void* W, int N, void* y, int ydt,
+                   int flags, void* ws) {
   GemvArgs a = {};
   a.x = x;
   a.W = W;
   a.y = y;
-  a.idx = idx;
-  a.cnt = cnt;
-  a.bitmap_out = idx ? nullptr : bitmap_out;
   a.status = reinterpret_cast<unsigned*>(ws);
   carve_gemv(ws, reinterpret_cast<unsigned char*>(ws) + kWsHeader, a);
   a.K = K;
@@ -285,42 +290,38 @@ int sfx_sparse_gemv(const void* x, int xdt, int B, int K, const void* W, int wdt
                                        : EPI_NONE;
   a.union_mask = (flags & SFX_FLAG_UNION_MASK) ? 1 : 0;
   a.no_tc = (flags & SFX_FLAG_CUDA_CORES) ? 1 : 0;
-  a.t = t;
   a.wait_ns = wait_limit_ns();
-  return launch_sparse_gemv(wdt, xdt, plan, a, as_stream(stream), false);
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int sfx_sparse_gemv(const void* x, int xdt, int B, int K, const void* W, int wdt, int N, float t,
+                    const int32_t* idx, const int32_t* cnt, void* y, int ydt, int flags,
+                    uint32_t* bitmap_out, void* ws, size_t ws_bytes, void* stream) {
+  const int rc = check_gemv(x, xdt, B, K, W, wdt, N, y, ydt, flags, ws, ws_bytes);
+  if (rc != SFX_OK) return rc;
+  if (idx && (!cnt || B != 1)) return SFX_ERR_ARG;
+  GemvArgs a = gemv_args(x, B, K, W, N, y, ydt, flags, ws);
+  a.idx = idx;
+  a.cnt = cnt;
+  a.bitmap_out = idx ? nullptr : bitmap_out;
+  a.t = t;
+  return launch_sparse_gemv(wdt, xdt, plan_gemv(K, N, B, idx != nullptr), a, as_stream(stream),
+                            false);
 }
 
 int sfx_sparse_gemv_mask(const void* x, int xdt, int B, int K, const void* W, int wdt, int N,
                          const uint32_t* mask, void* y, int ydt, int flags, void* ws,
                          size_t ws_bytes, void* stream) {
-  if (!x || !W || !y || !mask || B < 1 || B > 16 || K < 1 || N < 8) return SFX_ERR_ARG;
-  if ((flags & SFX_FLAG_GELU) && (flags & SFX_FLAG_GELU_TANH)) return SFX_ERR_ARG;
-  if ((flags & SFX_FLAG_SWIGLU) && (flags & (SFX_FLAG_GELU | SFX_FLAG_GELU_TANH))) return SFX_ERR_ARG;
-  if (!(wdt == SFX_F16 || wdt == SFX_BF16) || !(xdt == wdt || xdt == SFX_F32) || !valid_dtype(ydt))
-    return SFX_ERR_DTYPE;
-  if ((flags & SFX_FLAG_SWIGLU) && ydt != SFX_F32) return SFX_ERR_DTYPE;
-  if (N % 8 != 0 || !aligned16(W)) return SFX_ERR_ALIGN;
-  if (!ws || ws_bytes < sfx_workspace_bytes(SFX_OP_SPARSE_GEMV, B, K, N, xdt, 0, 0))
-    return SFX_ERR_WORKSPACE;
-  GemvArgs a = {};
-  a.x = x;
-  a.W = W;
-  a.y = y;
+  if (!mask) return SFX_ERR_ARG;
+  const int rc = check_gemv(x, xdt, B, K, W, wdt, N, y, ydt, flags, ws, ws_bytes);
+  if (rc != SFX_OK) return rc;
+  GemvArgs a = gemv_args(x, B, K, W, N, y, ydt, flags, ws);
   a.mask_in = mask;
-  a.status = reinterpret_cast<unsigned*>(ws);
-  carve_gemv(ws, reinterpret_cast<unsigned char*>(ws) + kWsHeader, a);
-  a.K = K;
-  a.N = N;
-  a.B = B;
-  a.ydt = ydt;
-  a.epi = (flags & SFX_FLAG_SWIGLU) ? EPI_SWIGLU
-        : (flags & SFX_FLAG_GELU)   ? EPI_GELU
-        : (flags & SFX_FLAG_GELU_TANH) ? EPI_GELU_TANH
-                                       : EPI_NONE;
-  a.union_mask = (flags & SFX_FLAG_UNION_MASK) ? 1 : 0;
-  a.no_tc = 1;
-  a.t = 0.f;
-  a.wait_ns = wait_limit_ns();
+  a.no_tc = 1;  // the mask comes in: the CUDA-core kernel for every batch
   return launch_sparse_gemv(wdt, xdt, plan_gemv(K, N, B, false), a, as_stream(stream), false);
 }
 
