@@ -349,6 +349,53 @@ def test_gemv_given_mask_matches_oracle(B, K, N, dens, wdt, xdt, flags):
     assert_close(to64(y), O.round_to(want, "f32"), f"given mask B={B} K={K}")
 
 
+@pytest.mark.parametrize("xdt", ["bf16", "f32"])
+def test_gemv_misaligned_x_on_both_mask_paths(xdt):
+    # x one element past a 16-byte boundary (a view into a larger buffer): the
+    # compaction's vector loads fall back to element loads; the fused threshold
+    # and the given mask must still match the oracle
+    B, K, N = 1, 3000, 512
+    big = synth.eval_draw("misaligned", "x", 1, K + 1, xdt)
+    x = dev(big)[:, 1:]  # not 16-byte aligned, still row-contiguous
+    assert x.data_ptr() % 16 != 0
+    W = weights(K, N, "misaligned", "bf16")
+    t = 0.7
+    y_t = sb.sfx_sparse_gemv(x, dev(W), t=t, out_dtype=torch.float32)
+    m = O.magnitude_mask(to64(big[:, 1:]), t)
+    y_m = sb.sfx_sparse_gemv_mask(x, dev(W), dev(torch.from_numpy(pack_bitmap(m))),
+                                  out_dtype=torch.float32)
+    want = O.masked_gemv(to64(big[:, 1:]), m, to64(W))
+    assert_close(to64(y_t), O.round_to(want, "f32"), "threshold, misaligned x")
+    assert_close(to64(y_m), O.round_to(want, "f32"), "given mask, misaligned x")
+
+
+def test_topk_gxo_at_the_largest_batch():
+    # 64 tokens (the top-k's limit), one CTA each, every token its own k-th key
+    B, K, k = 64, 1500, 333
+    h = synth.normal((B, K), synth.seed_of("gxo-b64", "h"), 1.0, "f32")
+    g = synth.normal((B, K), synth.seed_of("gxo-b64", "g"), 1.0, "f32")
+    out = sb.sfx_mask_compact(dev(h), sb.SFX_SEL_TOPK_GXO, k=k, score_l=dev(g))
+    for b in range(B):
+        m = O.topk_mask(O.gxo_score(h.numpy()[b], g.numpy()[b]), k)
+        assert int(out["cnt"][b]) == k
+        assert np.array_equal(out["idx"][b, :k].cpu().numpy(), O.compact(m)[0]), b
+    assert np.array_equal(out["bitmap"].cpu().numpy(),
+                          pack_bitmap(np.stack([O.topk_mask(O.gxo_score(h.numpy()[b], g.numpy()[b]), k)
+                                                for b in range(B)])))
+
+
+def test_gemv_given_mask_at_the_largest_k():
+    # K = 49152 rows (beyond one CTA's list capacity at one split: the plan
+    # splits K), a sparse mask, fp32 x
+    B, K, N = 1, 49152, 256
+    x = synth.eval_draw("given-mask-bigk", "x", B, K, "f32")
+    W = weights(K, N, "given-mask-bigk", "bf16")
+    m = np.random.default_rng(9).random((B, K)) < 0.05
+    y = sb.sfx_sparse_gemv_mask(dev(x), dev(W), dev(torch.from_numpy(pack_bitmap(m))),
+                                out_dtype=torch.float32)
+    assert_close(to64(y), O.round_to(O.masked_gemv(to64(x), m, to64(W)), "f32"), "K = 49152")
+
+
 def test_gemv_given_mask_empty_and_full():
     B, K, N = 2, 3000, 256
     x = synth.eval_draw("given-mask-ef", "x", B, K, "bf16")
