@@ -55,8 +55,7 @@ def expert_thresholds(name, Wg64, experts, p, d, dtype):
     return te
 
 
-def run_case(name, B, E, d, ffn, top_k, ffn_s, p, flags=0, expert_subset=None):
-    dtype = "bf16"
+def run_case(name, B, E, d, ffn, top_k, ffn_s, p, flags=0, expert_subset=None, dtype="bf16"):
     Wg, WuT, Wd, sh = make_moe(name, E, d, ffn, ffn_s, dtype)
     x = synth.eval_draw(name, "x", B, d, dtype)
     logits = synth.normal((B, E), synth.seed_of(name, "logits", B), 1.0, "f32")
@@ -100,6 +99,12 @@ def run_case(name, B, E, d, ffn, top_k, ffn_s, p, flags=0, expert_subset=None):
 @pytest.mark.parametrize("B,p", [(1, 0.5), (3, 0.8), (16, 0.9), (2, 0.0)])
 def test_moe_small_ragged(B, p):
     run_case("moe-small", B, 16, 264, 72, 4, 136, p)
+
+
+@pytest.mark.parametrize("B,p", [(1, 0.5), (6, 0.7)])
+def test_moe_fp16_weights(B, p):
+    # the fp16 instantiation of the expert kernel (mma.sync f16 tiles)
+    run_case("moe-f16", B, 16, 256, 96, 4, 128, p, dtype="f16")
 
 
 def test_moe_without_shared_expert_and_raw_weights():
