@@ -840,6 +840,8 @@ PROFILE_CASES = {
     "ffn_down": "the headline down GEMV on the gate|up stage's h, batch 1",
     "ffn": "the headline SwiGLU FFN call, batch 1",
     "union_gate_up_b16": "the gate|up product of 16 tokens (batch-union kernels), same layer",
+    "union_down_b16": "the down product of 16 tokens on their fp32 h (batch-union kernels; the "
+                      "union keeps every row, so the dense kernel with the split x runs), same layer",
     "union_mma_gate_up_8b_b16": "a Llama-3-8B-shaped gate|up product (W 4096 x 28672) of 16 "
                                 "correlated tokens on the gathered-union mma.sync kernel",
     "union_tc_gate_up_8b_b16": "the same product on the tcgen05 union kernel (kept for comparison)",
@@ -917,7 +919,7 @@ def profile_other(name, p, dev, launches):
 def profile_case(name, p, dev, launches=6):
     """One kernel (or call) of a small case, `launches` times, then exit: the
     headline layer's, or another workload's. The ncu captures in profiles/ run this."""
-    if name not in ("ffn_gate_up", "ffn_down", "ffn", "union_gate_up_b16"):
+    if name not in ("ffn_gate_up", "ffn_down", "ffn", "union_gate_up_b16", "union_down_b16"):
         profile_other(name, p, dev, launches)
         print(json.dumps({"profile_case": name, "sparsity": p, "launches": launches,
                           "what": PROFILE_CASES[name]}), flush=True)
@@ -931,6 +933,9 @@ def profile_case(name, p, dev, launches=6):
     sb.sfx_sparse_gemv(x, stack.Wgu[0], t=t_in, flags=sb.SFX_FLAG_SWIGLU, y=h, ws=stack.ws)
     x16 = stack.draws("iid", 16)
     h16 = torch.empty((16, F70), dtype=torch.float32, device=dev)
+    y16 = torch.empty((16, D70), dtype=torch.bfloat16, device=dev)
+    if name == "union_down_b16":
+        sb.sfx_sparse_gemv(x16, stack.Wgu[0], t=t_in, flags=sb.SFX_FLAG_SWIGLU, y=h16, ws=stack.ws)
     for _ in range(launches):
         if name == "ffn_gate_up":
             sb.sfx_sparse_gemv(x, stack.Wgu[0], t=t_in, flags=sb.SFX_FLAG_SWIGLU, y=h, ws=stack.ws)
@@ -941,6 +946,8 @@ def profile_case(name, p, dev, launches=6):
         elif name == "union_gate_up_b16":
             sb.sfx_sparse_gemv(x16, stack.Wgu[0], t=t_in, flags=sb.SFX_FLAG_SWIGLU, y=h16,
                                ws=stack.ws)
+        elif name == "union_down_b16":
+            sb.sfx_sparse_gemv(h16, stack.Wd[0], t=t_h, y=y16, ws=stack.ws)
     torch.cuda.synchronize()
     print(json.dumps({"profile_case": name, "sparsity": p, "launches": launches,
                       "what": PROFILE_CASES[name]}), flush=True)
